@@ -1,0 +1,19 @@
+"""B200 (sm_100a) exact attention: fused forward with online softmax and a
+recompute-based backward, behind the C ABI of include/attn.h.
+
+    from exact_attention_156_b200 import attn_fwd, attn_bwd
+    o, lse = attn_fwd(q, k, v, causal=True)              # q, k, v: bf16 (B, S, H, D) CUDA
+    dq, dk, dv = attn_bwd(q, k, v, o, do, lse, causal=True)
+"""
+from ._binding import (  # noqa: F401
+    ATTN_STATUS,
+    LIB_PATH,
+    AttnError,
+    attn_bwd,
+    attn_bwd_workspace_size,
+    attn_fwd,
+    device_timeout_selftest,
+    get_last_device_error,
+    lib,
+    status_string,
+)

@@ -1,0 +1,163 @@
+"""ctypes binding of the C ABI in include/attn.h (argument marshalling only).
+
+Every step of attention runs in the CUDA kernels of ``libattn156.so``; this
+module only turns torch tensors into pointers, sizes and the current stream,
+and turns status codes into exceptions.  There is no CPU path: if the library
+is missing the import fails.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from typing import Optional, Tuple
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libattn156.so")
+
+ATTN_STATUS = {
+    0: "ATTN_OK", 1: "ATTN_ERR_NULLPTR", 2: "ATTN_ERR_SHAPE", 3: "ATTN_ERR_HEADDIM",
+    4: "ATTN_ERR_ALIGN", 5: "ATTN_ERR_WINDOW", 6: "ATTN_ERR_ARCH", 7: "ATTN_ERR_DEVICE",
+    8: "ATTN_ERR_LAUNCH", 9: "ATTN_ERR_TIMEOUT", 10: "ATTN_ERR_WORKSPACE",
+}
+
+
+class AttnError(RuntimeError):
+    def __init__(self, status: int, func: str):
+        self.status = status
+        self.name = ATTN_STATUS.get(status, str(status))
+        super().__init__(f"{func}: {self.name}: {status_string(status)}")
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"{LIB_PATH} is missing: build it with `python -m exact_attention_156_b200.build` "
+            "(there is no CPU fallback)")
+    lib = ctypes.CDLL(LIB_PATH)
+    vp, i, f, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+    lib.attn_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, i, i, i, vp]
+    lib.attn_fwd.restype = i
+    lib.attn_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, i, i,
+                             vp, sz, vp]
+    lib.attn_bwd.restype = i
+    lib.attn_bwd_workspace_size.argtypes = [i, i, i, i]
+    lib.attn_bwd_workspace_size.restype = sz
+    lib.attn_status_string.argtypes = [i]
+    lib.attn_status_string.restype = ctypes.c_char_p
+    lib.attn_get_last_device_error.argtypes = []
+    lib.attn_get_last_device_error.restype = i
+    lib.attn_device_timeout_selftest.argtypes = [i, vp]
+    lib.attn_device_timeout_selftest.restype = i
+    return lib
+
+
+lib = _load()
+
+
+def status_string(status: int) -> str:
+    return lib.attn_status_string(int(status)).decode()
+
+
+def _stream_handle(stream, device) -> int:
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    return int(stream.cuda_stream)
+
+
+def _check(t, name, dtype, ndim):
+    import torch
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor (no CPU path exists)")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dimensions, got {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous (batch, seqlen, nheads, head_dim)")
+
+
+def _scale(softmax_scale, D):
+    return float(1.0 / math.sqrt(D)) if softmax_scale is None else float(softmax_scale)
+
+
+def _window(causal, window_size):
+    wl, wr = (-1, -1) if window_size is None else (int(window_size[0]), int(window_size[1]))
+    return (1 if causal else 0), wl, wr
+
+
+def attn_fwd(q, k, v, softmax_scale: Optional[float] = None, causal: bool = False,
+             window_size: Optional[Tuple[int, int]] = None, out=None, lse=None,
+             stream=None):
+    """O, LSE = exact attention of q (B,Sq,H,D), k, v (B,Sk,H,D), all bf16 CUDA.
+
+    ``softmax_scale=None`` means 1/sqrt(D).  ``window_size=(left, right)`` with
+    -1 for an unbounded side.  Returns (o bf16 (B,Sq,H,D), lse fp32 (B,H,Sq)).
+    """
+    import torch
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _check(t, n, torch.bfloat16, 4)
+    B, Sq, H, D = q.shape
+    Sk = k.shape[1]
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, H, Sq), dtype=torch.float32, device=q.device)
+    _check(out, "out", torch.bfloat16, 4)
+    _check(lse, "lse", torch.float32, 3)
+    c, wl, wr = _window(causal, window_size)
+    st = lib.attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                      B, Sq, Sk, H, D, _scale(softmax_scale, D), c, wl, wr,
+                      _stream_handle(stream, q.device))
+    if st != 0:
+        raise AttnError(st, "attn_fwd")
+    return out, lse
+
+
+def attn_bwd_workspace_size(B: int, Sq: int, H: int, D: int) -> int:
+    return int(lib.attn_bwd_workspace_size(B, Sq, H, D))
+
+
+def attn_bwd(q, k, v, out, dout, lse, softmax_scale: Optional[float] = None,
+             causal: bool = False, window_size: Optional[Tuple[int, int]] = None,
+             dq=None, dk=None, dv=None, workspace=None, stream=None):
+    """dQ, dK, dV of exact attention given the forward's O and LSE and dO.
+
+    ``workspace`` (a uint8 CUDA tensor of at least attn_bwd_workspace_size
+    bytes) is allocated by torch when not given.  Returns (dq, dk, dv) bf16.
+    """
+    import torch
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (out, "out"), (dout, "dout")):
+        _check(t, n, torch.bfloat16, 4)
+    _check(lse, "lse", torch.float32, 3)
+    B, Sq, H, D = q.shape
+    Sk = k.shape[1]
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    need = attn_bwd_workspace_size(B, Sq, H, D)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    c, wl, wr = _window(causal, window_size)
+    st = lib.attn_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), dout.data_ptr(),
+                      lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
+                      B, Sq, Sk, H, D, _scale(softmax_scale, D), c, wl, wr,
+                      workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                      _stream_handle(stream, q.device))
+    if st != 0:
+        raise AttnError(st, "attn_bwd")
+    return dq, dk, dv
+
+
+def get_last_device_error() -> int:
+    """Synchronises the device; returns the status a timed-out wait recorded (0 if none)."""
+    return int(lib.attn_get_last_device_error())
+
+
+def device_timeout_selftest(limit_us: int, stream=None) -> int:
+    import torch
+    dev = torch.device("cuda", torch.cuda.current_device())
+    return int(lib.attn_device_timeout_selftest(int(limit_us), _stream_handle(stream, dev)))

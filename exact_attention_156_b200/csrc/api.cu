@@ -1,0 +1,332 @@
+// api.cu - the C ABI declared in include/attn.h: argument validation, launch
+// planning (tile shapes per head_dim, grids), TMA descriptor encoding and
+// kernel launches.  Nothing here computes attention; every step of the path
+// runs in the kernels of fwd_sm100.cuh and bwd_sm100.cuh.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <math.h>
+#include <mutex>
+#include <stdint.h>
+#include <string.h>
+
+#include "../../include/attn.h"
+#include "bwd_sm100.cuh"
+#include "fwd_sm100.cuh"
+
+using namespace attn156;
+
+namespace {
+
+// Device error word written by timed-out waits (and by the alignment guard).
+__device__ uint32_t g_attn_err = 0;
+
+constexpr uint64_t kTimeoutNs = 1000000000ull;  // 1 s per device-side wait
+constexpr int kMaxDevices = 64;
+
+struct DeviceState {
+  bool init = false;
+  bool arch_ok = false;
+  uint32_t* err = nullptr;
+  int num_sms = 0;
+};
+DeviceState g_dev[kMaxDevices];
+std::mutex g_mu;
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn g_encode = nullptr;
+
+template <typename K>
+cudaError_t set_smem(K kernel, int bytes) {
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+}
+
+// One-time per-device set-up: architecture check, error-word address, kernel attributes.
+attn_status device_state(DeviceState** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return ATTN_ERR_DEVICE;
+  if (dev < 0 || dev >= kMaxDevices) return ATTN_ERR_DEVICE;
+  std::lock_guard<std::mutex> lock(g_mu);
+  DeviceState& s = g_dev[dev];
+  if (!s.init) {
+    int major = 0, minor = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+      return ATTN_ERR_DEVICE;
+    cudaDeviceGetAttribute(&s.num_sms, cudaDevAttrMultiProcessorCount, dev);
+    s.arch_ok = (major == 10 && minor == 0);
+    if (s.arch_ok) {
+      if (cudaGetSymbolAddress(reinterpret_cast<void**>(&s.err), g_attn_err) != cudaSuccess)
+        return ATTN_ERR_LAUNCH;
+      if (set_smem(fwd::attn_fwd_kernel<64>, fwd::Cfg<64>::kSmemBytes) != cudaSuccess ||
+          set_smem(fwd::attn_fwd_kernel<128>, fwd::Cfg<128>::kSmemBytes) != cudaSuccess ||
+          set_smem(bwd::attn_bwd_main_kernel<64>, bwd::Cfg<64>::kSmemBytes) != cudaSuccess ||
+          set_smem(bwd::attn_bwd_main_kernel<128>, bwd::Cfg<128>::kSmemBytes) != cudaSuccess)
+        return ATTN_ERR_LAUNCH;
+      if (g_encode == nullptr) {
+        void* fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) !=
+                cudaSuccess ||
+            q != cudaDriverEntryPointSuccess || fn == nullptr)
+          return ATTN_ERR_LAUNCH;
+        g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+      }
+    }
+    s.init = true;
+  }
+  if (!s.arch_ok) return ATTN_ERR_ARCH;
+  *out = &s;
+  return ATTN_OK;
+}
+
+// A pointer must be device (or managed) memory visible from the current device.
+bool on_current_device(const void* p) {
+  cudaPointerAttributes a;
+  if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  int dev = -1;
+  cudaGetDevice(&dev);
+  if (a.type == cudaMemoryTypeDevice) return a.device == dev;
+  if (a.type == cudaMemoryTypeManaged) return true;
+  return false;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+attn_status check_common(int B, int Sq, int Sk, int H, int D, float scale, int win_left,
+                         int win_right) {
+  if (B < 1 || Sq < 1 || Sk < 1 || H < 1) return ATTN_ERR_SHAPE;
+  if (B > 65535 || H > 65535) return ATTN_ERR_SHAPE;
+  if (D != 64 && D != 128) return ATTN_ERR_HEADDIM;
+  const long long row = (long long)H * D;
+  if ((long long)B * Sq * row >= (1ll << 31) || (long long)B * Sk * row >= (1ll << 31))
+    return ATTN_ERR_SHAPE;
+  if (!(scale > 0.f) || !isfinite(scale)) return ATTN_ERR_SHAPE;
+  if (win_left < -1 || win_right < -1) return ATTN_ERR_WINDOW;
+  return ATTN_OK;
+}
+
+// 4-D bf16 map over a (B, S, H, D) tensor, box = 64 x 1 x 128 x 1, 128-byte swizzle.
+attn_status make_map(CUtensorMap* map, const void* base, int B, int S, int H, int D) {
+  const cuuint64_t dims[4] = {cuuint64_t(D), cuuint64_t(H), cuuint64_t(S), cuuint64_t(B)};
+  const cuuint64_t strides[3] = {cuuint64_t(D) * 2, cuuint64_t(H) * D * 2,
+                                 cuuint64_t(S) * H * D * 2};
+  const cuuint32_t box[4] = {64, 1, 128, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  const CUresult r =
+      g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides,
+               box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? ATTN_OK : ATTN_ERR_LAUNCH;
+}
+
+int sq_pad(int Sq) { return ((Sq + 127) / 128) * 128; }
+
+size_t workspace_bytes(int B, int Sq, int H, int D) {
+  const size_t rows = size_t(B) * H * sq_pad(Sq);
+  return rows * D * 4 + rows * 4 * 2;
+}
+
+template <int D>
+attn_status launch_fwd(const DeviceState& st, const void* q, const void* k, const void* v, void* o,
+                       float* lse, int B, int Sq, int Sk, int H, float scale, int causal,
+                       int win_left, int win_right, cudaStream_t stream) {
+  alignas(64) CUtensorMap mq, mk, mv;
+  if (make_map(&mq, q, B, Sq, H, D) != ATTN_OK || make_map(&mk, k, B, Sk, H, D) != ATTN_OK ||
+      make_map(&mv, v, B, Sk, H, D) != ATTN_OK)
+    return ATTN_ERR_LAUNCH;
+  fwd::Params p;
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  p.B = B;
+  p.H = H;
+  p.Sq = Sq;
+  p.Sk = Sk;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.causal = causal ? 1 : 0;
+  p.win_left = win_left;
+  p.win_right = win_right;
+  p.num_mblocks = (Sq + fwd::NQ * fwd::BM - 1) / (fwd::NQ * fwd::BM);
+  p.err = st.err;
+  p.timeout_ns = kTimeoutNs;
+  dim3 grid(p.num_mblocks, H, B);
+  fwd::attn_fwd_kernel<D><<<grid, fwd::kThreads, fwd::Cfg<D>::kSmemBytes, stream>>>(mq, mk, mv, p);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_LAUNCH;
+}
+
+template <int D>
+attn_status launch_bwd(const DeviceState& st, const void* q, const void* k, const void* v,
+                       const void* o, const void* dout, const float* lse, void* dq, void* dk,
+                       void* dv, int B, int Sq, int Sk, int H, float scale, int causal,
+                       int win_left, int win_right, void* workspace, cudaStream_t stream) {
+  const int Sqp = sq_pad(Sq);
+  const size_t rows = size_t(B) * H * Sqp;
+  float* dq_acc = static_cast<float*>(workspace);
+  float* lse2 = dq_acc + rows * D;
+  float* delta = lse2 + rows;
+
+  {
+    const long long warps = (long long)rows;
+    const unsigned blocks = unsigned((warps + 7) / 8);
+    bwd::attn_bwd_pre_kernel<D><<<blocks, 256, 0, stream>>>(
+        static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout), lse, lse2,
+        delta, dq_acc, B, H, Sq, Sqp);
+    if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_LAUNCH;
+  }
+  {
+    alignas(64) CUtensorMap mq, mk, mv, mdo;
+    if (make_map(&mq, q, B, Sq, H, D) != ATTN_OK || make_map(&mk, k, B, Sk, H, D) != ATTN_OK ||
+        make_map(&mv, v, B, Sk, H, D) != ATTN_OK || make_map(&mdo, dout, B, Sq, H, D) != ATTN_OK)
+      return ATTN_ERR_LAUNCH;
+    bwd::Params p;
+    p.dk = static_cast<__nv_bfloat16*>(dk);
+    p.dv = static_cast<__nv_bfloat16*>(dv);
+    p.lse2 = lse2;
+    p.delta = delta;
+    p.dq_acc = dq_acc;
+    p.B = B;
+    p.H = H;
+    p.Sq = Sq;
+    p.Sk = Sk;
+    p.Sq_pad = Sqp;
+    p.scale = scale;
+    p.scale_log2 = scale * 1.4426950408889634f;
+    p.causal = causal ? 1 : 0;
+    p.win_left = win_left;
+    p.win_right = win_right;
+    p.err = st.err;
+    p.timeout_ns = kTimeoutNs;
+    dim3 grid((Sk + bwd::BN - 1) / bwd::BN, H, B);
+    bwd::attn_bwd_main_kernel<D>
+        <<<grid, bwd::kThreads, bwd::Cfg<D>::kSmemBytes, stream>>>(mq, mk, mv, mdo, p);
+    if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_LAUNCH;
+  }
+  {
+    const long long total = (long long)B * Sq * H * (D / 8);
+    const unsigned blocks = unsigned((total + 255) / 256);
+    bwd::attn_bwd_dq_kernel<D><<<blocks, 256, 0, stream>>>(
+        dq_acc, static_cast<__nv_bfloat16*>(dq), B, H, Sq, Sqp, scale);
+    if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_LAUNCH;
+  }
+  return ATTN_OK;
+}
+
+__global__ void attn_timeout_selftest_kernel(uint32_t* err, uint64_t limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bar), 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  Bounded bw{&abort_flag, err, limit_ns};
+  // Nothing ever arrives on `bar`, so this wait runs out after limit_ns.
+  bw.wait(smem_u32(&bar), 0, 99);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* attn_status_string(attn_status s) {
+  switch (s) {
+    case ATTN_OK: return "ok";
+    case ATTN_ERR_NULLPTR: return "a required pointer is NULL";
+    case ATTN_ERR_SHAPE: return "bad shape or scale (B, H, Sq, Sk >= 1, sizes < 2^31, scale finite > 0)";
+    case ATTN_ERR_HEADDIM: return "head_dim must be 64 or 128";
+    case ATTN_ERR_ALIGN: return "tensor pointers must be 16-byte aligned";
+    case ATTN_ERR_WINDOW: return "window sizes must be -1 (unbounded) or >= 0";
+    case ATTN_ERR_ARCH: return "the current device is not compute capability 10.0 (sm_100a)";
+    case ATTN_ERR_DEVICE: return "a pointer is not device memory of the current GPU";
+    case ATTN_ERR_LAUNCH: return "a CUDA call failed (descriptor encoding or kernel launch)";
+    case ATTN_ERR_TIMEOUT: return "a device-side bounded wait ran out";
+    case ATTN_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+  }
+  return "unknown status";
+}
+
+attn_status attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                     int Sq, int Sk, int H, int D, float scale, int causal, int win_left,
+                     int win_right, void* stream) {
+  if (!q || !k || !v || !o || !lse) return ATTN_ERR_NULLPTR;
+  attn_status s = check_common(B, Sq, Sk, H, D, scale, win_left, win_right);
+  if (s != ATTN_OK) return s;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) ||
+      (reinterpret_cast<uintptr_t>(lse) & 3u))
+    return ATTN_ERR_ALIGN;
+  DeviceState* st = nullptr;
+  s = device_state(&st);
+  if (s != ATTN_OK) return s;
+  if (!on_current_device(q) || !on_current_device(k) || !on_current_device(v) ||
+      !on_current_device(o) || !on_current_device(lse))
+    return ATTN_ERR_DEVICE;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  if (D == 64)
+    return launch_fwd<64>(*st, q, k, v, o, lse, B, Sq, Sk, H, scale, causal, win_left, win_right, cs);
+  return launch_fwd<128>(*st, q, k, v, o, lse, B, Sq, Sk, H, scale, causal, win_left, win_right, cs);
+}
+
+size_t attn_bwd_workspace_size(int B, int Sq, int H, int D) {
+  if (B < 1 || Sq < 1 || H < 1 || (D != 64 && D != 128)) return 0;
+  return workspace_bytes(B, Sq, H, D);
+}
+
+attn_status attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                     const float* lse, void* dq, void* dk, void* dv, int B, int Sq, int Sk, int H,
+                     int D, float scale, int causal, int win_left, int win_right, void* workspace,
+                     size_t workspace_size, void* stream) {
+  if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv) return ATTN_ERR_NULLPTR;
+  attn_status s = check_common(B, Sq, Sk, H, D, scale, win_left, win_right);
+  if (s != ATTN_OK) return s;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) ||
+      !aligned16(dq) || !aligned16(dk) || !aligned16(dv) ||
+      (reinterpret_cast<uintptr_t>(lse) & 3u))
+    return ATTN_ERR_ALIGN;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) ||
+      workspace_size < workspace_bytes(B, Sq, H, D))
+    return ATTN_ERR_WORKSPACE;
+  DeviceState* st = nullptr;
+  s = device_state(&st);
+  if (s != ATTN_OK) return s;
+  const void* ptrs[] = {q, k, v, o, dout, lse, dq, dk, dv, workspace};
+  for (const void* ptr : ptrs)
+    if (!on_current_device(ptr)) return ATTN_ERR_DEVICE;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  if (D == 64)
+    return launch_bwd<64>(*st, q, k, v, o, dout, lse, dq, dk, dv, B, Sq, Sk, H, scale, causal,
+                          win_left, win_right, workspace, cs);
+  return launch_bwd<128>(*st, q, k, v, o, dout, lse, dq, dk, dv, B, Sq, Sk, H, scale, causal,
+                         win_left, win_right, workspace, cs);
+}
+
+attn_status attn_get_last_device_error(void) {
+  DeviceState* st = nullptr;
+  attn_status s = device_state(&st);
+  if (s != ATTN_OK) return s;
+  if (cudaDeviceSynchronize() != cudaSuccess) return ATTN_ERR_LAUNCH;
+  uint32_t word = 0;
+  if (cudaMemcpyFromSymbol(&word, g_attn_err, sizeof(word)) != cudaSuccess) return ATTN_ERR_LAUNCH;
+  if (word == 0) return ATTN_OK;
+  const uint32_t zero = 0;
+  cudaMemcpyToSymbol(g_attn_err, &zero, sizeof(zero));
+  return (word & 0xFFu) == kErrTimeout ? ATTN_ERR_TIMEOUT : ATTN_ERR_LAUNCH;
+}
+
+attn_status attn_device_timeout_selftest(int limit_us, void* stream) {
+  if (limit_us < 1 || limit_us > 1000000) return ATTN_ERR_SHAPE;
+  DeviceState* st = nullptr;
+  attn_status s = device_state(&st);
+  if (s != ATTN_OK) return s;
+  attn_timeout_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
+      st->err, uint64_t(limit_us) * 1000ull);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_LAUNCH;
+}
+
+}  // extern "C"

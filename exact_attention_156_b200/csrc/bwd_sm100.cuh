@@ -1,0 +1,519 @@
+// bwd_sm100.cuh - recompute-based exact-attention backward for B200 (sm_100a).
+//
+// Method: the backward rebuilds the attention probabilities from Q, K and the
+// forward's per-row log-sum-exp instead of storing them (flash-attn install
+// guide, yfxerp.com, section 1: "the backward recomputes the attention
+// scores"; FlashAttention-2 overview, lshu.cn, section 2.1, second anti-pattern:
+// the standard backward re-reads Q, K, V several times).  The gradient is the
+// analytic one of O = softmax(scale Q K^T) V:
+//   P = exp(scale S - LSE), dV = P^T dO, dP = dO V^T, Delta_i = rowsum(dO*O),
+//   dS = P * (dP - Delta), dK = scale dS^T Q, dQ = scale dS K.
+//
+// Kernels:
+//  1. bwd_pre: Delta_i (fp32), LSE in base 2 (padded rows: +inf so P = 0),
+//     and zeroes the fp32 dQ accumulator.  Memory bound.
+//  2. bwd_main: one CTA per (128-key tile, head, batch); K_j and V_j stay in
+//     shared memory while the CTA streams the query tiles that can see them.
+//     Transposed products put the key index on tensor-memory lanes:
+//       S^T = K Q^T  and  dP^T = V dO^T   (M = keys, N = queries, K = D)
+//       dV += P^T dO  (A = P^T from tensor memory)
+//       dK += dS^T Q  (A = dS^T from shared memory, K-major)
+//       dQ_tile = dS K (A = the same dS^T buffer read MN-major) -> fp32 atomics
+//     warps 0-3: P and dS (one thread = one key row); warps 4-7: drain dQ
+//     from tensor memory into the fp32 accumulator with vector reductions;
+//     warp 8: MMA issue; warp 9: TMA / bulk loads.
+//  3. bwd_dq_finalize: dQ = bf16(scale * accumulator).
+// Tensor memory (512 columns): dK [0,D) dV [D,2D) S^T/P^T [2D,2D+128)
+// dP^T / dQ [2D+128, 2D+256).
+#pragma once
+
+#include <cuda.h>
+#include <math.h>
+
+#include "common.cuh"
+#include "ptx.cuh"
+
+namespace attn156 {
+namespace bwd {
+
+constexpr int BM = 128;  // query rows per tile
+constexpr int BN = 128;  // key rows per CTA
+constexpr int kThreads = 320;
+constexpr int kDrainWarp0 = 4;
+constexpr int kMmaWarp = 8;
+constexpr int kLoadWarp = 9;
+constexpr int kStages = 2;
+
+template <int D>
+struct Cfg {
+  static constexpr int kBoxBytes = 128 * 128;
+  static constexpr int kBoxes = D / 64;
+  static constexpr int kTileBytes = 128 * D * 2;
+  static constexpr int kKOff = 0;
+  static constexpr int kVOff = kKOff + kTileBytes;
+  static constexpr int kQOff = kVOff + kTileBytes;
+  static constexpr int kDOOff = kQOff + kStages * kTileBytes;
+  static constexpr int kDSOff = kDOOff + kStages * kTileBytes;  // dS^T, 128 x 128 bf16
+  static constexpr int kLseOff = kDSOff + BN * BM * 2;          // [kStages][BM] fp32
+  static constexpr int kDeltaOff = kLseOff + kStages * BM * 4;  // [kStages][BM] fp32
+  static constexpr int kBarOff = kDeltaOff + kStages * BM * 4;
+  static constexpr int kBarKV = 0;
+  static constexpr int kBarFull = 1;
+  static constexpr int kBarEmpty = kBarFull + kStages;
+  static constexpr int kBarS = kBarEmpty + kStages;
+  static constexpr int kBarDP = kBarS + 1;
+  static constexpr int kBarP = kBarDP + 1;
+  static constexpr int kBarDS = kBarP + 1;
+  static constexpr int kBarDSEmpty = kBarDS + 1;
+  static constexpr int kBarDQFull = kBarDSEmpty + 1;
+  static constexpr int kBarDQEmpty = kBarDQFull + 1;
+  static constexpr int kBarDone = kBarDQEmpty + 1;
+  static constexpr int kNumBars = kBarDone + 1;
+  static constexpr int kMiscOff = kBarOff + kNumBars * 8;
+  static constexpr int kSmemBytes = kMiscOff + 16;
+  static constexpr uint32_t kColDK = 0;
+  static constexpr uint32_t kColDV = D;
+  static constexpr uint32_t kColS = 2 * D;
+  static constexpr uint32_t kColDP = 2 * D + 128;
+};
+
+struct Params {
+  __nv_bfloat16* dk;
+  __nv_bfloat16* dv;
+  const float* lse2;   // [B*H][Sq_pad] LSE * log2(e); +inf for padding rows
+  const float* delta;  // [B*H][Sq_pad]
+  float* dq_acc;       // [B*H][Sq_pad][D]
+  int B, H, Sq, Sk, Sq_pad;
+  float scale;
+  float scale_log2;
+  int causal, win_left, win_right;
+  uint32_t* err;
+  uint64_t timeout_ns;
+};
+
+// ---------------------------------------------------------------------------
+// 1. preprocess: one warp per (b, h, row of the padded query axis)
+// ---------------------------------------------------------------------------
+template <int D>
+__global__ void __launch_bounds__(256) attn_bwd_pre_kernel(
+    const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* __restrict__ dout,
+    const float* __restrict__ lse, float* __restrict__ lse2, float* __restrict__ delta,
+    float* __restrict__ dq_acc, int B, int H, int Sq, int Sq_pad) {
+  const long long gw = (long long)blockIdx.x * 8 + threadIdx.x / 32;
+  const int lane = threadIdx.x % 32;
+  const long long rows = (long long)B * H * Sq_pad;
+  if (gw >= rows) return;
+  const int i = int(gw % Sq_pad);
+  const long long bh = gw / Sq_pad;
+  const int h = int(bh % H);
+  const int b = int(bh / H);
+  float dot = 0.f;
+  if (i < Sq) {
+    const size_t base = ((size_t(b) * Sq + i) * H + h) * D;
+    constexpr int kPer = D / 32;  // bf16 elements per lane (2 or 4)
+    if constexpr (kPer == 4) {
+      const uint2 ov = *reinterpret_cast<const uint2*>(o + base + lane * 4);
+      const uint2 dv = *reinterpret_cast<const uint2*>(dout + base + lane * 4);
+      const __nv_bfloat162* o2 = reinterpret_cast<const __nv_bfloat162*>(&ov);
+      const __nv_bfloat162* d2 = reinterpret_cast<const __nv_bfloat162*>(&dv);
+#pragma unroll
+      for (int t = 0; t < 2; ++t) {
+        const float2 a = __bfloat1622float2(o2[t]);
+        const float2 c = __bfloat1622float2(d2[t]);
+        dot = fmaf(a.x, c.x, dot);
+        dot = fmaf(a.y, c.y, dot);
+      }
+    } else {
+      const __nv_bfloat162 ov = *reinterpret_cast<const __nv_bfloat162*>(o + base + lane * 2);
+      const __nv_bfloat162 dv = *reinterpret_cast<const __nv_bfloat162*>(dout + base + lane * 2);
+      const float2 a = __bfloat1622float2(ov);
+      const float2 c = __bfloat1622float2(dv);
+      dot = fmaf(a.x, c.x, dot);
+      dot = fmaf(a.y, c.y, dot);
+    }
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, off);
+  if (lane == 0) {
+    const size_t r = size_t(bh) * Sq_pad + i;
+    float l2 = INFINITY;  // padding rows and rows that see no key: P = 0
+    if (i < Sq) {
+      const float l = lse[size_t(bh) * Sq + i];
+      if (l != -INFINITY) l2 = l * 1.4426950408889634f;
+    }
+    lse2[r] = l2;
+    delta[r] = dot;
+  }
+  float4* acc = reinterpret_cast<float4*>(dq_acc + (size_t(bh) * Sq_pad + i) * D);
+  for (int c = lane; c < D / 4; c += 32) acc[c] = make_float4(0.f, 0.f, 0.f, 0.f);
+}
+
+// ---------------------------------------------------------------------------
+// 3. dQ finalize: dq[b, i, h, :] = bf16(scale * acc[b, h, i, :]); 8 elements per thread
+// ---------------------------------------------------------------------------
+template <int D>
+__global__ void __launch_bounds__(256) attn_bwd_dq_kernel(const float* __restrict__ dq_acc,
+                                                          __nv_bfloat16* __restrict__ dq, int B,
+                                                          int H, int Sq, int Sq_pad, float scale) {
+  const long long t = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  constexpr int kVec = D / 8;
+  const long long total = (long long)B * Sq * H * kVec;
+  if (t >= total) return;
+  const int v = int(t % kVec);
+  long long r = t / kVec;  // (b, i, h) in BSHD order
+  const int h = int(r % H);
+  r /= H;
+  const int i = int(r % Sq);
+  const int b = int(r / Sq);
+  const float4* src =
+      reinterpret_cast<const float4*>(dq_acc + ((size_t(b) * H + h) * Sq_pad + i) * D + v * 8);
+  const float4 a = src[0];
+  const float4 c = src[1];
+  uint4 w;
+  w.x = pack_bf16x2(a.x * scale, a.y * scale);
+  w.y = pack_bf16x2(a.z * scale, a.w * scale);
+  w.z = pack_bf16x2(c.x * scale, c.y * scale);
+  w.w = pack_bf16x2(c.z * scale, c.w * scale);
+  *reinterpret_cast<uint4*>(dq + ((size_t(b) * Sq + i) * H + h) * D + v * 8) = w;
+}
+
+// ---------------------------------------------------------------------------
+// 2. main backward kernel
+// ---------------------------------------------------------------------------
+// Query-tile range [qlo, qhi) that can see keys [n0, n1]; empty if qhi <= qlo.
+__device__ __forceinline__ void qtile_range(const MaskGeom& g, int n0, int n1, int& qlo, int& qhi) {
+  const int a = max(0, g.qmin(n0));
+  const int z = min(g.Sq - 1, g.qmax(n1));
+  if (n0 >= g.Sk || z < a) {
+    qlo = 0;
+    qhi = 0;
+    return;
+  }
+  qlo = a / BM;
+  qhi = z / BM + 1;
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ,
+                         const __grid_constant__ CUtensorMap tmK,
+                         const __grid_constant__ CUtensorMap tmV,
+                         const __grid_constant__ CUtensorMap tmDO, const Params p) {
+  using C = Cfg<D>;
+  extern __shared__ __align__(1024) uint8_t smem[];
+  const int warp = threadIdx.x / 32;
+  const int lane = threadIdx.x % 32;
+  const uint32_t sbase = smem_u32(smem);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kBarOff);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kMiscOff);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kMiscOff + 4);
+  auto bar = [&](int idx) { return smem_u32(&bars[idx]); };
+  if ((sbase & 1023u) != 0) {
+    if (threadIdx.x == 0) atomicCAS(p.err, 0u, 8u);
+    return;
+  }
+
+  const int kt = blockIdx.x;  // key tile; low indices see the most query tiles when causal
+  const int h = blockIdx.y;
+  const int b = blockIdx.z;
+  const int bh = b * p.H + h;
+  const MaskGeom g = MaskGeom::make(p.Sq, p.Sk, p.causal, p.win_left, p.win_right);
+  const int n0 = kt * BN;
+  const int n1 = min(n0 + BN - 1, p.Sk - 1);
+  int qlo, qhi;
+  qtile_range(g, n0, n1, qlo, qhi);
+  const int nq = qhi - qlo;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < C::kNumBars; ++i) {
+      uint32_t count = 1;
+      if (i == C::kBarP || i == C::kBarDS || i == C::kBarDQEmpty) count = 128;
+      mbar_init(bar(i), count);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  Bounded bw{abort_flag, p.err, p.timeout_ns};
+  auto q_addr = [&](int s) { return sbase + C::kQOff + s * C::kTileBytes; };
+  auto do_addr = [&](int s) { return sbase + C::kDOOff + s * C::kTileBytes; };
+  const uint32_t k_addr = sbase + C::kKOff;
+  const uint32_t v_addr = sbase + C::kVOff;
+  const uint32_t ds_addr = sbase + C::kDSOff;
+  int load_count[kStages] = {0, 0};
+
+  if (warp == kLoadWarp) {
+    // ------------------------------------------------------------ loads
+    if (lane == 0 && nq > 0) {
+      tma_prefetch_desc(&tmQ);
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
+      tma_prefetch_desc(&tmDO);
+      mbar_arrive_expect_tx(bar(C::kBarKV), 2 * C::kTileBytes);
+      for (int x = 0; x < C::kBoxes; ++x) {
+        tma_load_4d(k_addr + x * C::kBoxBytes, &tmK, bar(C::kBarKV), x * 64, h, n0, b);
+        tma_load_4d(v_addr + x * C::kBoxBytes, &tmV, bar(C::kBarKV), x * 64, h, n0, b);
+      }
+      for (int t = 0; t < nq; ++t) {
+        const int s = t % kStages;
+        const int u = t / kStages;
+        if (u > 0 && !bw.wait(bar(C::kBarEmpty + s), (u - 1) & 1, 20)) break;
+        const int i0 = (qlo + t) * BM;
+        const uint32_t fb = bar(C::kBarFull + s);
+        mbar_arrive_expect_tx(fb, 2 * C::kTileBytes + 2 * BM * 4);
+        for (int x = 0; x < C::kBoxes; ++x) {
+          tma_load_4d(q_addr(s) + x * C::kBoxBytes, &tmQ, fb, x * 64, h, i0, b);
+          tma_load_4d(do_addr(s) + x * C::kBoxBytes, &tmDO, fb, x * 64, h, i0, b);
+        }
+        const size_t roff = size_t(bh) * p.Sq_pad + i0;
+        bulk_load(sbase + C::kLseOff + s * BM * 4, p.lse2 + roff, BM * 4, fb);
+        bulk_load(sbase + C::kDeltaOff + s * BM * 4, p.delta + roff, BM * 4, fb);
+        load_count[s]++;
+      }
+    }
+  } else if (warp == kMmaWarp) {
+    // ------------------------------------------------------------ MMA issue
+    if (lane == 0 && nq > 0) {
+      constexpr uint32_t id_s = idesc_bf16_f32(BN, BM, false, false);   // S^T, dP^T
+      constexpr uint32_t id_dv = idesc_bf16_f32(BN, D, false, true);    // dV, dK
+      constexpr uint32_t id_dq = idesc_bf16_f32(BM, D, true, true);     // dQ
+      auto issue_kmajor = [&](uint32_t d_col, uint32_t a_base, uint32_t b_base) {
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk / 4) * C::kBoxBytes + (kk % 4) * 32;
+          mma_bf16_ss(tmem + d_col, sdesc_sw128(a_base + off, 16), sdesc_sw128(b_base + off, 16),
+                      id_s, kk > 0 ? 1u : 0u);
+        }
+      };
+      bool ok = bw.wait(bar(C::kBarKV), 0, 21);
+      if (ok) ok = bw.wait(bar(C::kBarFull + 0), 0, 22);
+      if (ok) {
+        tc_fence_after();
+        issue_kmajor(C::kColS, k_addr, q_addr(0));
+        tc_commit(bar(C::kBarS));
+        issue_kmajor(C::kColDP, v_addr, do_addr(0));
+        tc_commit(bar(C::kBarDP));
+      }
+      for (int t = 0; ok && t < nq; ++t) {
+        const int s = t % kStages;
+        // dV += P^T dO   (A = P^T in tensor memory, K = query index)
+        if (!bw.wait(bar(C::kBarP), t & 1, 23)) { ok = false; break; }
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < BM / 16; ++kk)
+          mma_bf16_ts(tmem + C::kColDV, tmem + C::kColS + kk * 8,
+                      sdesc_sw128(do_addr(s) + kk * 16 * 128, C::kBoxBytes), id_dv,
+                      (t > 0 || kk > 0) ? 1u : 0u);
+        // dK += dS^T Q   (A = dS^T in shared memory, K-major over the query index)
+        if (!bw.wait(bar(C::kBarDS), t & 1, 24)) { ok = false; break; }
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < BM / 16; ++kk) {
+          const uint32_t aoff = (kk / 4) * C::kBoxBytes + (kk % 4) * 32;
+          mma_bf16_ss(tmem + C::kColDK, sdesc_sw128(ds_addr + aoff, 16),
+                      sdesc_sw128(q_addr(s) + kk * 16 * 128, C::kBoxBytes), id_dv,
+                      (t > 0 || kk > 0) ? 1u : 0u);
+        }
+        // next S^T while this tile's dQ is formed and drained
+        const bool more = t + 1 < nq;
+        const int s1 = (t + 1) % kStages;
+        if (more) {
+          if (!bw.wait(bar(C::kBarFull + s1), ((t + 1) / kStages) & 1, 25)) { ok = false; break; }
+          tc_fence_after();
+          issue_kmajor(C::kColS, k_addr, q_addr(s1));
+          tc_commit(bar(C::kBarS));
+        }
+        // dQ_tile = dS K  (A = dS read MN-major: rows of the buffer are keys = K index)
+#pragma unroll
+        for (int kk = 0; kk < BN / 16; ++kk)
+          mma_bf16_ss(tmem + C::kColDP, sdesc_sw128(ds_addr + kk * 16 * 128, C::kBoxBytes),
+                      sdesc_sw128(k_addr + kk * 16 * 128, C::kBoxBytes), id_dq,
+                      kk > 0 ? 1u : 0u);
+        tc_commit(bar(C::kBarDQFull));
+        tc_commit(bar(C::kBarEmpty + s));
+        tc_commit(bar(C::kBarDSEmpty));
+        if (more) {
+          if (!bw.wait(bar(C::kBarDQEmpty), t & 1, 26)) { ok = false; break; }
+          tc_fence_after();
+          issue_kmajor(C::kColDP, v_addr, do_addr(s1));
+          tc_commit(bar(C::kBarDP));
+        }
+      }
+    }
+  } else if (warp < kDrainWarp0) {
+    // ------------------------------------------------------------ P and dS
+    const int quad = warp % 4;
+    const int r = quad * 32 + lane;  // key row within the tile
+    const int kk_idx = n0 + r;       // key index
+    const uint32_t lane_off = uint32_t(quad * 32) << 16;
+    const uint32_t tS = tmem + lane_off + C::kColS;
+    const uint32_t tDP = tmem + lane_off + C::kColDP;
+    const float sl2 = p.scale_log2;
+    const int qmin_k = g.qmin(kk_idx);
+    const int qmax_k = min(g.qmax(kk_idx), p.Sq - 1);
+    const bool key_ok = kk_idx < p.Sk;
+    // rows of the dS^T buffer: 128 bytes per 64 columns, 16-byte chunks swizzled by row % 8
+    const uint32_t ds_row = ds_addr + uint32_t(r) * 128;
+    const uint32_t sw = uint32_t(r & 7);
+    bool ok = true;
+    for (int t = 0; t < nq; ++t) {
+      const int s = t % kStages;
+      const int i0 = (qlo + t) * BM;
+      const float* lse2 = reinterpret_cast<const float*>(smem + C::kLseOff + s * BM * 4);
+      const float* dlt = reinterpret_cast<const float*>(smem + C::kDeltaOff + s * BM * 4);
+      if (!bw.wait_warp(bar(C::kBarS), t & 1, 27)) { ok = false; break; }
+      tc_fence_after();
+      float pr[BM];
+#pragma unroll
+      for (int c0 = 0; c0 < BM; c0 += 32) {
+        uint32_t rr[32];
+        tmem_ld32(tS + c0, rr);
+#pragma unroll
+        for (int c = 0; c < 32; ++c)
+          pr[c0 + c] = ex2_approx(fmaf(__uint_as_float(rr[c]), sl2, -lse2[c0 + c]));
+      }
+      const bool full = key_ok && n0 + BN - 1 <= p.Sk - 1 && i0 + BM - 1 <= p.Sq - 1 &&
+                        i0 >= g.qmin(n0 + BN - 1) && i0 + BM - 1 <= g.qmax(n0);
+      if (!full) {
+        const int c_lo = key_ok ? qmin_k - i0 : (1 << 30);
+        const int c_hi = qmax_k - i0;
+#pragma unroll
+        for (int c = 0; c < BM; ++c)
+          if (c < c_lo || c > c_hi) pr[c] = 0.f;
+      }
+      {
+        uint32_t w[32];
+#pragma unroll
+        for (int c = 0; c < 32; ++c) w[c] = pack_bf16x2(pr[2 * c], pr[2 * c + 1]);
+        tmem_st32(tS, w);
+#pragma unroll
+        for (int c = 0; c < 32; ++c) w[c] = pack_bf16x2(pr[64 + 2 * c], pr[64 + 2 * c + 1]);
+        tmem_st32(tS + 32, w);
+      }
+      tc_fence_before();
+      mbar_arrive(bar(C::kBarP));
+
+      if (!bw.wait_warp(bar(C::kBarDP), t & 1, 28)) { ok = false; break; }
+      if (t > 0 && !bw.wait_warp(bar(C::kBarDSEmpty), (t - 1) & 1, 29)) { ok = false; break; }
+      tc_fence_after();
+#pragma unroll
+      for (int c0 = 0; c0 < BM; c0 += 32) {
+        uint32_t rr[32];
+        tmem_ld32(tDP + c0, rr);
+        uint32_t w[16];
+#pragma unroll
+        for (int c = 0; c < 32; c += 2) {
+          const float d0 = pr[c0 + c] * (__uint_as_float(rr[c]) - dlt[c0 + c]);
+          const float d1 = pr[c0 + c + 1] * (__uint_as_float(rr[c + 1]) - dlt[c0 + c + 1]);
+          w[c / 2] = pack_bf16x2(d0, d1);
+        }
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int col = c0 + 8 * q;            // first of 8 columns in this chunk
+          const uint32_t box = uint32_t(col / 64);
+          const uint32_t chunk = uint32_t((col % 64) / 8);
+          st_shared_v4(ds_row + box * C::kBoxBytes + ((chunk ^ sw) << 4), w[4 * q], w[4 * q + 1],
+                       w[4 * q + 2], w[4 * q + 3]);
+        }
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(bar(C::kBarDS));
+    }
+    // epilogue: dK = scale * acc, dV = acc (bf16)
+    if (ok && nq > 0) ok = bw.wait_warp(bar(C::kBarDQFull), (nq - 1) & 1, 30);
+    if (ok) {
+      tc_fence_after();
+      const size_t orow = ((size_t(b) * p.Sk + size_t(kk_idx)) * p.H + h) * D;
+#pragma unroll 1
+      for (int which = 0; which < 2; ++which) {
+        const uint32_t col = which == 0 ? C::kColDK : C::kColDV;
+        const float mul = which == 0 ? p.scale : 1.0f;
+        __nv_bfloat16* outp = which == 0 ? p.dk : p.dv;
+#pragma unroll 1
+        for (int c0 = 0; c0 < D; c0 += 32) {
+          uint32_t rr[32];
+          if (nq > 0) {
+            tmem_ld32(tmem + lane_off + col + c0, rr);
+          } else {
+#pragma unroll
+            for (int c = 0; c < 32; ++c) rr[c] = 0u;
+          }
+          uint32_t w[16];
+#pragma unroll
+          for (int c = 0; c < 16; ++c)
+            w[c] = pack_bf16x2(__uint_as_float(rr[2 * c]) * mul, __uint_as_float(rr[2 * c + 1]) * mul);
+          if (key_ok) {
+            uint8_t* dst = reinterpret_cast<uint8_t*>(outp + orow + c0);
+#pragma unroll
+            for (int v = 0; v < 4; ++v)
+              st_global_v4(dst + 16 * v, w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
+          }
+        }
+      }
+    }
+  } else if (warp < kMmaWarp) {
+    // ------------------------------------------------------------ dQ drain
+    const int quad = warp % 4;
+    const int r = quad * 32 + lane;  // query row within the tile
+    const uint32_t tDQ = tmem + (uint32_t(quad * 32) << 16) + C::kColDP;
+    for (int t = 0; t < nq; ++t) {
+      const int i = (qlo + t) * BM + r;
+      if (!bw.wait_warp(bar(C::kBarDQFull), t & 1, 31)) break;
+      tc_fence_after();
+      float* dst = p.dq_acc + (size_t(bh) * p.Sq_pad + i) * D;
+#pragma unroll
+      for (int c0 = 0; c0 < D; c0 += 32) {
+        uint32_t rr[32];
+        tmem_ld32(tDQ + c0, rr);
+#pragma unroll
+        for (int v = 0; v < 8; ++v)
+          red_add_v4(dst + c0 + 4 * v, __uint_as_float(rr[4 * v]), __uint_as_float(rr[4 * v + 1]),
+                     __uint_as_float(rr[4 * v + 2]), __uint_as_float(rr[4 * v + 3]));
+      }
+      tc_fence_before();
+      mbar_arrive(bar(C::kBarDQEmpty));
+    }
+  }
+
+  // ------------------------------------------------------------ teardown
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  if (*abort_flag) {
+    const uint64_t drain_ns = 2000000000ull;
+    if (warp == kLoadWarp && lane == 0 && nq > 0) {
+      for (int s = 0; s < kStages; ++s) {
+        if (load_count[s] == 0) continue;
+        const uint64_t t0 = globaltimer_ns();
+        while (!mbar_try_wait(bar(C::kBarFull + s), (load_count[s] - 1) & 1))
+          if (globaltimer_ns() - t0 > drain_ns) break;
+      }
+      const uint64_t t0 = globaltimer_ns();
+      while (!mbar_try_wait(bar(C::kBarKV), 0))
+        if (globaltimer_ns() - t0 > drain_ns) break;
+    }
+    if (warp == kMmaWarp && lane == 0) {
+      tc_commit(bar(C::kBarDone));
+      const uint64_t t0 = globaltimer_ns();
+      while (!mbar_try_wait(bar(C::kBarDone), 0))
+        if (globaltimer_ns() - t0 > drain_ns) break;
+    }
+    tc_fence_before();
+    __syncthreads();
+  }
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace bwd
+}  // namespace attn156

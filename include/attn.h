@@ -1,0 +1,144 @@
+/*
+ * attn.h - C ABI of the B200 (sm_100a) exact-attention library.
+ *
+ * The operation is exact scaled dot-product attention, computed as one fused,
+ * tiled kernel with an online softmax, and its recompute-based backward:
+ *
+ *   S = scale * Q K^T  (masked),  O = softmax_rows(S) V,  LSE_i = ln sum_j exp(S_ij)
+ *
+ * Sources: FlashAttention-2 overview (lshu.cn), section 2.1 (the three standard
+ * steps: Q K^T, row softmax, weighted sum of V) and section 2.2 (tiled fusion,
+ * online softmax with running row max m_i and row sum l_i, asynchronous
+ * prefetch of the next tile); section 3.3 (the call
+ * flash_attn_func(q, k, v, dropout_p, softmax_scale, causal) on tensors laid out
+ * (batch, seqlen, nheads, head_dim)); section 4.2 problem 4 (causal = upper-
+ * triangular mask).  The flash-attn install guide (yfxerp.com), section 1,
+ * names the sliding window (window_size) and the backward that recomputes the
+ * attention scores instead of storing them.
+ *
+ * Conventions for every entry point:
+ *   - Tensors Q, K, V, O, dO, dQ, dK, dV are bfloat16, row-major
+ *     (batch, seqlen, nheads, head_dim) with head_dim contiguous and no padding
+ *     between rows ("BSHD"), 16-byte aligned.  Q, O, dO, dQ have seqlen Sq;
+ *     K, V, dK, dV have seqlen Sk.
+ *   - lse is float32 (batch, nheads, Sq), natural-log log-sum-exp of the scaled,
+ *     masked scores; -inf for a query row that sees no key (its O row is 0).
+ *   - All pointers are device pointers owned by the caller; the library never
+ *     allocates, frees or retains them.  Calls are asynchronous on `stream`
+ *     (a cudaStream_t, may be 0 for the legacy default stream).
+ *   - Arguments are validated on the host before anything is launched; on any
+ *     error nothing is launched and the status says why.
+ *   - Masks (delta = Sk - Sq; bounds inclusive): key j is visible to query i iff
+ *       (causal == 0    or j <= i + delta)
+ *       (win_left  < 0  or j >= i + delta - win_left)
+ *       (win_right < 0  or j <= i + delta + win_right)
+ *     -1 means "unbounded" for a window side.  Causal is aligned to the
+ *     bottom-right corner when Sq != Sk.
+ *   - scale must be finite and > 0 (callers wanting the default pass
+ *     1/sqrt(head_dim)).
+ *   - head_dim D must be 64 or 128.  B, H, Sq, Sk must be >= 1 and every
+ *     tensor must hold fewer than 2^31 elements.
+ *   - The device must be compute capability 10.0 (B200, sm_100a).
+ *   - Device-side waits are bounded (about one second); a wait that runs out
+ *     makes the kernel stop early, record ATTN_ERR_TIMEOUT in a device error
+ *     word, release its tensor memory and return.  attn_get_last_device_error
+ *     reads (and clears) that word.
+ */
+#ifndef EXACT_ATTENTION_156_B200_ATTN_H
+#define EXACT_ATTENTION_156_B200_ATTN_H
+
+#include <stddef.h>
+
+#if defined(__GNUC__)
+#define ATTN_API __attribute__((visibility("default")))
+#else
+#define ATTN_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    ATTN_OK = 0,
+    ATTN_ERR_NULLPTR = 1,   /* a required pointer is NULL                         */
+    ATTN_ERR_SHAPE = 2,     /* B, H, Sq or Sk < 1, a size overflows, or bad scale */
+    ATTN_ERR_HEADDIM = 3,   /* head_dim not in {64, 128}                          */
+    ATTN_ERR_ALIGN = 4,     /* a tensor pointer is not 16-byte aligned            */
+    ATTN_ERR_WINDOW = 5,    /* win_left or win_right < -1                         */
+    ATTN_ERR_ARCH = 6,      /* current device is not compute capability 10.0      */
+    ATTN_ERR_DEVICE = 7,    /* a pointer is not device memory of the current GPU  */
+    ATTN_ERR_LAUNCH = 8,    /* a CUDA call (descriptor build, launch) failed      */
+    ATTN_ERR_TIMEOUT = 9,   /* a device-side bounded wait ran out                 */
+    ATTN_ERR_WORKSPACE = 10 /* workspace NULL, misaligned or smaller than needed  */
+} attn_status;
+
+/*
+ * attn_fwd - O and LSE of exact attention (FlashAttention-2 overview, section 2.2:
+ * tiled fusion + online softmax; the N x N score matrix never reaches memory).
+ *
+ *   q   [B, Sq, H, D] bf16 (in)      k, v [B, Sk, H, D] bf16 (in)
+ *   o   [B, Sq, H, D] bf16 (out)     lse  [B, H, Sq] float32 (out)
+ *   scale: multiplies Q K^T; causal: 0/1; win_left, win_right: -1 or >= 0.
+ * Errors: see attn_status; on error nothing is written.
+ */
+ATTN_API attn_status attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+                     int B, int Sq, int Sk, int H, int D, float scale, int causal,
+                     int win_left, int win_right, void* stream);
+
+/*
+ * attn_bwd_workspace_size - bytes of device workspace attn_bwd needs:
+ * a float32 dQ accumulator [B, H, ceil(Sq/128)*128, D] plus two float32 row
+ * vectors [B, H, ceil(Sq/128)*128] (Delta_i = sum_d dO_id O_id, and LSE in
+ * base 2).  Returns 0 if the arguments are out of range.
+ */
+ATTN_API size_t attn_bwd_workspace_size(int B, int Sq, int H, int D);
+
+/*
+ * attn_bwd - gradients of exact attention by recomputation (flash-attn install
+ * guide, section 1: the backward recomputes the scores; FlashAttention-2
+ * overview, section 2.1, second anti-pattern: the standard backward re-reads
+ * Q, K, V several times).  P is rebuilt from Q, K and the forward's LSE;
+ *   dV = P^T dO,  dP = dO V^T,  Delta_i = rowsum(dO * O),  dS = P * (dP - Delta),
+ *   dQ = scale dS K,  dK = scale dS^T Q.
+ *
+ *   q, k, v, o, dout, lse: as produced/consumed by attn_fwd (in)
+ *   dq [B, Sq, H, D], dk, dv [B, Sk, H, D] bf16 (out, fully overwritten)
+ *   workspace: device memory of at least attn_bwd_workspace_size(B, Sq, H, D)
+ *   bytes, 256-byte aligned; its contents on entry do not matter and on exit
+ *   are unspecified.  Must not alias any tensor argument.
+ * Errors: see attn_status; ATTN_ERR_WORKSPACE if the workspace is missing,
+ * misaligned or too small.
+ */
+ATTN_API attn_status attn_bwd(const void* q, const void* k, const void* v, const void* o,
+                     const void* dout, const float* lse, void* dq, void* dk, void* dv,
+                     int B, int Sq, int Sk, int H, int D, float scale, int causal,
+                     int win_left, int win_right, void* workspace, size_t workspace_bytes,
+                     void* stream);
+
+/* attn_status_string - static English text for a status code (never NULL). */
+ATTN_API const char* attn_status_string(attn_status s);
+
+/*
+ * attn_get_last_device_error - synchronises the current device, then returns
+ * ATTN_ERR_TIMEOUT if a kernel of this library recorded a timed-out wait since
+ * the last call (and clears the record), ATTN_ERR_LAUNCH if the device reports
+ * an error, ATTN_OK otherwise.
+ */
+ATTN_API attn_status attn_get_last_device_error(void);
+
+/*
+ * attn_device_timeout_selftest - launches one tiny kernel whose only work is
+ * a bounded wait on a barrier that nothing completes, using the same bounded
+ * wait as the attention kernels but with a limit of `limit_us` microseconds
+ * (1..1000000).  It exercises the timeout path without faulting the GPU.
+ * Returns ATTN_OK if launched; read the outcome with
+ * attn_get_last_device_error (expected: ATTN_ERR_TIMEOUT).
+ */
+ATTN_API attn_status attn_device_timeout_selftest(int limit_us, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* EXACT_ATTENTION_156_B200_ATTN_H */

@@ -1,0 +1,105 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports
+every entry point include/attn.h declares, and rejects bad arguments before
+touching CUDA."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "attn.h")
+LIB = os.path.join(ROOT, "exact_attention_156_b200", "libattn156.so")
+
+OK, NULLPTR, SHAPE, HEADDIM, ALIGN, WINDOW, ARCH, DEVICE = 0, 1, 2, 3, 4, 5, 6, 7
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    names = re.findall(r"ATTN_API\s+[\w\s\*]+?\b(attn_\w+)\s*\(", text)
+    assert names, "no declarations found"
+    return names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = ctypes.CDLL(LIB)
+    names = declared_functions()
+    assert {"attn_fwd", "attn_bwd", "attn_bwd_workspace_size", "attn_status_string"} <= set(names)
+    for n in names:
+        assert hasattr(lib, n), f"{n} declared in attn.h but not exported"
+
+
+def test_status_enum_matches_binding():
+    from exact_attention_156_b200 import ATTN_STATUS
+    text = open(HEADER).read()
+    enum = dict((int(v), k) for k, v in re.findall(r"(ATTN_\w+)\s*=\s*(\d+)", text))
+    assert enum == ATTN_STATUS
+
+
+def test_status_strings():
+    from exact_attention_156_b200 import status_string
+    for s in range(11):
+        assert status_string(s) and status_string(s) != "unknown status"
+    assert status_string(99) == "unknown status"
+
+
+def _fwd(lib, q=0x1000, k=0x2000, v=0x3000, o=0x4000, lse=0x5000, B=1, Sq=128, Sk=128, H=2,
+         D=128, scale=0.125, causal=0, wl=-1, wr=-1):
+    return lib.attn_fwd(q, k, v, o, lse, B, Sq, Sk, H, D, scale, causal, wl, wr, None)
+
+
+def test_fwd_validation_order_and_codes():
+    from exact_attention_156_b200 import lib
+    assert _fwd(lib, q=None) == NULLPTR
+    assert _fwd(lib, lse=None) == NULLPTR
+    assert _fwd(lib, B=0) == SHAPE
+    assert _fwd(lib, Sk=0) == SHAPE
+    assert _fwd(lib, H=70000) == SHAPE
+    assert _fwd(lib, Sq=1 << 20, H=32, D=128) == SHAPE       # 2^32 elements
+    assert _fwd(lib, D=96) == HEADDIM
+    assert _fwd(lib, D=256) == HEADDIM
+    assert _fwd(lib, scale=0.0) == SHAPE
+    assert _fwd(lib, scale=float("nan")) == SHAPE
+    assert _fwd(lib, scale=float("inf")) == SHAPE
+    assert _fwd(lib, wl=-2) == WINDOW
+    assert _fwd(lib, wr=-5) == WINDOW
+    assert _fwd(lib, q=0x1008) == ALIGN
+    assert _fwd(lib, lse=0x5002) == ALIGN
+
+
+def test_bwd_validation_and_workspace_size():
+    from exact_attention_156_b200 import lib
+    assert lib.attn_bwd_workspace_size(1, 128, 2, 64) == 128 * 2 * (64 * 4 + 8)
+    assert lib.attn_bwd_workspace_size(1, 129, 2, 128) == 256 * 2 * (128 * 4 + 8)
+    assert lib.attn_bwd_workspace_size(0, 128, 2, 64) == 0
+    assert lib.attn_bwd_workspace_size(1, 128, 2, 80) == 0
+    p = [0x1000 * (i + 1) for i in range(9)]
+    ws = lib.attn_bwd_workspace_size(1, 128, 2, 128)
+
+    def bwd(ptrs=p, B=1, Sq=128, Sk=128, H=2, D=128, wsp=0x100000, wsz=ws, wl=-1):
+        return lib.attn_bwd(*ptrs, B, Sq, Sk, H, D, 0.1, 1, wl, -1, wsp, wsz, None)
+
+    assert bwd(ptrs=[None] + p[1:]) == NULLPTR
+    assert bwd(B=0) == SHAPE
+    assert bwd(D=32) == HEADDIM
+    assert bwd(wl=-3) == WINDOW
+    assert bwd(ptrs=p[:6] + [0x7004] + p[7:]) == ALIGN
+    assert bwd(wsp=None) == 10
+    assert bwd(wsp=0x100010) == 10          # not 256-byte aligned
+    assert bwd(wsz=ws - 4) == 10
+
+
+def test_valid_arguments_without_a_gpu_fail_on_device_checks():
+    """With well-formed arguments the next gate is the device: on a machine
+    without a B200 (or with pointers that are not device memory) the call
+    must refuse rather than launch."""
+    from exact_attention_156_b200 import lib
+    assert _fwd(lib) in (ARCH, DEVICE)
+
+
+def test_binding_refuses_cpu_tensors():
+    import torch
+    from exact_attention_156_b200 import attn_fwd
+    q = torch.zeros(1, 128, 2, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="CUDA"):
+        attn_fwd(q, q, q)
