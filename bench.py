@@ -1,0 +1,447 @@
+#!/usr/bin/env python
+"""Benchmark of the exact-attention hot path on B200.
+
+One step = one pass of the whole path over one batch: the fused forward
+(O, LSE) followed by the recompute backward (preprocess, main, dQ finalize)
+on the fwd+bwd workload: batch 1, 32 heads, Sq = Sk = 8192, head_dim 128,
+causal, Q/K/V/dO i.i.d. N(0,1)*0.5 in bf16 (seeded, synthetic).
+
+Throughput is attention TFLOP/s: forward 4*B*H*Sq*Sk*D (halved for causal)
+plus backward 2.5x that (five products, one of them the recomputed scores).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+N > 1 runs under torchrun, one process per GPU; every rank processes its own
+independent copy of the workload (weak scaling, no collective on the data
+path); times are taken on the device and reduced with a max over ranks.
+``--impl reference`` times the float64 CPU oracle (rank 0 only) on bounded
+samples of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "attention fwd/bwd TFLOPS at seq 8K–32K, D=128, bf16 vs B200 dense BF16 peak"
+UNIT = "TFLOP/s"
+WORKLOAD = dict(name="c5_b1h32s8192d128_fwdbwd", B=1, H=32, Sq=8192, Sk=8192, D=128,
+                causal=1, win_left=-1, win_right=-1, input_scale=0.5, seed=1005)
+FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "hbm_gbs": 6650.0, "source": "fallback"}
+BWD_KERNEL_SOURCES = ["bwd_sm100.cuh", "ptx.cuh", "common.cuh"]
+FWD_KERNEL_SOURCES = ["fwd_sm100.cuh", "ptx.cuh", "common.cuh"]
+ORACLE_ROWS_PER_SAMPLE = 512
+
+
+# ---------------------------------------------------------------------------
+# work accounting
+# ---------------------------------------------------------------------------
+def fwd_flops(w) -> float:
+    f = 4.0 * w["B"] * w["H"] * w["Sq"] * w["Sk"] * w["D"]
+    return f / 2 if w["causal"] else f
+
+
+def bwd_flops(w) -> float:
+    return 2.5 * fwd_flops(w)
+
+
+def step_flops(w) -> float:
+    return fwd_flops(w) + bwd_flops(w)
+
+
+def visible_keys(i, w) -> int:
+    d = w["Sk"] - w["Sq"]
+    lo, hi = 0, w["Sk"] - 1
+    if w["causal"]:
+        hi = min(hi, i + d)
+    if w["win_left"] >= 0:
+        lo = max(lo, i + d - w["win_left"])
+    if w["win_right"] >= 0:
+        hi = min(hi, i + d + w["win_right"])
+    return max(0, hi - lo + 1)
+
+
+# ---------------------------------------------------------------------------
+# distributed plumbing (no collective touches attention data)
+# ---------------------------------------------------------------------------
+def dist_env():
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def reduce_max(value: float, device=None) -> float:
+    """Max of a float over all ranks (identity when not distributed)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64,
+                     device=device if device is not None else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(device=None):
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized():
+        if device is not None and dist.get_backend() == "nccl":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+def aggregate_value(per_rank_flops: float, n_ranks: int, max_ms: float) -> float:
+    """Whole-job TFLOP/s: all ranks' work over the slowest rank's time."""
+    return per_rank_flops * n_ranks / (max_ms * 1e-3) / 1e12
+
+
+# ---------------------------------------------------------------------------
+# peaks, clocks, committed ncu traffic
+# ---------------------------------------------------------------------------
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        d["source"] = "measured"
+        return d
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS)
+
+
+def sources_sha(files) -> str:
+    h = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(ROOT, "exact_attention_156_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:12]
+
+
+def committed_traffic(kernel: str, sha: str):
+    """DRAM bytes per launch recorded from an ncu capture, if the kernel's
+    sources have not changed since (profiles/traffic_per_launch.txt)."""
+    path = os.path.join(ROOT, "profiles", "traffic_per_launch.txt")
+    try:
+        for line in open(path):
+            parts = line.split()
+            if len(parts) >= 3 and not line.startswith("#") and parts[0] == kernel:
+                if parts[1] == sha:
+                    return float(parts[2])
+    except OSError:
+        pass
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons while it runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.gpu_id, f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.15)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) >= 9:
+                rows.append(parts)
+        os.unlink(self.path)
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        smax = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[j] for r in rows for j in range(4) if r[5 + j] == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle samples (cpu_baseline leg and --impl reference)
+# ---------------------------------------------------------------------------
+def oracle_sample_inputs(w):
+    from synth import bf16_bits_to_f32, make_inputs
+    bits = make_inputs(w["B"], w["Sq"], w["Sk"], w["H"], w["D"], w["seed"], w["input_scale"],
+                       with_dout=True)
+    return {n: bf16_bits_to_f32(bits[n]) for n in ("q", "k", "v", "do")}
+
+
+def oracle_sample(inputs, w, sample_idx: int):
+    """fwd+bwd of the oracle for ORACLE_ROWS_PER_SAMPLE seeded query rows of
+    one head (their O, LSE, dQ and their share of dK, dV).  Returns
+    (seconds, attention flops of that sample by the metric's convention)."""
+    import numpy as np
+    import oracle
+    rng = np.random.default_rng(10_000 + sample_idx)
+    h = int(rng.integers(0, w["H"]))
+    rows = np.sort(rng.choice(w["Sq"], size=ORACLE_ROWS_PER_SAMPLE, replace=False))
+    pairs = sum(visible_keys(int(i), w) for i in rows)
+    t0 = time.perf_counter()
+    oracle.attention_backward_rows(inputs["q"], inputs["k"], inputs["v"], inputs["do"], 0, h,
+                                   rows, 1.0 / math.sqrt(w["D"]), w["causal"], w["win_left"],
+                                   w["win_right"])
+    dt = time.perf_counter() - t0
+    return dt, 14.0 * w["D"] * pairs  # 4*D (fwd) + 10*D (bwd) per visible pair
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads") for i in threadpool_info() if i.get("user_api") == "blas"]
+        return int(max(n)) if n else os.cpu_count()
+    except Exception:
+        return os.cpu_count()
+
+
+def cpu_baseline(w, budget_s: float = 15.0):
+    inputs = oracle_sample_inputs(w)
+    tot_s, tot_f, n = 0.0, 0.0, 0
+    while tot_s < budget_s and n < 64:
+        dt, fl = oracle_sample(inputs, w, n)
+        tot_s += dt
+        tot_f += fl
+        n += 1
+    return {"value": tot_f / tot_s / 1e12, "unit": UNIT, "cores": blas_threads(),
+            "kind": "oracle",
+            "sample": f"{n} samples x {ORACLE_ROWS_PER_SAMPLE} seeded query rows of one head of "
+                      f"{w['name']} (fwd O/LSE, bwd dQ rows and their dK/dV share), float64 numpy, "
+                      f"{tot_s:.1f} s total; flops counted as 14*D per visible pair"}
+
+
+def run_reference(args):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return 0
+    w = WORKLOAD
+    inputs = oracle_sample_inputs(w)
+    for i in range(args.warmup):
+        oracle_sample(inputs, w, 1000 + i)
+    tot_s, tot_f = 0.0, 0.0
+    for i in range(args.steps):
+        dt, fl = oracle_sample(inputs, w, i)
+        tot_s += dt
+        tot_f += fl
+    value = tot_f / tot_s / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": tot_s / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": config_dict(w),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+                         "sample": f"each step: {ORACLE_ROWS_PER_SAMPLE} seeded query rows of one "
+                                   f"head of {w['name']}, fwd+bwd in float64 numpy"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def config_dict(w):
+    return {"workload": f"{w['name']}: fwd+bwd, B={w['B']} H={w['H']} Sq=Sk={w['Sq']} "
+                        f"D={w['D']} causal bf16, inputs N(0,1)*{w['input_scale']}",
+            "B": w["B"], "H": w["H"], "Sq": w["Sq"], "Sk": w["Sk"], "D": w["D"],
+            "causal": bool(w["causal"]),
+            "l2": "no flush: inputs (Q,K,V,dO 256 MiB) and outputs exceed the 126 MB L2"}
+
+
+# ---------------------------------------------------------------------------
+# GPU arm
+# ---------------------------------------------------------------------------
+def run_gpu(args):
+    import torch
+    rank, world, local = dist_env()
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    device = torch.device("cuda", local if world > 1 else torch.cuda.current_device())
+    torch.cuda.set_device(device)
+    from exact_attention_156_b200 import (attn_bwd_stages, attn_bwd_workspace_size, attn_fwd,
+                                          get_last_device_error)
+    from synth import make_inputs
+
+    w = WORKLOAD
+    B, H, Sq, Sk, D = w["B"], w["H"], w["Sq"], w["Sk"], w["D"]
+    causal = bool(w["causal"])
+    win = (w["win_left"], w["win_right"])
+    bits = make_inputs(B, Sq, Sk, H, D, w["seed"] + rank, w["input_scale"], with_dout=True)
+    host = {n: torch.from_numpy(bits[n].view("int16")).view(torch.bfloat16).pin_memory()
+            for n in ("q", "k", "v", "do")}
+    dev = {n: t.to(device) for n, t in host.items()}
+    q, k, v, do = dev["q"], dev["k"], dev["v"], dev["do"]
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, Sq), dtype=torch.float32, device=device)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws = torch.empty(attn_bwd_workspace_size(B, Sq, H, D), dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream(device)
+
+    names = ["fwd", "bwd_preprocess", "bwd_main", "bwd_dq_finalize"]
+
+    def step(evs=None):
+        if evs is not None:
+            evs[0].record(stream)
+        attn_fwd(q, k, v, causal=causal, window_size=win, out=o, lse=lse, stream=stream)
+        rec = (lambda i: evs[i + 1].record(stream)) if evs is not None else None
+        attn_bwd_stages(q, k, v, o, do, lse, dq, dk, dv, ws, causal=causal, window_size=win,
+                        stream=stream, between=rec)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(device)
+    if get_last_device_error() != 0:
+        raise RuntimeError("device-side timeout during warm-up")
+
+    # timed region: K steps, per-kernel events on the launching stream
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler("GPU-" + str(torch.cuda.get_device_properties(device).uuid))
+    barrier(device)
+    torch.cuda.synchronize(device)
+    sampler.start()
+    start.record(stream)
+    for i in range(args.steps):
+        step(evs[i])
+    end.record(stream)
+    torch.cuda.synchronize(device)
+    barrier(device)
+    clocks = sampler.stop()
+    total_ms = start.elapsed_time(end)
+    per_kernel = [statistics.mean(evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(args.steps))
+                  for j in range(4)]
+    launches = 4 * args.steps
+    if get_last_device_error() != 0:
+        raise RuntimeError("device-side timeout during the timed region")
+    max_ms = reduce_max(total_ms, device)
+    ms_per_step = max_ms / args.steps
+    value = aggregate_value(step_flops(w), world, ms_per_step)
+
+    # end to end through the public API with host buffers: H2D of the step's
+    # inputs from pinned memory, the step, D2H of its results (O, LSE, dQ, dK, dV)
+    out_host = {n: torch.empty(t.shape, dtype=t.dtype).pin_memory()
+                for n, t in (("o", o), ("lse", lse), ("dq", dq), ("dk", dk), ("dv", dv))}
+    e2e_steps = max(3, min(args.steps, 10))
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = sum(t.numel() * t.element_size() for t in out_host.values())
+
+    def e2e_step():
+        for n in ("q", "k", "v", "do"):
+            dev[n].copy_(host[n], non_blocking=True)
+        step()
+        for n, t in (("o", o), ("lse", lse), ("dq", dq), ("dk", dk), ("dv", dv)):
+            out_host[n].copy_(t, non_blocking=True)
+
+    e2e = None
+    if not args.no_e2e:
+        e2e_step()
+        torch.cuda.synchronize(device)
+        barrier(device)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(e2e_steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize(device)
+        barrier(device)
+        e2e_ms = reduce_max(e0.elapsed_time(e1), device) / e2e_steps
+        e2e = {"value": aggregate_value(step_flops(w), world, e2e_ms), "unit": UNIT,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
+               "steps": e2e_steps}
+
+    peaks = load_peaks()
+    peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    bwd_main_tflops = bwd_flops(w) / (per_kernel[2] * 1e-3) / 1e12
+    fwd_tflops = fwd_flops(w) / (per_kernel[0] * 1e-3) / 1e12
+    kernels = {
+        "fwd": {"ms": per_kernel[0], "tflops": fwd_tflops, "frac": fwd_tflops / peak},
+        "bwd_preprocess": {"ms": per_kernel[1]},
+        "bwd_main": {"ms": per_kernel[2], "tflops": bwd_main_tflops,
+                     "frac": bwd_main_tflops / peak},
+        "bwd_dq_finalize": {"ms": per_kernel[3]},
+    }
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": config_dict(w),
+        "roofline": {"bound": "tensor", "kernel": "attn_bwd_main_kernel<128>",
+                     "achieved": bwd_main_tflops, "peak": peak, "unit": "TFLOP/s",
+                     "frac": bwd_main_tflops / peak,
+                     "peak_source": f"{peaks.get('source')} bf16_tflops (burst)",
+                     "traffic": committed_traffic("attn_bwd_main_kernel",
+                                                  sources_sha(BWD_KERNEL_SOURCES))},
+        "kernels": kernels,
+        "fwd_roofline": {"bound": "tensor", "kernel": "attn_fwd_kernel<128>",
+                         "achieved": fwd_tflops, "peak": peak, "unit": "TFLOP/s",
+                         "frac": fwd_tflops / peak,
+                         "traffic": committed_traffic("attn_fwd_kernel",
+                                                      sources_sha(FWD_KERNEL_SOURCES))},
+        "e2e": e2e,
+        "gpu_launches": launches,
+        "clocks": clocks,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true",
+                    help="skip the timed oracle sample (it adds ~15 s of CPU time)")
+    ap.add_argument("--no-e2e", action="store_true",
+                    help="skip the host-buffer end-to-end leg (fewer launches under a profiler)")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_gpu(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -10,6 +10,7 @@ from ._binding import (  # noqa: F401
     LIB_PATH,
     AttnError,
     attn_bwd,
+    attn_bwd_stages,
     attn_bwd_workspace_size,
     attn_fwd,
     device_timeout_selftest,

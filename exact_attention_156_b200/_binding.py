@@ -41,6 +41,12 @@ def _load() -> ctypes.CDLL:
     lib.attn_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, i, i,
                              vp, sz, vp]
     lib.attn_bwd.restype = i
+    lib.attn_bwd_preprocess.argtypes = [vp, vp, vp, i, i, i, i, vp, sz, vp]
+    lib.attn_bwd_preprocess.restype = i
+    lib.attn_bwd_main.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, i, i, vp, sz, vp]
+    lib.attn_bwd_main.restype = i
+    lib.attn_bwd_dq_finalize.argtypes = [vp, i, i, i, i, f, vp, sz, vp]
+    lib.attn_bwd_dq_finalize.restype = i
     lib.attn_bwd_workspace_size.argtypes = [i, i, i, i]
     lib.attn_bwd_workspace_size.restype = sz
     lib.attn_status_string.argtypes = [i]
@@ -149,6 +155,43 @@ def attn_bwd(q, k, v, out, dout, lse, softmax_scale: Optional[float] = None,
                       _stream_handle(stream, q.device))
     if st != 0:
         raise AttnError(st, "attn_bwd")
+    return dq, dk, dv
+
+
+def attn_bwd_stages(q, k, v, out, dout, lse, dq, dk, dv, workspace,
+                    softmax_scale: Optional[float] = None, causal: bool = False,
+                    window_size: Optional[Tuple[int, int]] = None, stream=None, between=None):
+    """attn_bwd as its three C-ABI stages (preprocess, main, dq finalize).
+
+    ``between(i)`` is called before stage i (0, 1, 2) and after the last one
+    (i = 3) with no arguments otherwise; callers use it to record timing events
+    on the same stream.  All tensors must be preallocated.
+    """
+    B, Sq, H, D = q.shape
+    Sk = k.shape[1]
+    c, wl, wr = _window(causal, window_size)
+    sc = _scale(softmax_scale, D)
+    hs = _stream_handle(stream, q.device)
+    wp, wb = workspace.data_ptr(), workspace.numel() * workspace.element_size()
+    if between:
+        between(0)
+    st = lib.attn_bwd_preprocess(out.data_ptr(), dout.data_ptr(), lse.data_ptr(), B, Sq, H, D,
+                                 wp, wb, hs)
+    if st != 0:
+        raise AttnError(st, "attn_bwd_preprocess")
+    if between:
+        between(1)
+    st = lib.attn_bwd_main(q.data_ptr(), k.data_ptr(), v.data_ptr(), dout.data_ptr(),
+                           dk.data_ptr(), dv.data_ptr(), B, Sq, Sk, H, D, sc, c, wl, wr, wp, wb, hs)
+    if st != 0:
+        raise AttnError(st, "attn_bwd_main")
+    if between:
+        between(2)
+    st = lib.attn_bwd_dq_finalize(dq.data_ptr(), B, Sq, H, D, sc, wp, wb, hs)
+    if st != 0:
+        raise AttnError(st, "attn_bwd_dq_finalize")
+    if between:
+        between(3)
     return dq, dk, dv
 
 

@@ -6,6 +6,7 @@
 #include <cuda_runtime.h>
 
 #include <math.h>
+#include <initializer_list>
 #include <mutex>
 #include <stdint.h>
 #include <string.h>
@@ -160,61 +161,88 @@ attn_status launch_fwd(const DeviceState& st, const void* q, const void* k, cons
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_LAUNCH;
 }
 
-template <int D>
-attn_status launch_bwd(const DeviceState& st, const void* q, const void* k, const void* v,
-                       const void* o, const void* dout, const float* lse, void* dq, void* dk,
-                       void* dv, int B, int Sq, int Sk, int H, float scale, int causal,
-                       int win_left, int win_right, void* workspace, cudaStream_t stream) {
-  const int Sqp = sq_pad(Sq);
-  const size_t rows = size_t(B) * H * Sqp;
-  float* dq_acc = static_cast<float*>(workspace);
-  float* lse2 = dq_acc + rows * D;
-  float* delta = lse2 + rows;
+struct Workspace {
+  float* dq_acc;  // [B*H][Sq_pad][D]
+  float* lse2;    // [B*H][Sq_pad]
+  float* delta;   // [B*H][Sq_pad]
+  int Sq_pad;
+};
 
-  {
-    const long long warps = (long long)rows;
-    const unsigned blocks = unsigned((warps + 7) / 8);
-    bwd::attn_bwd_pre_kernel<D><<<blocks, 256, 0, stream>>>(
-        static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout), lse, lse2,
-        delta, dq_acc, B, H, Sq, Sqp);
-    if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_LAUNCH;
-  }
-  {
-    alignas(64) CUtensorMap mq, mk, mv, mdo;
-    if (make_map(&mq, q, B, Sq, H, D) != ATTN_OK || make_map(&mk, k, B, Sk, H, D) != ATTN_OK ||
-        make_map(&mv, v, B, Sk, H, D) != ATTN_OK || make_map(&mdo, dout, B, Sq, H, D) != ATTN_OK)
-      return ATTN_ERR_LAUNCH;
-    bwd::Params p;
-    p.dk = static_cast<__nv_bfloat16*>(dk);
-    p.dv = static_cast<__nv_bfloat16*>(dv);
-    p.lse2 = lse2;
-    p.delta = delta;
-    p.dq_acc = dq_acc;
-    p.B = B;
-    p.H = H;
-    p.Sq = Sq;
-    p.Sk = Sk;
-    p.Sq_pad = Sqp;
-    p.scale = scale;
-    p.scale_log2 = scale * 1.4426950408889634f;
-    p.causal = causal ? 1 : 0;
-    p.win_left = win_left;
-    p.win_right = win_right;
-    p.err = st.err;
-    p.timeout_ns = kTimeoutNs;
-    dim3 grid((Sk + bwd::BN - 1) / bwd::BN, H, B);
-    bwd::attn_bwd_main_kernel<D>
-        <<<grid, bwd::kThreads, bwd::Cfg<D>::kSmemBytes, stream>>>(mq, mk, mv, mdo, p);
-    if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_LAUNCH;
-  }
-  {
-    const long long total = (long long)B * Sq * H * (D / 8);
-    const unsigned blocks = unsigned((total + 255) / 256);
-    bwd::attn_bwd_dq_kernel<D><<<blocks, 256, 0, stream>>>(
-        dq_acc, static_cast<__nv_bfloat16*>(dq), B, H, Sq, Sqp, scale);
-    if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_LAUNCH;
-  }
+Workspace carve(void* workspace, int B, int Sq, int H, int D) {
+  Workspace w;
+  w.Sq_pad = sq_pad(Sq);
+  const size_t rows = size_t(B) * H * w.Sq_pad;
+  w.dq_acc = static_cast<float*>(workspace);
+  w.lse2 = w.dq_acc + rows * D;
+  w.delta = w.lse2 + rows;
+  return w;
+}
+
+template <int D>
+attn_status launch_bwd_pre(const void* o, const void* dout, const float* lse, int B, int Sq,
+                           int H, const Workspace& w, cudaStream_t stream) {
+  const long long rows = (long long)B * H * w.Sq_pad;
+  const unsigned blocks = unsigned((rows + 7) / 8);
+  bwd::attn_bwd_pre_kernel<D><<<blocks, 256, 0, stream>>>(
+      static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout), lse, w.lse2,
+      w.delta, w.dq_acc, B, H, Sq, w.Sq_pad);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_LAUNCH;
+}
+
+template <int D>
+attn_status launch_bwd_main(const DeviceState& st, const void* q, const void* k, const void* v,
+                            const void* dout, void* dk, void* dv, int B, int Sq, int Sk, int H,
+                            float scale, int causal, int win_left, int win_right,
+                            const Workspace& w, cudaStream_t stream) {
+  alignas(64) CUtensorMap mq, mk, mv, mdo;
+  if (make_map(&mq, q, B, Sq, H, D) != ATTN_OK || make_map(&mk, k, B, Sk, H, D) != ATTN_OK ||
+      make_map(&mv, v, B, Sk, H, D) != ATTN_OK || make_map(&mdo, dout, B, Sq, H, D) != ATTN_OK)
+    return ATTN_ERR_LAUNCH;
+  bwd::Params p;
+  p.dk = static_cast<__nv_bfloat16*>(dk);
+  p.dv = static_cast<__nv_bfloat16*>(dv);
+  p.lse2 = w.lse2;
+  p.delta = w.delta;
+  p.dq_acc = w.dq_acc;
+  p.B = B;
+  p.H = H;
+  p.Sq = Sq;
+  p.Sk = Sk;
+  p.Sq_pad = w.Sq_pad;
+  p.scale = scale;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.causal = causal ? 1 : 0;
+  p.win_left = win_left;
+  p.win_right = win_right;
+  p.err = st.err;
+  p.timeout_ns = kTimeoutNs;
+  dim3 grid((Sk + bwd::BN - 1) / bwd::BN, H, B);
+  bwd::attn_bwd_main_kernel<D>
+      <<<grid, bwd::kThreads, bwd::Cfg<D>::kSmemBytes, stream>>>(mq, mk, mv, mdo, p);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_LAUNCH;
+}
+
+template <int D>
+attn_status launch_bwd_dq(void* dq, int B, int Sq, int H, float scale, const Workspace& w,
+                          cudaStream_t stream) {
+  const long long total = (long long)B * Sq * H * (D / 8);
+  const unsigned blocks = unsigned((total + 255) / 256);
+  bwd::attn_bwd_dq_kernel<D><<<blocks, 256, 0, stream>>>(
+      w.dq_acc, static_cast<__nv_bfloat16*>(dq), B, H, Sq, w.Sq_pad, scale);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_LAUNCH;
+}
+
+attn_status check_workspace(const void* workspace, size_t bytes, int B, int Sq, int H, int D) {
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) ||
+      bytes < workspace_bytes(B, Sq, H, D))
+    return ATTN_ERR_WORKSPACE;
   return ATTN_OK;
+}
+
+bool all_on_device(std::initializer_list<const void*> ptrs) {
+  for (const void* p : ptrs)
+    if (!on_current_device(p)) return false;
+  return true;
 }
 
 __global__ void attn_timeout_selftest_kernel(uint32_t* err, uint64_t limit_ns) {
@@ -289,21 +317,90 @@ attn_status attn_bwd(const void* q, const void* k, const void* v, const void* o,
       !aligned16(dq) || !aligned16(dk) || !aligned16(dv) ||
       (reinterpret_cast<uintptr_t>(lse) & 3u))
     return ATTN_ERR_ALIGN;
-  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) ||
-      workspace_size < workspace_bytes(B, Sq, H, D))
-    return ATTN_ERR_WORKSPACE;
+  s = check_workspace(workspace, workspace_size, B, Sq, H, D);
+  if (s != ATTN_OK) return s;
   DeviceState* st = nullptr;
   s = device_state(&st);
   if (s != ATTN_OK) return s;
-  const void* ptrs[] = {q, k, v, o, dout, lse, dq, dk, dv, workspace};
-  for (const void* ptr : ptrs)
-    if (!on_current_device(ptr)) return ATTN_ERR_DEVICE;
+  if (!all_on_device({q, k, v, o, dout, lse, dq, dk, dv, workspace})) return ATTN_ERR_DEVICE;
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
-  if (D == 64)
-    return launch_bwd<64>(*st, q, k, v, o, dout, lse, dq, dk, dv, B, Sq, Sk, H, scale, causal,
-                          win_left, win_right, workspace, cs);
-  return launch_bwd<128>(*st, q, k, v, o, dout, lse, dq, dk, dv, B, Sq, Sk, H, scale, causal,
-                         win_left, win_right, workspace, cs);
+  const Workspace w = carve(workspace, B, Sq, H, D);
+  if (D == 64) {
+    s = launch_bwd_pre<64>(o, dout, lse, B, Sq, H, w, cs);
+    if (s == ATTN_OK)
+      s = launch_bwd_main<64>(*st, q, k, v, dout, dk, dv, B, Sq, Sk, H, scale, causal, win_left,
+                              win_right, w, cs);
+    if (s == ATTN_OK) s = launch_bwd_dq<64>(dq, B, Sq, H, scale, w, cs);
+  } else {
+    s = launch_bwd_pre<128>(o, dout, lse, B, Sq, H, w, cs);
+    if (s == ATTN_OK)
+      s = launch_bwd_main<128>(*st, q, k, v, dout, dk, dv, B, Sq, Sk, H, scale, causal, win_left,
+                               win_right, w, cs);
+    if (s == ATTN_OK) s = launch_bwd_dq<128>(dq, B, Sq, H, scale, w, cs);
+  }
+  return s;
+}
+
+attn_status attn_bwd_preprocess(const void* o, const void* dout, const float* lse, int B, int Sq,
+                                int H, int D, void* workspace, size_t workspace_size,
+                                void* stream) {
+  if (!o || !dout || !lse) return ATTN_ERR_NULLPTR;
+  attn_status s = check_common(B, Sq, 1, H, D, 1.0f, -1, -1);
+  if (s != ATTN_OK) return s;
+  if (!aligned16(o) || !aligned16(dout) || (reinterpret_cast<uintptr_t>(lse) & 3u))
+    return ATTN_ERR_ALIGN;
+  s = check_workspace(workspace, workspace_size, B, Sq, H, D);
+  if (s != ATTN_OK) return s;
+  DeviceState* st = nullptr;
+  s = device_state(&st);
+  if (s != ATTN_OK) return s;
+  if (!all_on_device({o, dout, lse, workspace})) return ATTN_ERR_DEVICE;
+  const Workspace w = carve(workspace, B, Sq, H, D);
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  return D == 64 ? launch_bwd_pre<64>(o, dout, lse, B, Sq, H, w, cs)
+                 : launch_bwd_pre<128>(o, dout, lse, B, Sq, H, w, cs);
+}
+
+attn_status attn_bwd_main(const void* q, const void* k, const void* v, const void* dout,
+                          void* dk, void* dv, int B, int Sq, int Sk, int H, int D, float scale,
+                          int causal, int win_left, int win_right, void* workspace,
+                          size_t workspace_size, void* stream) {
+  if (!q || !k || !v || !dout || !dk || !dv) return ATTN_ERR_NULLPTR;
+  attn_status s = check_common(B, Sq, Sk, H, D, scale, win_left, win_right);
+  if (s != ATTN_OK) return s;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dout) || !aligned16(dk) ||
+      !aligned16(dv))
+    return ATTN_ERR_ALIGN;
+  s = check_workspace(workspace, workspace_size, B, Sq, H, D);
+  if (s != ATTN_OK) return s;
+  DeviceState* st = nullptr;
+  s = device_state(&st);
+  if (s != ATTN_OK) return s;
+  if (!all_on_device({q, k, v, dout, dk, dv, workspace})) return ATTN_ERR_DEVICE;
+  const Workspace w = carve(workspace, B, Sq, H, D);
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  return D == 64 ? launch_bwd_main<64>(*st, q, k, v, dout, dk, dv, B, Sq, Sk, H, scale, causal,
+                                       win_left, win_right, w, cs)
+                 : launch_bwd_main<128>(*st, q, k, v, dout, dk, dv, B, Sq, Sk, H, scale, causal,
+                                        win_left, win_right, w, cs);
+}
+
+attn_status attn_bwd_dq_finalize(void* dq, int B, int Sq, int H, int D, float scale,
+                                 void* workspace, size_t workspace_size, void* stream) {
+  if (!dq) return ATTN_ERR_NULLPTR;
+  attn_status s = check_common(B, Sq, 1, H, D, scale, -1, -1);
+  if (s != ATTN_OK) return s;
+  if (!aligned16(dq)) return ATTN_ERR_ALIGN;
+  s = check_workspace(workspace, workspace_size, B, Sq, H, D);
+  if (s != ATTN_OK) return s;
+  DeviceState* st = nullptr;
+  s = device_state(&st);
+  if (s != ATTN_OK) return s;
+  if (!all_on_device({dq, workspace})) return ATTN_ERR_DEVICE;
+  const Workspace w = carve(workspace, B, Sq, H, D);
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  return D == 64 ? launch_bwd_dq<64>(dq, B, Sq, H, scale, w, cs)
+                 : launch_bwd_dq<128>(dq, B, Sq, H, scale, w, cs);
 }
 
 attn_status attn_get_last_device_error(void) {

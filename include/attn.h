@@ -116,6 +116,29 @@ ATTN_API attn_status attn_bwd(const void* q, const void* k, const void* v, const
                      int win_left, int win_right, void* workspace, size_t workspace_bytes,
                      void* stream);
 
+/*
+ * The three stages attn_bwd runs, in this order on one stream, exposed so a
+ * caller can place work (or timing events) between them.  Arguments mean the
+ * same as in attn_bwd; the stages communicate through `workspace`.
+ *
+ * attn_bwd_preprocess - Delta_i = sum_d dO_id O_id (float32), the LSE in base 2,
+ *   and a zeroed float32 dQ accumulator, all written into `workspace`.
+ * attn_bwd_main - for every 128-key tile: recomputes P from Q, K and the
+ *   workspace LSE, accumulates dV = P^T dO and dK = scale dS^T Q in tensor
+ *   memory and writes them (bf16), and adds dS K into the workspace dQ
+ *   accumulator with float32 atomic reductions.
+ * attn_bwd_dq_finalize - dq = bf16(scale * accumulator).
+ */
+ATTN_API attn_status attn_bwd_preprocess(const void* o, const void* dout, const float* lse,
+                                         int B, int Sq, int H, int D, void* workspace,
+                                         size_t workspace_bytes, void* stream);
+ATTN_API attn_status attn_bwd_main(const void* q, const void* k, const void* v, const void* dout,
+                                   void* dk, void* dv, int B, int Sq, int Sk, int H, int D,
+                                   float scale, int causal, int win_left, int win_right,
+                                   void* workspace, size_t workspace_bytes, void* stream);
+ATTN_API attn_status attn_bwd_dq_finalize(void* dq, int B, int Sq, int H, int D, float scale,
+                                          void* workspace, size_t workspace_bytes, void* stream);
+
 /* attn_status_string - static English text for a status code (never NULL). */
 ATTN_API const char* attn_status_string(attn_status s);
 

@@ -7,6 +7,7 @@ code with it.
 from .attn_ref import (  # noqa: F401
     attention_backward,
     attention_backward_head,
+    attention_backward_rows,
     attention_backward_rows_dq,
     attention_forward,
     attention_forward_rows,

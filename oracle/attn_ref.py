@@ -217,6 +217,25 @@ def attention_backward_rows_dq(q, k, v, do, triples, scale: float, causal: int =
     return dq, dl
 
 
+def attention_backward_rows(q, k, v, do, b: int, h: int, rows, scale: float,
+                            causal: int = 0, win_left: int = -1, win_right: int = -1):
+    """Forward and backward pieces owed to a set of query rows of one head.
+
+    Returns (o_rows, lse_rows, dq_rows, dk_part, dv_part): O, LSE and dQ of
+    the given rows, and the terms those rows add to dK and dV (sum over rows
+    of dS^T Q and P^T dO).  Summing dk_part/dv_part over a partition of the
+    rows gives the head's dK and dV.
+    """
+    rows = np.asarray(rows, dtype=np.int64)
+    Sq = q.shape[1]
+    Sk = k.shape[1]
+    kh, vh = _f64(k[b, :, h]), _f64(v[b, :, h])
+    qh, doh = _f64(q[b, rows, h]), _f64(do[b, rows, h])
+    O, lse, _, P, dS = _head_backward(qh, kh, vh, doh, scale, rows, Sq, Sk,
+                                      causal, win_left, win_right)
+    return O, lse, scale * (dS @ kh), scale * (dS.T @ qh), P.T @ doh
+
+
 def attention_backward_head(q, k, v, do, b: int, h: int, scale: float,
                             causal: int = 0, win_left: int = -1, win_right: int = -1,
                             row_chunk: int = 1024):
@@ -227,16 +246,15 @@ def attention_backward_head(q, k, v, do, b: int, h: int, scale: float,
     """
     Sq = q.shape[1]
     Sk = k.shape[1]
-    kh, vh = _f64(k[b, :, h]), _f64(v[b, :, h])
-    dk = np.zeros_like(kh)
-    dv = np.zeros_like(vh)
+    D = k.shape[3]
+    dk = np.zeros((Sk, D))
+    dv = np.zeros((Sk, D))
     for r0 in range(0, Sq, row_chunk):
         rows = np.arange(r0, min(Sq, r0 + row_chunk))
-        qh, doh = _f64(q[b, rows, h]), _f64(do[b, rows, h])
-        _, _, _, P, dS = _head_backward(qh, kh, vh, doh, scale, rows, Sq, Sk,
-                                        causal, win_left, win_right)
-        dv += P.T @ doh
-        dk += scale * (dS.T @ qh)
+        _, _, _, dkp, dvp = attention_backward_rows(q, k, v, do, b, h, rows, scale,
+                                                    causal, win_left, win_right)
+        dk += dkp
+        dv += dvp
     return dk, dv
 
 

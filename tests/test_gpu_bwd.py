@@ -46,8 +46,10 @@ def test_backward_full_tensor(case):
     ref = oracle.attention_backward(f64(bits["q"]), f64(bits["k"]), f64(bits["v"]),
                                     f64(bits["do"]), scale, causal, wl, wr)
     check_fwd(to_f64(o), lse.cpu().numpy().astype(np.float64), ref["o"], ref["lse"], str(case))
+    # floor: 1e-3 of the largest gradient magnitude of the problem
+    floor = 1e-3 * max(np.abs(ref[n]).max() for n in ("dq", "dk", "dv"))
     for name, g in (("dq", dq), ("dk", dk), ("dv", dv)):
-        check_grad(to_f64(g), ref[name], f"{case} {name}")
+        check_grad(to_f64(g), ref[name], f"{case} {name}", floor)
 
 
 def test_config_h32_s8192_fwd_bwd_sampled():
