@@ -45,6 +45,13 @@ cudaError_t set_smem(K kernel, int bytes) {
   return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
 }
 
+template <typename K>
+int regs_of(K kernel) {
+  cudaFuncAttributes a;
+  if (cudaFuncGetAttributes(&a, kernel) != cudaSuccess) return -1;
+  return a.numRegs;
+}
+
 // One-time per-device set-up: architecture check, error-word address, kernel attributes.
 attn_status device_state(DeviceState** out) {
   int dev = 0;
@@ -66,6 +73,14 @@ attn_status device_state(DeviceState** out) {
           set_smem(fwd::attn_fwd_kernel<128>, fwd::Cfg<128>::kSmemBytes) != cudaSuccess ||
           set_smem(bwd::attn_bwd_main_kernel<64>, bwd::Cfg<64>::kSmemBytes) != cudaSuccess ||
           set_smem(bwd::attn_bwd_main_kernel<128>, bwd::Cfg<128>::kSmemBytes) != cudaSuccess)
+        return ATTN_ERR_LAUNCH;
+      // The warp-specialised kernels hand registers between warpgroups with
+      // setmaxnreg; the split is sized for exactly kLaunchRegs per thread at
+      // launch.  Refuse to launch a build whose allocation differs.
+      if (regs_of(fwd::attn_fwd_kernel<64>) != fwd::kLaunchRegs ||
+          regs_of(fwd::attn_fwd_kernel<128>) != fwd::kLaunchRegs ||
+          regs_of(bwd::attn_bwd_main_kernel<64>) != bwd::kLaunchRegs ||
+          regs_of(bwd::attn_bwd_main_kernel<128>) != bwd::kLaunchRegs)
         return ATTN_ERR_LAUNCH;
       if (g_encode == nullptr) {
         void* fn = nullptr;
@@ -122,6 +137,20 @@ attn_status make_map(CUtensorMap* map, const void* base, int B, int S, int H, in
   const cuuint32_t estr[4] = {1, 1, 1, 1};
   const CUresult r =
       g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides,
+               box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? ATTN_OK : ATTN_ERR_LAUNCH;
+}
+
+// 2-D fp32 map over the dQ accumulator [rows][D], box = 32 x 128, 128-byte swizzle
+// (the layout the backward's drain warps stage a dQ tile in).
+attn_status make_dq_map(CUtensorMap* map, const float* base, long long rows, int D) {
+  const cuuint64_t dims[2] = {cuuint64_t(D), cuuint64_t(rows)};
+  const cuuint64_t strides[1] = {cuuint64_t(D) * 4};
+  const cuuint32_t box[2] = {32, 128};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r =
+      g_encode(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(base), dims, strides,
                box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? ATTN_OK : ATTN_ERR_LAUNCH;
@@ -194,9 +223,10 @@ attn_status launch_bwd_main(const DeviceState& st, const void* q, const void* k,
                             const void* dout, void* dk, void* dv, int B, int Sq, int Sk, int H,
                             float scale, int causal, int win_left, int win_right,
                             const Workspace& w, cudaStream_t stream) {
-  alignas(64) CUtensorMap mq, mk, mv, mdo;
+  alignas(64) CUtensorMap mq, mk, mv, mdo, mdq;
   if (make_map(&mq, q, B, Sq, H, D) != ATTN_OK || make_map(&mk, k, B, Sk, H, D) != ATTN_OK ||
-      make_map(&mv, v, B, Sk, H, D) != ATTN_OK || make_map(&mdo, dout, B, Sq, H, D) != ATTN_OK)
+      make_map(&mv, v, B, Sk, H, D) != ATTN_OK || make_map(&mdo, dout, B, Sq, H, D) != ATTN_OK ||
+      make_dq_map(&mdq, w.dq_acc, (long long)B * H * w.Sq_pad, D) != ATTN_OK)
     return ATTN_ERR_LAUNCH;
   bwd::Params p;
   p.dk = static_cast<__nv_bfloat16*>(dk);
@@ -218,7 +248,7 @@ attn_status launch_bwd_main(const DeviceState& st, const void* q, const void* k,
   p.timeout_ns = kTimeoutNs;
   dim3 grid((Sk + bwd::BN - 1) / bwd::BN, H, B);
   bwd::attn_bwd_main_kernel<D>
-      <<<grid, bwd::kThreads, bwd::Cfg<D>::kSmemBytes, stream>>>(mq, mk, mv, mdo, p);
+      <<<grid, bwd::kThreads, bwd::Cfg<D>::kSmemBytes, stream>>>(mq, mk, mv, mdo, mdq, p);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_LAUNCH;
 }
 

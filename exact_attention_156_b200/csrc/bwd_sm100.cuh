@@ -38,11 +38,19 @@ namespace bwd {
 
 constexpr int BM = 128;  // query rows per tile
 constexpr int BN = 128;  // key rows per CTA
-constexpr int kThreads = 320;
+constexpr int kThreads = 384;  // compute WG, dQ-drain WG, control WG {MMA, TMA, 2 idle}
 constexpr int kDrainWarp0 = 4;
 constexpr int kMmaWarp = 8;
 constexpr int kLoadWarp = 9;
 constexpr int kStages = 2;
+// Register split after launch (168 per thread at launch: 384 x 168 = 64512):
+// compute 128 x 240 + drain 128 x 136 + control 128 x 80 = 58368.
+constexpr int kLaunchRegs = 168;
+constexpr int kComputeRegs = 240;
+constexpr int kDrainRegs = 136;
+constexpr int kControlRegs = 80;
+static_assert(128 * (kComputeRegs + kDrainRegs + kControlRegs) <= kThreads * kLaunchRegs,
+              "register split exceeds the launch allocation");
 
 template <int D>
 struct Cfg {
@@ -51,11 +59,13 @@ struct Cfg {
   static constexpr int kTileBytes = 128 * D * 2;
   static constexpr int kKOff = 0;
   static constexpr int kVOff = kKOff + kTileBytes;
-  static constexpr int kQOff = kVOff + kTileBytes;
-  static constexpr int kDOOff = kQOff + kStages * kTileBytes;
-  static constexpr int kDSOff = kDOOff + kStages * kTileBytes;  // dS^T, 128 x 128 bf16
-  static constexpr int kLseOff = kDSOff + BN * BM * 2;          // [kStages][BM] fp32
-  static constexpr int kDeltaOff = kLseOff + kStages * BM * 4;  // [kStages][BM] fp32
+  // stage s = [Q_s | dO_s]; once the MMAs of a stage are done, the whole stage
+  // (128 x D fp32 bytes) holds the dQ tile on its way to the TMA reduce-add.
+  static constexpr int kStageOff = kVOff + kTileBytes;
+  static constexpr int kStageBytes = 2 * kTileBytes;
+  static constexpr int kDSOff = kStageOff + kStages * kStageBytes;  // dS^T, 128 x 128 bf16
+  static constexpr int kLseOff = kDSOff + BN * BM * 2;             // [kStages][BM] fp32
+  static constexpr int kDeltaOff = kLseOff + kStages * BM * 4;     // [kStages][BM] fp32
   static constexpr int kBarOff = kDeltaOff + kStages * BM * 4;
   static constexpr int kBarKV = 0;
   static constexpr int kBarFull = 1;
@@ -75,6 +85,7 @@ struct Cfg {
   static constexpr uint32_t kColDV = D;
   static constexpr uint32_t kColS = 2 * D;
   static constexpr uint32_t kColDP = 2 * D + 128;
+  static_assert(kStageBytes == BM * D * 4, "a stage must hold one fp32 dQ tile");
 };
 
 struct Params {
@@ -198,7 +209,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     attn_bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ,
                          const __grid_constant__ CUtensorMap tmK,
                          const __grid_constant__ CUtensorMap tmV,
-                         const __grid_constant__ CUtensorMap tmDO, const Params p) {
+                         const __grid_constant__ CUtensorMap tmDO,
+                         const __grid_constant__ CUtensorMap tmDQ, const Params p) {
   using C = Cfg<D>;
   extern __shared__ __align__(1024) uint8_t smem[];
   const int warp = threadIdx.x / 32;
@@ -242,13 +254,224 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   Bounded bw{abort_flag, p.err, p.timeout_ns};
-  auto q_addr = [&](int s) { return sbase + C::kQOff + s * C::kTileBytes; };
-  auto do_addr = [&](int s) { return sbase + C::kDOOff + s * C::kTileBytes; };
+  auto stage_addr = [&](int s) { return sbase + C::kStageOff + s * C::kStageBytes; };
+  auto q_addr = [&](int s) { return stage_addr(s); };
+  auto do_addr = [&](int s) { return stage_addr(s) + C::kTileBytes; };
   const uint32_t k_addr = sbase + C::kKOff;
   const uint32_t v_addr = sbase + C::kVOff;
   const uint32_t ds_addr = sbase + C::kDSOff;
   int load_count[kStages] = {0, 0};
+  bool drain_issued = false;
 
+  // ------------------------------------------------------------ teardown
+  // Inlined at the end of every role (each role returns after it), so that
+  // each role's code is register-allocated on its own.
+  auto finish = [&]() {
+    __syncwarp();
+    tc_fence_before();
+    __syncthreads();
+    if (*abort_flag) {
+      const uint64_t drain_ns = 2000000000ull;
+      if (warp == kLoadWarp && lane == 0 && nq > 0) {
+        for (int s = 0; s < kStages; ++s) {
+          if (load_count[s] == 0) continue;
+          const uint64_t t0 = globaltimer_ns();
+          while (!mbar_try_wait(bar(C::kBarFull + s), (load_count[s] - 1) & 1))
+            if (globaltimer_ns() - t0 > drain_ns) break;
+        }
+        const uint64_t t0 = globaltimer_ns();
+        while (!mbar_try_wait(bar(C::kBarKV), 0))
+          if (globaltimer_ns() - t0 > drain_ns) break;
+      }
+      if (warp == kMmaWarp && lane == 0) {
+        tc_commit(bar(C::kBarDone));
+        const uint64_t t0 = globaltimer_ns();
+        while (!mbar_try_wait(bar(C::kBarDone), 0))
+          if (globaltimer_ns() - t0 > drain_ns) break;
+      }
+      tc_fence_before();
+      __syncthreads();
+    }
+    if (warp == 0) {
+      tc_fence_after();
+      tmem_dealloc(tmem, 512);
+    }
+  };
+
+  if (warp < kDrainWarp0) {
+    regs_inc<kComputeRegs>();
+    // ------------------------------------------------------------ P and dS
+    const int quad = warp % 4;
+    const int r = quad * 32 + lane;  // key row within the tile
+    const int kk_idx = n0 + r;       // key index
+    const uint32_t lane_off = uint32_t(quad * 32) << 16;
+    const uint32_t tS = tmem + lane_off + C::kColS;
+    const uint32_t tDP = tmem + lane_off + C::kColDP;
+    const float sl2 = p.scale_log2;
+    const int qmin_k = g.qmin(kk_idx);
+    const int qmax_k = min(g.qmax(kk_idx), p.Sq - 1);
+    const bool key_ok = kk_idx < p.Sk;
+    // rows of the dS^T buffer: 128 bytes per 64 columns, 16-byte chunks swizzled by row % 8
+    const uint32_t ds_row = ds_addr + uint32_t(r) * 128;
+    const uint32_t sw = uint32_t(r & 7);
+    bool ok = true;
+    for (int t = 0; t < nq; ++t) {
+      const int s = t % kStages;
+      const int i0 = (qlo + t) * BM;
+      const float4* lse2 = reinterpret_cast<const float4*>(smem + C::kLseOff + s * BM * 4);
+      const float4* dlt = reinterpret_cast<const float4*>(smem + C::kDeltaOff + s * BM * 4);
+      if (!bw.wait_warp(bar(C::kBarS), t & 1, 27)) { ok = false; break; }
+      tc_fence_after();
+      float pr[BM];
+      {
+        uint32_t rr[BM];
+        tmem_ld128(tS, rr);
+#pragma unroll
+        for (int c = 0; c < BM; c += 4) {
+          const float4 l4 = lse2[c / 4];
+          pr[c + 0] = ex2_approx(fmaf(__uint_as_float(rr[c + 0]), sl2, -l4.x));
+          pr[c + 1] = ex2_approx(fmaf(__uint_as_float(rr[c + 1]), sl2, -l4.y));
+          pr[c + 2] = ex2_approx(fmaf(__uint_as_float(rr[c + 2]), sl2, -l4.z));
+          pr[c + 3] = ex2_approx(fmaf(__uint_as_float(rr[c + 3]), sl2, -l4.w));
+        }
+      }
+      const bool full = key_ok && n0 + BN - 1 <= p.Sk - 1 && i0 + BM - 1 <= p.Sq - 1 &&
+                        i0 >= g.qmin(n0 + BN - 1) && i0 + BM - 1 <= g.qmax(n0);
+      if (!full) {
+        const int c_lo = key_ok ? qmin_k - i0 : (1 << 30);
+        const int c_hi = qmax_k - i0;
+#pragma unroll
+        for (int c = 0; c < BM; ++c)
+          if (c < c_lo || c > c_hi) pr[c] = 0.f;
+      }
+      {
+        uint32_t w[BM / 2];
+#pragma unroll
+        for (int c = 0; c < BM / 2; ++c) w[c] = pack_bf16x2(pr[2 * c], pr[2 * c + 1]);
+        tmem_st64(tS, w);
+      }
+      tc_fence_before();
+      mbar_arrive(bar(C::kBarP));
+
+      if (!bw.wait_warp(bar(C::kBarDP), t & 1, 28)) { ok = false; break; }
+      if (t > 0 && !bw.wait_warp(bar(C::kBarDSEmpty), (t - 1) & 1, 29)) { ok = false; break; }
+      tc_fence_after();
+#pragma unroll
+      for (int c0 = 0; c0 < BM; c0 += 64) {
+        uint32_t rr[64];
+        tmem_ld64(tDP + c0, rr);
+#pragma unroll
+        for (int cc = 0; cc < 64; cc += 8) {
+          const float4 d0 = dlt[(c0 + cc) / 4];
+          const float4 d1 = dlt[(c0 + cc) / 4 + 1];
+          const float dl[8] = {d0.x, d0.y, d0.z, d0.w, d1.x, d1.y, d1.z, d1.w};
+          uint32_t w[4];
+#pragma unroll
+          for (int e = 0; e < 8; e += 2) {
+            const float a0 = pr[c0 + cc + e] * (__uint_as_float(rr[cc + e]) - dl[e]);
+            const float a1 = pr[c0 + cc + e + 1] * (__uint_as_float(rr[cc + e + 1]) - dl[e + 1]);
+            w[e / 2] = pack_bf16x2(a0, a1);
+          }
+          const int col = c0 + cc;  // first of 8 columns in this 16-byte chunk
+          const uint32_t box = uint32_t(col / 64);
+          const uint32_t chunk = uint32_t((col % 64) / 8);
+          st_shared_v4(ds_row + box * C::kBoxBytes + ((chunk ^ sw) << 4), w[0], w[1], w[2], w[3]);
+        }
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(bar(C::kBarDS));
+    }
+    // epilogue: dK = scale * acc, dV = acc (bf16)
+    if (ok && nq > 0) ok = bw.wait_warp(bar(C::kBarDQFull), (nq - 1) & 1, 30);
+    if (ok) {
+      tc_fence_after();
+      const size_t orow = ((size_t(b) * p.Sk + size_t(kk_idx)) * p.H + h) * D;
+#pragma unroll 1
+      for (int which = 0; which < 2; ++which) {
+        const uint32_t col = which == 0 ? C::kColDK : C::kColDV;
+        const float mul = which == 0 ? p.scale : 1.0f;
+        __nv_bfloat16* outp = which == 0 ? p.dk : p.dv;
+#pragma unroll 1
+        for (int c0 = 0; c0 < D; c0 += 32) {
+          uint32_t rr[32];
+          if (nq > 0) {
+            tmem_ld32(tmem + lane_off + col + c0, rr);
+          } else {
+#pragma unroll
+            for (int c = 0; c < 32; ++c) rr[c] = 0u;
+          }
+          uint32_t w[16];
+#pragma unroll
+          for (int c = 0; c < 16; ++c)
+            w[c] = pack_bf16x2(__uint_as_float(rr[2 * c]) * mul, __uint_as_float(rr[2 * c + 1]) * mul);
+          if (key_ok) {
+            uint8_t* dst = reinterpret_cast<uint8_t*>(outp + orow + c0);
+#pragma unroll
+            for (int v = 0; v < 4; ++v)
+              st_global_v4(dst + 16 * v, w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
+          }
+        }
+      }
+    }
+    finish();
+    return;
+  }
+  if (warp < kMmaWarp) {
+    regs_dec<kDrainRegs>();
+    // ------------------------------------------------------------ dQ drain
+    // TMEM -> registers -> the finished Q/dO stage (as four 128x32 fp32 boxes,
+    // 128-byte swizzle) -> one TMA reduce-add per box into the fp32 accumulator.
+    const int quad = warp % 4;
+    const int r = quad * 32 + lane;  // query row within the tile
+    const uint32_t tDQ = tmem + (uint32_t(quad * 32) << 16) + C::kColDP;
+    const uint32_t sw = uint32_t(r & 7);
+    const bool leader = (warp == kDrainWarp0 && lane == 0);
+    if (leader) tma_prefetch_desc(&tmDQ);
+    for (int t = 0; t < nq; ++t) {
+      const int s = t % kStages;
+      // all four drain warps continue or stop together (they meet at named barriers)
+      if (!named_bar_and(1, 128, bw.wait(bar(C::kBarDQFull), t & 1, 31))) break;
+      tc_fence_after();
+      const uint32_t stg = stage_addr(s) + uint32_t(r) * 128;
+      auto stage_cols = [&](const uint32_t(&rr)[64], int c_base) {
+#pragma unroll
+        for (int c = 0; c < 64; c += 4) {
+          const int col = c_base + c;
+          const uint32_t box = uint32_t(col / 32);
+          const uint32_t chunk = uint32_t((col % 32) / 4);
+          st_shared_v4(stg + box * (128 * 128) + ((chunk ^ sw) << 4), rr[c], rr[c + 1],
+                       rr[c + 2], rr[c + 3]);
+        }
+      };
+      uint32_t rr[64];
+      tmem_ld64(tDQ, rr);
+      if constexpr (D == 128) {
+        stage_cols(rr, 0);
+        tmem_ld64(tDQ + 64, rr);
+      }
+      // tensor memory is free again: the MMA warp may start dP of the next tile
+      tc_fence_before();
+      mbar_arrive(bar(C::kBarDQEmpty));
+      stage_cols(rr, D - 64);
+      fence_proxy_async_smem();
+      named_bar_sync(1, 128);
+      if (leader) {
+        const int row0 = bh * p.Sq_pad + (qlo + t) * BM;
+#pragma unroll
+        for (int box = 0; box < D / 32; ++box)
+          tma_reduce_add_2d(&tmDQ, stage_addr(s) + box * (128 * 128), box * 32, row0);
+        bulk_commit();
+        bulk_wait_read_all();  // the stage may be refilled once the reduce has read it
+        mbar_arrive(bar(C::kBarEmpty + s));
+        drain_issued = true;
+      }
+    }
+    if (leader && drain_issued) bulk_wait_all();
+    finish();
+    return;
+  }
+  regs_dec<kControlRegs>();
   if (warp == kLoadWarp) {
     // ------------------------------------------------------------ loads
     if (lane == 0 && nq > 0) {
@@ -337,7 +560,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                       sdesc_sw128(k_addr + kk * 16 * 128, C::kBoxBytes), id_dq,
                       kk > 0 ? 1u : 0u);
         tc_commit(bar(C::kBarDQFull));
-        tc_commit(bar(C::kBarEmpty + s));
         tc_commit(bar(C::kBarDSEmpty));
         if (more) {
           if (!bw.wait(bar(C::kBarDQEmpty), t & 1, 26)) { ok = false; break; }
@@ -347,172 +569,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
-  } else if (warp < kDrainWarp0) {
-    // ------------------------------------------------------------ P and dS
-    const int quad = warp % 4;
-    const int r = quad * 32 + lane;  // key row within the tile
-    const int kk_idx = n0 + r;       // key index
-    const uint32_t lane_off = uint32_t(quad * 32) << 16;
-    const uint32_t tS = tmem + lane_off + C::kColS;
-    const uint32_t tDP = tmem + lane_off + C::kColDP;
-    const float sl2 = p.scale_log2;
-    const int qmin_k = g.qmin(kk_idx);
-    const int qmax_k = min(g.qmax(kk_idx), p.Sq - 1);
-    const bool key_ok = kk_idx < p.Sk;
-    // rows of the dS^T buffer: 128 bytes per 64 columns, 16-byte chunks swizzled by row % 8
-    const uint32_t ds_row = ds_addr + uint32_t(r) * 128;
-    const uint32_t sw = uint32_t(r & 7);
-    bool ok = true;
-    for (int t = 0; t < nq; ++t) {
-      const int s = t % kStages;
-      const int i0 = (qlo + t) * BM;
-      const float* lse2 = reinterpret_cast<const float*>(smem + C::kLseOff + s * BM * 4);
-      const float* dlt = reinterpret_cast<const float*>(smem + C::kDeltaOff + s * BM * 4);
-      if (!bw.wait_warp(bar(C::kBarS), t & 1, 27)) { ok = false; break; }
-      tc_fence_after();
-      float pr[BM];
-#pragma unroll
-      for (int c0 = 0; c0 < BM; c0 += 32) {
-        uint32_t rr[32];
-        tmem_ld32(tS + c0, rr);
-#pragma unroll
-        for (int c = 0; c < 32; ++c)
-          pr[c0 + c] = ex2_approx(fmaf(__uint_as_float(rr[c]), sl2, -lse2[c0 + c]));
-      }
-      const bool full = key_ok && n0 + BN - 1 <= p.Sk - 1 && i0 + BM - 1 <= p.Sq - 1 &&
-                        i0 >= g.qmin(n0 + BN - 1) && i0 + BM - 1 <= g.qmax(n0);
-      if (!full) {
-        const int c_lo = key_ok ? qmin_k - i0 : (1 << 30);
-        const int c_hi = qmax_k - i0;
-#pragma unroll
-        for (int c = 0; c < BM; ++c)
-          if (c < c_lo || c > c_hi) pr[c] = 0.f;
-      }
-      {
-        uint32_t w[32];
-#pragma unroll
-        for (int c = 0; c < 32; ++c) w[c] = pack_bf16x2(pr[2 * c], pr[2 * c + 1]);
-        tmem_st32(tS, w);
-#pragma unroll
-        for (int c = 0; c < 32; ++c) w[c] = pack_bf16x2(pr[64 + 2 * c], pr[64 + 2 * c + 1]);
-        tmem_st32(tS + 32, w);
-      }
-      tc_fence_before();
-      mbar_arrive(bar(C::kBarP));
-
-      if (!bw.wait_warp(bar(C::kBarDP), t & 1, 28)) { ok = false; break; }
-      if (t > 0 && !bw.wait_warp(bar(C::kBarDSEmpty), (t - 1) & 1, 29)) { ok = false; break; }
-      tc_fence_after();
-#pragma unroll
-      for (int c0 = 0; c0 < BM; c0 += 32) {
-        uint32_t rr[32];
-        tmem_ld32(tDP + c0, rr);
-        uint32_t w[16];
-#pragma unroll
-        for (int c = 0; c < 32; c += 2) {
-          const float d0 = pr[c0 + c] * (__uint_as_float(rr[c]) - dlt[c0 + c]);
-          const float d1 = pr[c0 + c + 1] * (__uint_as_float(rr[c + 1]) - dlt[c0 + c + 1]);
-          w[c / 2] = pack_bf16x2(d0, d1);
-        }
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int col = c0 + 8 * q;            // first of 8 columns in this chunk
-          const uint32_t box = uint32_t(col / 64);
-          const uint32_t chunk = uint32_t((col % 64) / 8);
-          st_shared_v4(ds_row + box * C::kBoxBytes + ((chunk ^ sw) << 4), w[4 * q], w[4 * q + 1],
-                       w[4 * q + 2], w[4 * q + 3]);
-        }
-      }
-      fence_proxy_async_smem();
-      tc_fence_before();
-      mbar_arrive(bar(C::kBarDS));
-    }
-    // epilogue: dK = scale * acc, dV = acc (bf16)
-    if (ok && nq > 0) ok = bw.wait_warp(bar(C::kBarDQFull), (nq - 1) & 1, 30);
-    if (ok) {
-      tc_fence_after();
-      const size_t orow = ((size_t(b) * p.Sk + size_t(kk_idx)) * p.H + h) * D;
-#pragma unroll 1
-      for (int which = 0; which < 2; ++which) {
-        const uint32_t col = which == 0 ? C::kColDK : C::kColDV;
-        const float mul = which == 0 ? p.scale : 1.0f;
-        __nv_bfloat16* outp = which == 0 ? p.dk : p.dv;
-#pragma unroll 1
-        for (int c0 = 0; c0 < D; c0 += 32) {
-          uint32_t rr[32];
-          if (nq > 0) {
-            tmem_ld32(tmem + lane_off + col + c0, rr);
-          } else {
-#pragma unroll
-            for (int c = 0; c < 32; ++c) rr[c] = 0u;
-          }
-          uint32_t w[16];
-#pragma unroll
-          for (int c = 0; c < 16; ++c)
-            w[c] = pack_bf16x2(__uint_as_float(rr[2 * c]) * mul, __uint_as_float(rr[2 * c + 1]) * mul);
-          if (key_ok) {
-            uint8_t* dst = reinterpret_cast<uint8_t*>(outp + orow + c0);
-#pragma unroll
-            for (int v = 0; v < 4; ++v)
-              st_global_v4(dst + 16 * v, w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
-          }
-        }
-      }
-    }
-  } else if (warp < kMmaWarp) {
-    // ------------------------------------------------------------ dQ drain
-    const int quad = warp % 4;
-    const int r = quad * 32 + lane;  // query row within the tile
-    const uint32_t tDQ = tmem + (uint32_t(quad * 32) << 16) + C::kColDP;
-    for (int t = 0; t < nq; ++t) {
-      const int i = (qlo + t) * BM + r;
-      if (!bw.wait_warp(bar(C::kBarDQFull), t & 1, 31)) break;
-      tc_fence_after();
-      float* dst = p.dq_acc + (size_t(bh) * p.Sq_pad + i) * D;
-#pragma unroll
-      for (int c0 = 0; c0 < D; c0 += 32) {
-        uint32_t rr[32];
-        tmem_ld32(tDQ + c0, rr);
-#pragma unroll
-        for (int v = 0; v < 8; ++v)
-          red_add_v4(dst + c0 + 4 * v, __uint_as_float(rr[4 * v]), __uint_as_float(rr[4 * v + 1]),
-                     __uint_as_float(rr[4 * v + 2]), __uint_as_float(rr[4 * v + 3]));
-      }
-      tc_fence_before();
-      mbar_arrive(bar(C::kBarDQEmpty));
-    }
   }
-
-  // ------------------------------------------------------------ teardown
-  __syncwarp();
-  tc_fence_before();
-  __syncthreads();
-  if (*abort_flag) {
-    const uint64_t drain_ns = 2000000000ull;
-    if (warp == kLoadWarp && lane == 0 && nq > 0) {
-      for (int s = 0; s < kStages; ++s) {
-        if (load_count[s] == 0) continue;
-        const uint64_t t0 = globaltimer_ns();
-        while (!mbar_try_wait(bar(C::kBarFull + s), (load_count[s] - 1) & 1))
-          if (globaltimer_ns() - t0 > drain_ns) break;
-      }
-      const uint64_t t0 = globaltimer_ns();
-      while (!mbar_try_wait(bar(C::kBarKV), 0))
-        if (globaltimer_ns() - t0 > drain_ns) break;
-    }
-    if (warp == kMmaWarp && lane == 0) {
-      tc_commit(bar(C::kBarDone));
-      const uint64_t t0 = globaltimer_ns();
-      while (!mbar_try_wait(bar(C::kBarDone), 0))
-        if (globaltimer_ns() - t0 > drain_ns) break;
-    }
-    tc_fence_before();
-    __syncthreads();
-  }
-  if (warp == 0) {
-    tc_fence_after();
-    tmem_dealloc(tmem, 512);
-  }
+  finish();
 }
 
 }  // namespace bwd

@@ -14,6 +14,8 @@
 //    memory, and O_k += P_k V_j with P_k read from tensor memory.  The order
 //    PV_0(j), S_0(j+1), PV_1(j), S_1(j+1) lets the softmax of one tile overlap
 //    the tensor-core work of the other.
+//  * warps 10-11 idle; after set-up the control warpgroup (8-11) gives registers
+//    to the two softmax warpgroups (setmaxnreg).
 //  * warps 0-3 / 4-7: softmax of tile 0 / tile 1; one thread owns one query row
 //    (= one TMEM lane), so the row max and row sum need no shuffles.  Scores
 //    are scaled by scale*log2(e) and exponentiated with ex2.  The running max
@@ -36,9 +38,16 @@ namespace fwd {
 constexpr int BM = 128;  // query rows per tile (= TMEM lanes)
 constexpr int BN = 128;  // keys per K/V tile
 constexpr int NQ = 2;    // query tiles per CTA
-constexpr int kThreads = 320;
+constexpr int kThreads = 384;  // 3 warpgroups: softmax 0, softmax 1, {MMA, TMA, 2 idle}
 constexpr int kMmaWarp = 8;
 constexpr int kLoadWarp = 9;
+// Register split after launch (168 per thread at launch: 384 x 168 = 64512):
+// softmax warpgroups 2 x 128 x 216 + control warpgroup 128 x 64 = 63488.
+constexpr int kLaunchRegs = 168;
+constexpr int kSoftmaxRegs = 216;
+constexpr int kControlRegs = 64;
+static_assert(128 * (2 * kSoftmaxRegs + kControlRegs) <= kThreads * kLaunchRegs,
+              "register split exceeds the launch allocation");
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: p <= 2^8 between rescales
 
 template <int D>
@@ -157,6 +166,176 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
   for (int s = 0; s < C::kStages; ++s) load_count[s] = 0;
 
+  // ------------------------------------------------------------ teardown
+  // Inlined at the end of every role (each role returns after it), so that
+  // each role's code is register-allocated on its own.
+  auto finish = [&]() {
+    __syncwarp();
+    tc_fence_before();
+    __syncthreads();
+    if (*abort_flag) {
+      // Drain what may still be in flight before the shared and tensor memory go away.
+      const uint64_t drain_ns = 2000000000ull;
+      if (warp == kLoadWarp && lane == 0) {
+        for (int s = 0; s < C::kStages; ++s) {
+          if (load_count[s] == 0) continue;
+          const uint64_t t0 = globaltimer_ns();
+          while (!mbar_try_wait(bar(C::kBarFull + s), (load_count[s] - 1) & 1))
+            if (globaltimer_ns() - t0 > drain_ns) break;
+        }
+        if (any_work) {
+          const uint64_t t0 = globaltimer_ns();
+          while (!mbar_try_wait(bar(C::kBarQ), 0))
+            if (globaltimer_ns() - t0 > drain_ns) break;
+        }
+      }
+      if (warp == kMmaWarp && lane == 0) {
+        tc_commit(bar(C::kBarDone));
+        const uint64_t t0 = globaltimer_ns();
+        while (!mbar_try_wait(bar(C::kBarDone), 0))
+          if (globaltimer_ns() - t0 > drain_ns) break;
+      }
+      tc_fence_before();
+      __syncthreads();
+    }
+    if (warp == 0) {
+      tc_fence_after();
+      tmem_dealloc(tmem, 512);
+    }
+  };
+
+  if (warp < 8) {
+    regs_inc<kSoftmaxRegs>();
+    // ------------------------------------------------------------ softmax + epilogue
+    const int k = warp / 4;            // query tile of this warpgroup
+    const int quad = warp % 4;         // TMEM lane quadrant
+    const int row = quad * 32 + lane;  // row within the tile
+    const int i = r0[k] + row;         // query index
+    const int n_k = jhi[k] - jlo[k];
+    const uint32_t lane_off = uint32_t(quad * 32) << 16;
+    const uint32_t tS = tmem + lane_off + C::col_s(k);
+    const uint32_t tO = tmem + lane_off + C::col_o(k);
+    const int lo_i = g.lo(i);
+    const int hi_i = g.hi(i);
+    const int r1 = min(r0[k] + BM - 1, p.Sq - 1);
+    const int tile_lo_max = g.lo(r1);  // largest row lower bound in this tile
+    const int tile_hi_min = g.hi(r0[k]);
+    const float sl2 = p.scale_log2;
+    float m_run = -INFINITY;
+    float l_run = 0.f;
+    bool ok = true;
+
+    for (int t = 0; t < n_k; ++t) {
+      const int j = jlo[k] + t;
+      if (!bw.wait_warp(bar(C::kBarS + k), t & 1, 10 + k)) { ok = false; break; }
+      tc_fence_after();
+      float s[BN];
+      {
+        uint32_t r[BN];
+        tmem_ld128(tS, r);
+#pragma unroll
+        for (int c = 0; c < BN; ++c) s[c] = __uint_as_float(r[c]);
+      }
+      const int n0 = j * BN;
+      const bool full = (n0 >= tile_lo_max) && (n0 + BN - 1 <= tile_hi_min);
+      if (!full) {
+        const int c_lo = lo_i - n0;
+        const int c_hi = hi_i - n0;
+#pragma unroll
+        for (int c = 0; c < BN; ++c)
+          if (c < c_lo || c > c_hi) s[c] = -INFINITY;
+      }
+      // row max as 8 independent chains, then a 3-level tree
+      float m8[8];
+#pragma unroll
+      for (int a = 0; a < 8; ++a) m8[a] = s[a];
+#pragma unroll
+      for (int c = 8; c < BN; ++c) m8[c % 8] = fmaxf(m8[c % 8], s[c]);
+      const float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                             fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+      const float m_cand = mx * sl2;
+      const bool bump = m_cand > m_run + kRescaleThreshold;
+      const float m_new = bump ? m_cand : m_run;
+      const float alpha = bump ? ex2_approx(m_run - m_new) : 1.0f;
+      const float m_eff = (m_new == -INFINITY) ? 0.0f : m_new;
+      float rs[8];
+#pragma unroll
+      for (int a = 0; a < 8; ++a) rs[a] = 0.f;
+      // P in two 64-column halves, each packed to bf16 pairs and stored to
+      // tensor memory (columns [0,32) and [32,64) of S_k) before the next half
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        uint32_t pk[32];
+#pragma unroll
+        for (int c = 0; c < 64; c += 2) {
+          const float p0 = ex2_approx(fmaf(s[half * 64 + c], sl2, -m_eff));
+          const float p1 = ex2_approx(fmaf(s[half * 64 + c + 1], sl2, -m_eff));
+          rs[(c / 2) % 8] += p0 + p1;
+          pk[c / 2] = pack_bf16x2(p0, p1);
+        }
+        tmem_st32(tS + half * 32, pk);
+      }
+      const float row_sum = ((rs[0] + rs[1]) + (rs[2] + rs[3])) + ((rs[4] + rs[5]) + (rs[6] + rs[7]));
+      l_run = l_run * alpha + row_sum;
+      m_run = m_new;
+      // Rescale O when this warp raised any row's max (rare after the first tile).
+      if (t > 0 && __any_sync(0xffffffffu, bump)) {
+        if (!bw.wait_warp(bar(C::kBarO + k), (t - 1) & 1, 12 + k)) { ok = false; break; }
+        tc_fence_after();
+#pragma unroll 1
+        for (int c0 = 0; c0 < D; c0 += 32) {
+          uint32_t r[32];
+          tmem_ld32(tO + c0, r);
+#pragma unroll
+          for (int c = 0; c < 32; ++c) r[c] = __float_as_uint(__uint_as_float(r[c]) * alpha);
+          tmem_st32(tO + c0, r);
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(bar(C::kBarP + k));
+    }
+
+    // Epilogue: O = O / l (bf16), LSE = (m + log2 l) ln 2.
+    if (valid[k] && ok) {
+      const bool row_ok = i < p.Sq;
+      const size_t orow = ((size_t(b) * p.Sq + size_t(i)) * p.H + h) * D;
+      if (n_k > 0) {
+        ok = bw.wait_warp(bar(C::kBarO + k), (n_k - 1) & 1, 14 + k);
+      }
+      if (ok) {
+        tc_fence_after();
+        const float inv_l = l_run > 0.f ? 1.0f / l_run : 0.0f;
+#pragma unroll 1
+        for (int c0 = 0; c0 < D; c0 += 32) {
+          uint32_t r[32];
+          if (n_k > 0) {
+            tmem_ld32(tO + c0, r);
+          } else {
+#pragma unroll
+            for (int c = 0; c < 32; ++c) r[c] = 0u;
+          }
+          uint32_t w[16];
+#pragma unroll
+          for (int c = 0; c < 16; ++c)
+            w[c] = pack_bf16x2(__uint_as_float(r[2 * c]) * inv_l, __uint_as_float(r[2 * c + 1]) * inv_l);
+          if (row_ok) {
+            uint8_t* dst = reinterpret_cast<uint8_t*>(p.o + orow + c0);
+#pragma unroll
+            for (int v = 0; v < 4; ++v)
+              st_global_v4(dst + 16 * v, w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
+          }
+        }
+        if (row_ok) {
+          const float lse = l_run > 0.f ? (m_run + __log2f(l_run)) * 0.69314718055994530942f : -INFINITY;
+          p.lse[(size_t(b) * p.H + h) * p.Sq + i] = lse;
+        }
+      }
+    }
+    finish();
+    return;
+  }
+
+  regs_dec<kControlRegs>();
   if (warp == kLoadWarp) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0 && any_work) {
@@ -256,164 +435,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
-  } else {
-    // ------------------------------------------------------------ softmax + epilogue
-    const int k = warp / 4;            // query tile of this warpgroup
-    const int quad = warp % 4;         // TMEM lane quadrant
-    const int row = quad * 32 + lane;  // row within the tile
-    const int i = r0[k] + row;         // query index
-    const int n_k = jhi[k] - jlo[k];
-    const uint32_t lane_off = uint32_t(quad * 32) << 16;
-    const uint32_t tS = tmem + lane_off + C::col_s(k);
-    const uint32_t tO = tmem + lane_off + C::col_o(k);
-    const int lo_i = g.lo(i);
-    const int hi_i = g.hi(i);
-    const int r1 = min(r0[k] + BM - 1, p.Sq - 1);
-    const int tile_lo_max = g.lo(r1);  // largest row lower bound in this tile
-    const int tile_hi_min = g.hi(r0[k]);
-    const float sl2 = p.scale_log2;
-    float m_run = -INFINITY;
-    float l_run = 0.f;
-    bool ok = true;
-
-    for (int t = 0; t < n_k; ++t) {
-      const int j = jlo[k] + t;
-      if (!bw.wait_warp(bar(C::kBarS + k), t & 1, 10 + k)) { ok = false; break; }
-      tc_fence_after();
-      float s[BN];
-#pragma unroll
-      for (int c0 = 0; c0 < BN; c0 += 32) {
-        uint32_t r[32];
-        tmem_ld32(tS + c0, r);
-#pragma unroll
-        for (int c = 0; c < 32; ++c) s[c0 + c] = __uint_as_float(r[c]);
-      }
-      const int n0 = j * BN;
-      const bool full = (n0 >= tile_lo_max) && (n0 + BN - 1 <= tile_hi_min);
-      if (!full) {
-        const int c_lo = lo_i - n0;
-        const int c_hi = hi_i - n0;
-#pragma unroll
-        for (int c = 0; c < BN; ++c)
-          if (c < c_lo || c > c_hi) s[c] = -INFINITY;
-      }
-      float mx = s[0];
-#pragma unroll
-      for (int c = 1; c < BN; ++c) mx = fmaxf(mx, s[c]);
-      const float m_cand = mx * sl2;
-      const bool bump = m_cand > m_run + kRescaleThreshold;
-      const float m_new = bump ? m_cand : m_run;
-      const float alpha = bump ? ex2_approx(m_run - m_new) : 1.0f;
-      const float m_eff = (m_new == -INFINITY) ? 0.0f : m_new;
-      float rs0 = 0.f, rs1 = 0.f;
-      uint32_t pk[BN / 2];
-#pragma unroll
-      for (int c = 0; c < BN; c += 2) {
-        const float p0 = ex2_approx(fmaf(s[c], sl2, -m_eff));
-        const float p1 = ex2_approx(fmaf(s[c + 1], sl2, -m_eff));
-        rs0 += p0;
-        rs1 += p1;
-        pk[c / 2] = pack_bf16x2(p0, p1);
-      }
-      l_run = l_run * alpha + (rs0 + rs1);
-      m_run = m_new;
-      // Rescale O when this warp raised any row's max (rare after the first tile).
-      if (t > 0 && __any_sync(0xffffffffu, bump)) {
-        if (!bw.wait_warp(bar(C::kBarO + k), (t - 1) & 1, 12 + k)) { ok = false; break; }
-        tc_fence_after();
-#pragma unroll 1
-        for (int c0 = 0; c0 < D; c0 += 32) {
-          uint32_t r[32];
-          tmem_ld32(tO + c0, r);
-#pragma unroll
-          for (int c = 0; c < 32; ++c) r[c] = __float_as_uint(__uint_as_float(r[c]) * alpha);
-          tmem_st32(tO + c0, r);
-        }
-      }
-      {
-        uint32_t r[32];
-#pragma unroll
-        for (int c = 0; c < 32; ++c) r[c] = pk[c];
-        tmem_st32(tS, r);
-#pragma unroll
-        for (int c = 0; c < 32; ++c) r[c] = pk[32 + c];
-        tmem_st32(tS + 32, r);
-      }
-      tc_fence_before();
-      mbar_arrive(bar(C::kBarP + k));
-    }
-
-    // Epilogue: O = O / l (bf16), LSE = (m + log2 l) ln 2.
-    if (valid[k] && ok) {
-      const bool row_ok = i < p.Sq;
-      const size_t orow = ((size_t(b) * p.Sq + size_t(i)) * p.H + h) * D;
-      if (n_k > 0) {
-        ok = bw.wait_warp(bar(C::kBarO + k), (n_k - 1) & 1, 14 + k);
-      }
-      if (ok) {
-        tc_fence_after();
-        const float inv_l = l_run > 0.f ? 1.0f / l_run : 0.0f;
-#pragma unroll 1
-        for (int c0 = 0; c0 < D; c0 += 32) {
-          uint32_t r[32];
-          if (n_k > 0) {
-            tmem_ld32(tO + c0, r);
-          } else {
-#pragma unroll
-            for (int c = 0; c < 32; ++c) r[c] = 0u;
-          }
-          uint32_t w[16];
-#pragma unroll
-          for (int c = 0; c < 16; ++c)
-            w[c] = pack_bf16x2(__uint_as_float(r[2 * c]) * inv_l, __uint_as_float(r[2 * c + 1]) * inv_l);
-          if (row_ok) {
-            uint8_t* dst = reinterpret_cast<uint8_t*>(p.o + orow + c0);
-#pragma unroll
-            for (int v = 0; v < 4; ++v)
-              st_global_v4(dst + 16 * v, w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
-          }
-        }
-        if (row_ok) {
-          const float lse = l_run > 0.f ? (m_run + __log2f(l_run)) * 0.69314718055994530942f : -INFINITY;
-          p.lse[(size_t(b) * p.H + h) * p.Sq + i] = lse;
-        }
-      }
-    }
   }
-
-  // ------------------------------------------------------------ teardown
-  __syncwarp();
-  tc_fence_before();
-  __syncthreads();
-  if (*abort_flag) {
-    // Drain what may still be in flight before the shared and tensor memory go away.
-    const uint64_t drain_ns = 2000000000ull;
-    if (warp == kLoadWarp && lane == 0) {
-      for (int s = 0; s < C::kStages; ++s) {
-        if (load_count[s] == 0) continue;
-        const uint64_t t0 = globaltimer_ns();
-        while (!mbar_try_wait(bar(C::kBarFull + s), (load_count[s] - 1) & 1))
-          if (globaltimer_ns() - t0 > drain_ns) break;
-      }
-      if (any_work) {
-        const uint64_t t0 = globaltimer_ns();
-        while (!mbar_try_wait(bar(C::kBarQ), 0))
-          if (globaltimer_ns() - t0 > drain_ns) break;
-      }
-    }
-    if (warp == kMmaWarp && lane == 0) {
-      tc_commit(bar(C::kBarDone));
-      const uint64_t t0 = globaltimer_ns();
-      while (!mbar_try_wait(bar(C::kBarDone), 0))
-        if (globaltimer_ns() - t0 > drain_ns) break;
-    }
-    tc_fence_before();
-    __syncthreads();
-  }
-  if (warp == 0) {
-    tc_fence_after();
-    tmem_dealloc(tmem, 512);
-  }
+  finish();
 }
 
 }  // namespace fwd
