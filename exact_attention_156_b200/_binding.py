@@ -19,6 +19,7 @@ ATTN_STATUS = {
     0: "ATTN_OK", 1: "ATTN_ERR_NULLPTR", 2: "ATTN_ERR_SHAPE", 3: "ATTN_ERR_HEADDIM",
     4: "ATTN_ERR_ALIGN", 5: "ATTN_ERR_WINDOW", 6: "ATTN_ERR_ARCH", 7: "ATTN_ERR_DEVICE",
     8: "ATTN_ERR_LAUNCH", 9: "ATTN_ERR_TIMEOUT", 10: "ATTN_ERR_WORKSPACE",
+    11: "ATTN_ERR_SCRATCH",
 }
 
 
@@ -47,6 +48,9 @@ def _load() -> ctypes.CDLL:
     lib.attn_bwd_main.restype = i
     lib.attn_bwd_dq_finalize.argtypes = [vp, i, i, i, i, f, vp, sz, vp]
     lib.attn_bwd_dq_finalize.restype = i
+    lib.attn_bwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, i,
+                                     i, vp]
+    lib.attn_bwd_noalloc.restype = i
     lib.attn_bwd_workspace_size.argtypes = [i, i, i, i]
     lib.attn_bwd_workspace_size.restype = sz
     lib.attn_status_string.argtypes = [i]

@@ -275,6 +275,36 @@ bool all_on_device(std::initializer_list<const void*> ptrs) {
   return true;
 }
 
+// ---------------------------------------------------------------------------
+// Scratch for attn_bwd_noalloc: one statically declared device array per GPU.
+// In host code `g_noalloc_scratch` is only a host-side stand-in for the
+// symbol, never a device address; its device address is looked up once per
+// device with cudaGetSymbolAddress (with that device current) and cached.
+// ---------------------------------------------------------------------------
+static __device__ __align__(256) uint8_t g_noalloc_scratch[ATTN_NOALLOC_SCRATCH_BYTES];
+
+struct ScratchState {
+  bool init = false;
+  void* ptr = nullptr;
+};
+ScratchState g_scratch[kMaxDevices];
+
+attn_status noalloc_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return ATTN_ERR_DEVICE;
+  std::lock_guard<std::mutex> lock(g_mu);
+  ScratchState& s = g_scratch[dev];
+  if (!s.init) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || ptr == nullptr)
+      return ATTN_ERR_LAUNCH;
+    s.ptr = ptr;
+    s.init = true;
+  }
+  *out = s.ptr;
+  return ATTN_OK;
+}
+
 __global__ void attn_timeout_selftest_kernel(uint32_t* err, uint64_t limit_ns) {
   __shared__ __align__(8) uint64_t bar;
   __shared__ int abort_flag;
@@ -306,6 +336,9 @@ const char* attn_status_string(attn_status s) {
     case ATTN_ERR_LAUNCH: return "a CUDA call failed (descriptor encoding or kernel launch)";
     case ATTN_ERR_TIMEOUT: return "a device-side bounded wait ran out";
     case ATTN_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    case ATTN_ERR_SCRATCH:
+      return "backward scratch for this problem exceeds the 64 MiB built into attn_bwd_noalloc "
+             "(call attn_bwd with a workspace instead)";
   }
   return "unknown status";
 }
@@ -431,6 +464,45 @@ attn_status attn_bwd_dq_finalize(void* dq, int B, int Sq, int H, int D, float sc
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
   return D == 64 ? launch_bwd_dq<64>(dq, B, Sq, H, scale, w, cs)
                  : launch_bwd_dq<128>(dq, B, Sq, H, scale, w, cs);
+}
+
+attn_status attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* o,
+                             const void* dout, const float* lse, void* dq, void* dk, void* dv,
+                             int B, int Sq, int Sk, int H, int D, float scale, int causal,
+                             int win_left, int win_right, void* stream) {
+  if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv) return ATTN_ERR_NULLPTR;
+  attn_status s = check_common(B, Sq, Sk, H, D, scale, win_left, win_right);
+  if (s != ATTN_OK) return s;
+  if (workspace_bytes(B, Sq, H, D) > ATTN_NOALLOC_SCRATCH_BYTES) return ATTN_ERR_SCRATCH;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) ||
+      !aligned16(dq) || !aligned16(dk) || !aligned16(dv) ||
+      (reinterpret_cast<uintptr_t>(lse) & 3u))
+    return ATTN_ERR_ALIGN;
+  DeviceState* st = nullptr;
+  s = device_state(&st);
+  if (s != ATTN_OK) return s;
+  if (!all_on_device({q, k, v, o, dout, lse, dq, dk, dv})) return ATTN_ERR_DEVICE;
+  void* scratch = nullptr;
+  s = noalloc_scratch(&scratch);
+  if (s != ATTN_OK) return s;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  // The preprocess kernel rewrites Delta and LSE rows and zeroes the dQ
+  // accumulator, so nothing left in the scratch by an earlier call is read.
+  const Workspace w = carve(scratch, B, Sq, H, D);
+  if (D == 64) {
+    s = launch_bwd_pre<64>(o, dout, lse, B, Sq, H, w, cs);
+    if (s == ATTN_OK)
+      s = launch_bwd_main<64>(*st, q, k, v, dout, dk, dv, B, Sq, Sk, H, scale, causal, win_left,
+                              win_right, w, cs);
+    if (s == ATTN_OK) s = launch_bwd_dq<64>(dq, B, Sq, H, scale, w, cs);
+  } else {
+    s = launch_bwd_pre<128>(o, dout, lse, B, Sq, H, w, cs);
+    if (s == ATTN_OK)
+      s = launch_bwd_main<128>(*st, q, k, v, dout, dk, dv, B, Sq, Sk, H, scale, causal, win_left,
+                               win_right, w, cs);
+    if (s == ATTN_OK) s = launch_bwd_dq<128>(dq, B, Sq, H, scale, w, cs);
+  }
+  return s;
 }
 
 attn_status attn_get_last_device_error(void) {

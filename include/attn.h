@@ -70,7 +70,8 @@ typedef enum {
     ATTN_ERR_DEVICE = 7,    /* a pointer is not device memory of the current GPU  */
     ATTN_ERR_LAUNCH = 8,    /* a CUDA call (descriptor build, launch) failed      */
     ATTN_ERR_TIMEOUT = 9,   /* a device-side bounded wait ran out                 */
-    ATTN_ERR_WORKSPACE = 10 /* workspace NULL, misaligned or smaller than needed  */
+    ATTN_ERR_WORKSPACE = 10, /* workspace NULL, misaligned or smaller than needed */
+    ATTN_ERR_SCRATCH = 11    /* problem too large for attn_bwd_noalloc's scratch  */
 } attn_status;
 
 /*
@@ -138,6 +139,37 @@ ATTN_API attn_status attn_bwd_main(const void* q, const void* k, const void* v, 
                                    void* workspace, size_t workspace_bytes, void* stream);
 ATTN_API attn_status attn_bwd_dq_finalize(void* dq, int B, int Sq, int H, int D, float scale,
                                           void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * attn_bwd_noalloc - attn_bwd for callers that cannot allocate device memory.
+ * The pages have no counterpart: this entry point exists only for callers that
+ * must not call cudaMalloc (or any allocator) at the moment they run the
+ * backward, e.g. code that owns no allocator of its own inside a host that
+ * manages all device memory, or latency-critical loops where an allocation
+ * would implicitly synchronise the device.
+ *
+ * Same arguments and results as attn_bwd, without the workspace: the backward
+ * scratch (the float32 dQ accumulator plus Delta and LSE rows) lives in one
+ * fixed array of ATTN_NOALLOC_SCRATCH_BYTES (64 MiB) of device memory that the
+ * library declares statically, so every GPU that loads the library holds it
+ * until the process exits.  This call allocates nothing and calls no allocator.
+ *
+ *  - Problems whose backward scratch, attn_bwd_workspace_size(B, Sq, H, D),
+ *    exceeds ATTN_NOALLOC_SCRATCH_BYTES are rejected with ATTN_ERR_SCRATCH
+ *    before anything is launched; use attn_bwd with a workspace for those.
+ *  - The first call on a device looks up the array's device address for that
+ *    device (a one-time set-up per device); make that first call before any
+ *    stream capture.
+ *  - Every call, on every stream, shares the one array, and it keeps the last
+ *    call's contents (each call re-initialises what it needs).  Calls whose
+ *    execution overlaps on the GPU (concurrent streams) race on it and give
+ *    wrong results: serialise them.
+ */
+#define ATTN_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)
+ATTN_API attn_status attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* o,
+                                      const void* dout, const float* lse, void* dq, void* dk,
+                                      void* dv, int B, int Sq, int Sk, int H, int D, float scale,
+                                      int causal, int win_left, int win_right, void* stream);
 
 /* attn_status_string - static English text for a status code (never NULL). */
 ATTN_API const char* attn_status_string(attn_status s);

@@ -38,7 +38,7 @@ def test_status_enum_matches_binding():
 
 def test_status_strings():
     from exact_attention_156_b200 import status_string
-    for s in range(11):
+    for s in range(12):
         assert status_string(s) and status_string(s) != "unknown status"
     assert status_string(99) == "unknown status"
 
