@@ -44,11 +44,11 @@ constexpr int kMmaWarp = 8;
 constexpr int kLoadWarp = 9;
 constexpr int kStages = 2;
 // Register split after launch (168 per thread at launch: 384 x 168 = 64512):
-// compute 128 x 240 + drain 128 x 136 + control 128 x 80 = 58368.
+// compute 128 x 240 + drain 128 x 144 + control 128 x 120 = 64512.
 constexpr int kLaunchRegs = 168;
 constexpr int kComputeRegs = 240;
-constexpr int kDrainRegs = 136;
-constexpr int kControlRegs = 80;
+constexpr int kDrainRegs = 144;
+constexpr int kControlRegs = 120;
 static_assert(128 * (kComputeRegs + kDrainRegs + kControlRegs) <= kThreads * kLaunchRegs,
               "register split exceeds the launch allocation");
 
@@ -508,12 +508,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr uint32_t id_dv = idesc_bf16_f32(BN, D, false, true);    // dV, dK
       constexpr uint32_t id_dq = idesc_bf16_f32(BM, D, true, true);     // dQ
       auto issue_kmajor = [&](uint32_t d_col, uint32_t a_base, uint32_t b_base) {
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk / 4) * C::kBoxBytes + (kk % 4) * 32;
-          mma_bf16_ss(tmem + d_col, sdesc_sw128(a_base + off, 16), sdesc_sw128(b_base + off, 16),
-                      id_s, kk > 0 ? 1u : 0u);
-        }
+        if constexpr (D == 128)
+          mma_chain_kk8(tmem + d_col, sdesc_sw128(a_base, 16), sdesc_sw128(b_base, 16), id_s, 0u);
+        else
+          mma_chain_kk4(tmem + d_col, sdesc_sw128(a_base, 16), sdesc_sw128(b_base, 16), id_s, 0u);
       };
       bool ok = bw.wait(bar(C::kBarKV), 0, 21);
       if (ok) ok = bw.wait(bar(C::kBarFull + 0), 0, 22);
@@ -529,21 +527,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         // dV += P^T dO   (A = P^T in tensor memory, K = query index)
         if (!bw.wait(bar(C::kBarP), t & 1, 23)) { ok = false; break; }
         tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < BM / 16; ++kk)
-          mma_bf16_ts(tmem + C::kColDV, tmem + C::kColS + kk * 8,
-                      sdesc_sw128(do_addr(s) + kk * 16 * 128, C::kBoxBytes), id_dv,
-                      (t > 0 || kk > 0) ? 1u : 0u);
+        mma_chain_ts_mn8(tmem + C::kColDV, tmem + C::kColS,
+                         sdesc_sw128(do_addr(s), C::kBoxBytes), id_dv, t > 0 ? 1u : 0u);
         // dK += dS^T Q   (A = dS^T in shared memory, K-major over the query index)
         if (!bw.wait(bar(C::kBarDS), t & 1, 24)) { ok = false; break; }
         tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < BM / 16; ++kk) {
-          const uint32_t aoff = (kk / 4) * C::kBoxBytes + (kk % 4) * 32;
-          mma_bf16_ss(tmem + C::kColDK, sdesc_sw128(ds_addr + aoff, 16),
-                      sdesc_sw128(q_addr(s) + kk * 16 * 128, C::kBoxBytes), id_dv,
-                      (t > 0 || kk > 0) ? 1u : 0u);
-        }
+        mma_chain_kmn8(tmem + C::kColDK, sdesc_sw128(ds_addr, 16),
+                       sdesc_sw128(q_addr(s), C::kBoxBytes), id_dv, t > 0 ? 1u : 0u);
         // next S^T while this tile's dQ is formed and drained
         const bool more = t + 1 < nq;
         const int s1 = (t + 1) % kStages;
@@ -554,11 +544,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_commit(bar(C::kBarS));
         }
         // dQ_tile = dS K  (A = dS read MN-major: rows of the buffer are keys = K index)
-#pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk)
-          mma_bf16_ss(tmem + C::kColDP, sdesc_sw128(ds_addr + kk * 16 * 128, C::kBoxBytes),
-                      sdesc_sw128(k_addr + kk * 16 * 128, C::kBoxBytes), id_dq,
-                      kk > 0 ? 1u : 0u);
+        mma_chain_mnmn8(tmem + C::kColDP, sdesc_sw128(ds_addr, C::kBoxBytes),
+                        sdesc_sw128(k_addr, C::kBoxBytes), id_dq, 0u);
         tc_commit(bar(C::kBarDQFull));
         tc_commit(bar(C::kBarDSEmpty));
         if (more) {

@@ -7,6 +7,8 @@
 //       mode 1: C = A B,   A K-major, B MN-major         (dK += dS^T Q)
 //       mode 2: C = A B,   A from tensor memory, B MN-major (O += P V; dV += P^T dO)
 //       mode 3: C = A^T B, A MN-major, B MN-major        (dQ = dS K)
+//       modes 4-7: the same four products through the fused multi-step
+//       chains the kernels issue (mma_chain_*)
 //   attn_diag_tma: a TMA load of a (1, 128, 1, 128) bf16 tensor with the
 //     same 4-D map and 128-byte swizzle as the kernels; the raw shared-memory
 //     bytes are copied out so the test can check the placement.
@@ -76,7 +78,7 @@ __global__ void __launch_bounds__(128, 1)
   const uint32_t lane_off = uint32_t(warp * 32) << 16;
   const int row = warp * 32 + (tid % 32);
 
-  if (mode == 2) {
+  if (mode == 2 || mode == 6) {
     // A into tensor memory columns [128, 192): lane m holds A[m][k] packed in pairs.
     uint32_t w[32];
     for (int half = 0; half < 2; ++half) {
@@ -96,22 +98,38 @@ __global__ void __launch_bounds__(128, 1)
 
   Bounded bw{&abort_flag, &g_diag_err, 1000000000ull};
   if (tid == 0) {
-    for (int kk = 0; kk < 8; ++kk) {
-      const uint32_t acc = kk > 0 ? 1u : 0u;
-      const uint32_t kmaj_off = (kk / 4) * kBox + (kk % 4) * 32;  // K-major: 16 K-elements
-      const uint32_t mn_off = kk * 16 * 128;                      // MN-major: 16 K-rows
-      if (mode == 0) {
-        mma_bf16_ss(tmem, sdesc_sw128(sa_u + kmaj_off, 16), sdesc_sw128(sb_u + kmaj_off, 16),
-                    idesc_bf16_f32(128, 128, false, false), acc);
-      } else if (mode == 1) {
-        mma_bf16_ss(tmem, sdesc_sw128(sa_u + kmaj_off, 16), sdesc_sw128(sb_u + mn_off, kBox),
-                    idesc_bf16_f32(128, 128, false, true), acc);
-      } else if (mode == 2) {
-        mma_bf16_ts(tmem, tmem + 128 + kk * 8, sdesc_sw128(sb_u + mn_off, kBox),
-                    idesc_bf16_f32(128, 128, false, true), acc);
-      } else {
-        mma_bf16_ss(tmem, sdesc_sw128(sa_u + mn_off, kBox), sdesc_sw128(sb_u + mn_off, kBox),
-                    idesc_bf16_f32(128, 128, true, true), acc);
+    if (mode >= 4) {
+      // the fused chains of the attention kernels
+      if (mode == 4)
+        mma_chain_kk8(tmem, sdesc_sw128(sa_u, 16), sdesc_sw128(sb_u, 16),
+                      idesc_bf16_f32(128, 128, false, false), 0u);
+      else if (mode == 5)
+        mma_chain_kmn8(tmem, sdesc_sw128(sa_u, 16), sdesc_sw128(sb_u, kBox),
+                       idesc_bf16_f32(128, 128, false, true), 0u);
+      else if (mode == 6)
+        mma_chain_ts_mn8(tmem, tmem + 128, sdesc_sw128(sb_u, kBox),
+                         idesc_bf16_f32(128, 128, false, true), 0u);
+      else
+        mma_chain_mnmn8(tmem, sdesc_sw128(sa_u, kBox), sdesc_sw128(sb_u, kBox),
+                        idesc_bf16_f32(128, 128, true, true), 0u);
+    } else {
+      for (int kk = 0; kk < 8; ++kk) {
+        const uint32_t acc = kk > 0 ? 1u : 0u;
+        const uint32_t kmaj_off = (kk / 4) * kBox + (kk % 4) * 32;  // K-major: 16 K-elements
+        const uint32_t mn_off = kk * 16 * 128;                      // MN-major: 16 K-rows
+        if (mode == 0) {
+          mma_bf16_ss(tmem, sdesc_sw128(sa_u + kmaj_off, 16), sdesc_sw128(sb_u + kmaj_off, 16),
+                      idesc_bf16_f32(128, 128, false, false), acc);
+        } else if (mode == 1) {
+          mma_bf16_ss(tmem, sdesc_sw128(sa_u + kmaj_off, 16), sdesc_sw128(sb_u + mn_off, kBox),
+                      idesc_bf16_f32(128, 128, false, true), acc);
+        } else if (mode == 2) {
+          mma_bf16_ts(tmem, tmem + 128 + kk * 8, sdesc_sw128(sb_u + mn_off, kBox),
+                      idesc_bf16_f32(128, 128, false, true), acc);
+        } else {
+          mma_bf16_ss(tmem, sdesc_sw128(sa_u + mn_off, kBox), sdesc_sw128(sb_u + mn_off, kBox),
+                      idesc_bf16_f32(128, 128, true, true), acc);
+        }
       }
     }
     tc_commit(smem_u32(&bar));
@@ -159,6 +177,16 @@ __global__ void __launch_bounds__(32, 1)
     for (int e = threadIdx.x; e < 2 * kBox; e += 32) out[e] = smem[e];
 }
 
+__global__ void diag_exp2_kernel(const float* x, float* y, int n) {
+  const int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
+  if (i + 1 < n) {
+    float r0, r1;
+    f2_unpack(f2_exp2_poly(f2_pack(x[i], x[i + 1])), r0, r1);
+    y[i] = r0;
+    y[i + 1] = r1;
+  }
+}
+
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
@@ -170,7 +198,7 @@ extern "C" {
 
 __attribute__((visibility("default"))) int attn_diag_mma(int mode, const void* A, const void* B,
                                                          float* C, void* stream) {
-  if (mode < 0 || mode > 3 || !A || !B || !C) return 1;
+  if (mode < 0 || mode > 7 || !A || !B || !C) return 1;
   const int smem = 4 * kBox + 64;
   if (cudaFuncSetAttribute(diag_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
       cudaSuccess)
@@ -205,6 +233,15 @@ __attribute__((visibility("default"))) int attn_diag_tma(const void* A, void* ou
   diag_tma_kernel<<<1, 32, smem, static_cast<cudaStream_t>(stream)>>>(map,
                                                                        static_cast<uint8_t*>(out));
   return cudaGetLastError() == cudaSuccess ? 0 : 5;
+}
+
+// y = the softmax's polynomial 2^x (pairs); n must be even.
+__attribute__((visibility("default"))) int attn_diag_exp2(const float* x, float* y, int n,
+                                                          void* stream) {
+  if (!x || !y || n <= 0 || (n & 1)) return 1;
+  const int pairs = n / 2;
+  diag_exp2_kernel<<<(pairs + 255) / 256, 256, 0, static_cast<cudaStream_t>(stream)>>>(x, y, n);
+  return cudaGetLastError() == cudaSuccess ? 0 : 3;
 }
 
 __attribute__((visibility("default"))) int attn_diag_error(void) {

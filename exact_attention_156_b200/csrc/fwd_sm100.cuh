@@ -29,6 +29,8 @@
 #include <cuda.h>
 #include <math.h>
 
+#include <type_traits>
+
 #include "common.cuh"
 #include "ptx.cuh"
 
@@ -245,37 +247,68 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int c = 0; c < BN; ++c)
           if (c < c_lo || c > c_hi) s[c] = -INFINITY;
       }
-      // row max as 8 independent chains, then a 3-level tree
-      float m8[8];
+      // row max: 8 independent chains of 3-input max, then a small tree
+      float mx8[8];
 #pragma unroll
-      for (int a = 0; a < 8; ++a) m8[a] = s[a];
+      for (int a = 0; a < 8; ++a) {
+        float acc = s[a];
 #pragma unroll
-      for (int c = 8; c < BN; ++c) m8[c % 8] = fmaxf(m8[c % 8], s[c]);
-      const float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
-                             fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+        for (int q = 1; q < 15; q += 2) acc = max3f(acc, s[8 * q + a], s[8 * (q + 1) + a]);
+        mx8[a] = fmaxf(acc, s[120 + a]);
+      }
+      const float mx = max3f(max3f(mx8[0], mx8[1], mx8[2]), max3f(mx8[3], mx8[4], mx8[5]),
+                             fmaxf(mx8[6], mx8[7]));
       const float m_cand = mx * sl2;
       const bool bump = m_cand > m_run + kRescaleThreshold;
       const float m_new = bump ? m_cand : m_run;
       const float alpha = bump ? ex2_approx(m_run - m_new) : 1.0f;
       const float m_eff = (m_new == -INFINITY) ? 0.0f : m_new;
-      float rs[8];
+      const uint64_t scale2 = f2_pack(sl2, sl2);
+      const uint64_t negm2 = f2_pack(-m_eff, -m_eff);
+      uint64_t acc2[4];
 #pragma unroll
-      for (int a = 0; a < 8; ++a) rs[a] = 0.f;
-      // P in two 64-column halves, each packed to bf16 pairs and stored to
-      // tensor memory (columns [0,32) and [32,64) of S_k) before the next half
+      for (int a = 0; a < 4; ++a) acc2[a] = 0ull;  // (+0.0f, +0.0f)
+      // p = 2^(s * scale * log2(e) - m): pairs in f32x2.  On fully visible
+      // tiles one pair in four is exponentiated on the FMA pipe (polynomial),
+      // the rest on MUFU; tiles with masked (-inf) scores use MUFU only, whose
+      // ex2(-inf) is exactly 0.  P goes to tensor memory as bf16 pairs in two
+      // 64-column halves (columns [0,32) and [32,64) of S_k).
+      auto exp_store = [&](auto use_poly) {
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        uint32_t pk[32];
+        for (int half = 0; half < 2; ++half) {
+          uint32_t pk[32];
 #pragma unroll
-        for (int c = 0; c < 64; c += 2) {
-          const float p0 = ex2_approx(fmaf(s[half * 64 + c], sl2, -m_eff));
-          const float p1 = ex2_approx(fmaf(s[half * 64 + c + 1], sl2, -m_eff));
-          rs[(c / 2) % 8] += p0 + p1;
-          pk[c / 2] = pack_bf16x2(p0, p1);
+          for (int c = 0; c < 32; ++c) {
+            const int e = half * 64 + 2 * c;
+            const uint64_t x2 = f2_fma(f2_pack(s[e], s[e + 1]), scale2, negm2);
+            uint64_t p2;
+            if (decltype(use_poly)::value && (c & 3) == 3) {
+              p2 = f2_exp2_poly(x2);
+            } else {
+              float x0, x1;
+              f2_unpack(x2, x0, x1);
+              p2 = f2_pack(ex2_approx(x0), ex2_approx(x1));
+            }
+            acc2[c & 3] = f2_add(acc2[c & 3], p2);
+            float p0, p1;
+            f2_unpack(p2, p0, p1);
+            pk[c] = pack_bf16x2(p0, p1);
+          }
+          tmem_st32(tS + half * 32, pk);
         }
-        tmem_st32(tS + half * 32, pk);
+      };
+      if (full) {
+        exp_store(std::true_type{});
+      } else {
+        exp_store(std::false_type{});
       }
-      const float row_sum = ((rs[0] + rs[1]) + (rs[2] + rs[3])) + ((rs[4] + rs[5]) + (rs[6] + rs[7]));
+      float row_sum;
+      {
+        const uint64_t t2 = f2_add(f2_add(acc2[0], acc2[1]), f2_add(acc2[2], acc2[3]));
+        float lo, hi;
+        f2_unpack(t2, lo, hi);
+        row_sum = lo + hi;
+      }
       l_run = l_run * alpha + row_sum;
       m_run = m_new;
       // Rescale O when this warp raised any row's max (rare after the first tile).
@@ -371,21 +404,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr uint32_t idesc_pv = idesc_bf16_f32(BM, D, false, true);
       auto in_range = [&](int k, int j) { return j >= jlo[k] && j < jhi[k]; };
       auto issue_s = [&](int k, int s) {
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk / 4) * C::kBoxBytes + (kk % 4) * 32;
-          mma_bf16_ss(tmem + C::col_s(k), sdesc_sw128(q_addr(k) + off, 16),
-                      sdesc_sw128(kv_addr(s) + off, 16), idesc_qk, kk > 0 ? 1u : 0u);
-        }
+        if constexpr (D == 128)
+          mma_chain_kk8(tmem + C::col_s(k), sdesc_sw128(q_addr(k), 16), sdesc_sw128(kv_addr(s), 16),
+                        idesc_qk, 0u);
+        else
+          mma_chain_kk4(tmem + C::col_s(k), sdesc_sw128(q_addr(k), 16), sdesc_sw128(kv_addr(s), 16),
+                        idesc_qk, 0u);
         tc_commit(bar(C::kBarS + k));
       };
       auto issue_pv = [&](int k, int s, bool acc) {
-#pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk) {
-          mma_bf16_ts(tmem + C::col_o(k), tmem + C::col_s(k) + kk * 8,
-                      sdesc_sw128(kv_addr(s) + kk * 16 * 128, C::kBoxBytes), idesc_pv,
-                      (acc || kk > 0) ? 1u : 0u);
-        }
+        mma_chain_ts_mn8(tmem + C::col_o(k), tmem + C::col_s(k),
+                         sdesc_sw128(kv_addr(s), C::kBoxBytes), idesc_pv, acc ? 1u : 0u);
         tc_commit(bar(C::kBarO + k));
       };
       auto slot_of = [&](int L) { return L % C::kStages; };

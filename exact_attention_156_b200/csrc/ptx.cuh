@@ -169,6 +169,185 @@ __device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, ui
       : "memory");
 }
 
+// ----------------------------------------------------------------------------
+// Fused MMA chains: one asm block issues all K-steps of a 128-row product, so
+// the issuing thread spends about three instructions per tcgen05.mma.  The
+// descriptors of step kk are the base descriptors with the start-address field
+// (16-byte units, low 32 bits) advanced by: K-major 128B-swizzled tiles
+// ((kk / 4) * 1024 + (kk % 4) * 2), i.e. 32 bytes per 16-element step inside a
+// 64-column box and the next 16 KB box every four steps; MN-major tiles
+// (kk * 128), i.e. 16 rows of 128 bytes per step.  Start addresses stay below
+// 256 KB, so the low half never carries into the high half.  The first step
+// accumulates iff `accumulate` is non-zero; later steps always accumulate.
+// ----------------------------------------------------------------------------
+// 8 chained K-steps, A K-major, B K-major (SS form).
+__device__ __forceinline__ void mma_chain_kk8(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                   uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .b32 alo, ahi, blo, bhi, al, bl;\n\t.reg .b64 ad, bd;\n\t.reg .pred pa, pt;\n\t"
+      "mov.b64 {alo, ahi}, %1;\n\tmov.b64 {blo, bhi}, %2;\n\t"
+      "setp.ne.b32 pa, %4, 0;\n\tsetp.eq.b32 pt, 0, 0;\n\t"
+      "add.u32 al, alo, 0;\n\tadd.u32 bl, blo, 0;\n\t"
+      "mov.b64 ad, {al, ahi};\n\tmov.b64 bd, {bl, bhi};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], ad, bd, %3, pa;\n\t"
+      "add.u32 al, alo, 2;\n\tadd.u32 bl, blo, 2;\n\t"
+      "mov.b64 ad, {al, ahi};\n\tmov.b64 bd, {bl, bhi};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], ad, bd, %3, pt;\n\t"
+      "add.u32 al, alo, 4;\n\tadd.u32 bl, blo, 4;\n\t"
+      "mov.b64 ad, {al, ahi};\n\tmov.b64 bd, {bl, bhi};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], ad, bd, %3, pt;\n\t"
+      "add.u32 al, alo, 6;\n\tadd.u32 bl, blo, 6;\n\t"
+      "mov.b64 ad, {al, ahi};\n\tmov.b64 bd, {bl, bhi};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], ad, bd, %3, pt;\n\t"
+      "add.u32 al, alo, 1024;\n\tadd.u32 bl, blo, 1024;\n\t"
+      "mov.b64 ad, {al, ahi};\n\tmov.b64 bd, {bl, bhi};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], ad, bd, %3, pt;\n\t"
+      "add.u32 al, alo, 1026;\n\tadd.u32 bl, blo, 1026;\n\t"
+      "mov.b64 ad, {al, ahi};\n\tmov.b64 bd, {bl, bhi};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], ad, bd, %3, pt;\n\t"
+      "add.u32 al, alo, 1028;\n\tadd.u32 bl, blo, 1028;\n\t"
+      "mov.b64 ad, {al, ahi};\n\tmov.b64 bd, {bl, bhi};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], ad, bd, %3, pt;\n\t"
+      "add.u32 al, alo, 1030;\n\tadd.u32 bl, blo, 1030;\n\t"
+      "mov.b64 ad, {al, ahi};\n\tmov.b64 bd, {bl, bhi};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], ad, bd, %3, pt;\n\t"
+      "}"
+      :: "r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// 4 chained K-steps, A K-major, B K-major (SS form).
+__device__ __forceinline__ void mma_chain_kk4(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                   uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .b32 alo, ahi, blo, bhi, al, bl;\n\t.reg .b64 ad, bd;\n\t.reg .pred pa, pt;\n\t"
+      "mov.b64 {alo, ahi}, %1;\n\tmov.b64 {blo, bhi}, %2;\n\t"
+      "setp.ne.b32 pa, %4, 0;\n\tsetp.eq.b32 pt, 0, 0;\n\t"
+      "add.u32 al, alo, 0;\n\tadd.u32 bl, blo, 0;\n\t"
+      "mov.b64 ad, {al, ahi};\n\tmov.b64 bd, {bl, bhi};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], ad, bd, %3, pa;\n\t"
+      "add.u32 al, alo, 2;\n\tadd.u32 bl, blo, 2;\n\t"
+      "mov.b64 ad, {al, ahi};\n\tmov.b64 bd, {bl, bhi};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], ad, bd, %3, pt;\n\t"
+      "add.u32 al, alo, 4;\n\tadd.u32 bl, blo, 4;\n\t"
+      "mov.b64 ad, {al, ahi};\n\tmov.b64 bd, {bl, bhi};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], ad, bd, %3, pt;\n\t"
+      "add.u32 al, alo, 6;\n\tadd.u32 bl, blo, 6;\n\t"
+      "mov.b64 ad, {al, ahi};\n\tmov.b64 bd, {bl, bhi};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], ad, bd, %3, pt;\n\t"
+      "}"
+      :: "r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// 8 chained K-steps, A K-major, B MN-major (SS form).
+__device__ __forceinline__ void mma_chain_kmn8(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                   uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .b32 alo, ahi, blo, bhi, al, bl;\n\t.reg .b64 ad, bd;\n\t.reg .pred pa, pt;\n\t"
+      "mov.b64 {alo, ahi}, %1;\n\tmov.b64 {blo, bhi}, %2;\n\t"
+      "setp.ne.b32 pa, %4, 0;\n\tsetp.eq.b32 pt, 0, 0;\n\t"
+      "add.u32 al, alo, 0;\n\tadd.u32 bl, blo, 0;\n\t"
+      "mov.b64 ad, {al, ahi};\n\tmov.b64 bd, {bl, bhi};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], ad, bd, %3, pa;\n\t"
+      "add.u32 al, alo, 2;\n\tadd.u32 bl, blo, 128;\n\t"
+      "mov.b64 ad, {al, ahi};\n\tmov.b64 bd, {bl, bhi};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], ad, bd, %3, pt;\n\t"
+      "add.u32 al, alo, 4;\n\tadd.u32 bl, blo, 256;\n\t"
+      "mov.b64 ad, {al, ahi};\n\tmov.b64 bd, {bl, bhi};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], ad, bd, %3, pt;\n\t"
+      "add.u32 al, alo, 6;\n\tadd.u32 bl, blo, 384;\n\t"
+      "mov.b64 ad, {al, ahi};\n\tmov.b64 bd, {bl, bhi};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], ad, bd, %3, pt;\n\t"
+      "add.u32 al, alo, 1024;\n\tadd.u32 bl, blo, 512;\n\t"
+      "mov.b64 ad, {al, ahi};\n\tmov.b64 bd, {bl, bhi};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], ad, bd, %3, pt;\n\t"
+      "add.u32 al, alo, 1026;\n\tadd.u32 bl, blo, 640;\n\t"
+      "mov.b64 ad, {al, ahi};\n\tmov.b64 bd, {bl, bhi};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], ad, bd, %3, pt;\n\t"
+      "add.u32 al, alo, 1028;\n\tadd.u32 bl, blo, 768;\n\t"
+      "mov.b64 ad, {al, ahi};\n\tmov.b64 bd, {bl, bhi};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], ad, bd, %3, pt;\n\t"
+      "add.u32 al, alo, 1030;\n\tadd.u32 bl, blo, 896;\n\t"
+      "mov.b64 ad, {al, ahi};\n\tmov.b64 bd, {bl, bhi};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], ad, bd, %3, pt;\n\t"
+      "}"
+      :: "r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// 8 chained K-steps, A MN-major, B MN-major (SS form).
+__device__ __forceinline__ void mma_chain_mnmn8(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                   uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .b32 alo, ahi, blo, bhi, al, bl;\n\t.reg .b64 ad, bd;\n\t.reg .pred pa, pt;\n\t"
+      "mov.b64 {alo, ahi}, %1;\n\tmov.b64 {blo, bhi}, %2;\n\t"
+      "setp.ne.b32 pa, %4, 0;\n\tsetp.eq.b32 pt, 0, 0;\n\t"
+      "add.u32 al, alo, 0;\n\tadd.u32 bl, blo, 0;\n\t"
+      "mov.b64 ad, {al, ahi};\n\tmov.b64 bd, {bl, bhi};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], ad, bd, %3, pa;\n\t"
+      "add.u32 al, alo, 128;\n\tadd.u32 bl, blo, 128;\n\t"
+      "mov.b64 ad, {al, ahi};\n\tmov.b64 bd, {bl, bhi};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], ad, bd, %3, pt;\n\t"
+      "add.u32 al, alo, 256;\n\tadd.u32 bl, blo, 256;\n\t"
+      "mov.b64 ad, {al, ahi};\n\tmov.b64 bd, {bl, bhi};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], ad, bd, %3, pt;\n\t"
+      "add.u32 al, alo, 384;\n\tadd.u32 bl, blo, 384;\n\t"
+      "mov.b64 ad, {al, ahi};\n\tmov.b64 bd, {bl, bhi};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], ad, bd, %3, pt;\n\t"
+      "add.u32 al, alo, 512;\n\tadd.u32 bl, blo, 512;\n\t"
+      "mov.b64 ad, {al, ahi};\n\tmov.b64 bd, {bl, bhi};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], ad, bd, %3, pt;\n\t"
+      "add.u32 al, alo, 640;\n\tadd.u32 bl, blo, 640;\n\t"
+      "mov.b64 ad, {al, ahi};\n\tmov.b64 bd, {bl, bhi};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], ad, bd, %3, pt;\n\t"
+      "add.u32 al, alo, 768;\n\tadd.u32 bl, blo, 768;\n\t"
+      "mov.b64 ad, {al, ahi};\n\tmov.b64 bd, {bl, bhi};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], ad, bd, %3, pt;\n\t"
+      "add.u32 al, alo, 896;\n\tadd.u32 bl, blo, 896;\n\t"
+      "mov.b64 ad, {al, ahi};\n\tmov.b64 bd, {bl, bhi};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], ad, bd, %3, pt;\n\t"
+      "}"
+      :: "r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// 8 chained K-steps, A from tensor memory (8 columns per step), B MN-major (TS form).
+__device__ __forceinline__ void mma_chain_ts_mn8(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                   uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .b32 blo, bhi, bl, at;\n\t.reg .b64 bd;\n\t.reg .pred pa, pt;\n\t"
+      "mov.b64 {blo, bhi}, %2;\n\t"
+      "setp.ne.b32 pa, %4, 0;\n\tsetp.eq.b32 pt, 0, 0;\n\t"
+      "add.u32 at, %1, 0;\n\tadd.u32 bl, blo, 0;\n\t"
+      "mov.b64 bd, {bl, bhi};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [at], bd, %3, pa;\n\t"
+      "add.u32 at, %1, 8;\n\tadd.u32 bl, blo, 128;\n\t"
+      "mov.b64 bd, {bl, bhi};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [at], bd, %3, pt;\n\t"
+      "add.u32 at, %1, 16;\n\tadd.u32 bl, blo, 256;\n\t"
+      "mov.b64 bd, {bl, bhi};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [at], bd, %3, pt;\n\t"
+      "add.u32 at, %1, 24;\n\tadd.u32 bl, blo, 384;\n\t"
+      "mov.b64 bd, {bl, bhi};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [at], bd, %3, pt;\n\t"
+      "add.u32 at, %1, 32;\n\tadd.u32 bl, blo, 512;\n\t"
+      "mov.b64 bd, {bl, bhi};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [at], bd, %3, pt;\n\t"
+      "add.u32 at, %1, 40;\n\tadd.u32 bl, blo, 640;\n\t"
+      "mov.b64 bd, {bl, bhi};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [at], bd, %3, pt;\n\t"
+      "add.u32 at, %1, 48;\n\tadd.u32 bl, blo, 768;\n\t"
+      "mov.b64 bd, {bl, bhi};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [at], bd, %3, pt;\n\t"
+      "add.u32 at, %1, 56;\n\tadd.u32 bl, blo, 896;\n\t"
+      "mov.b64 bd, {bl, bhi};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [at], bd, %3, pt;\n\t"
+      "}"
+      :: "r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // Instruction descriptor for kind::f16 with bf16 A/B and f32 accumulate.
 // Fields: [4,6) D format (1 = f32), [7,10) A format (1 = bf16), [10,13) B format,
 // [15] A major (1 = MN-major), [16] B major, [17,23) N>>3, [24,29) M>>4.
@@ -326,6 +505,65 @@ __device__ __forceinline__ void bulk_wait_read_all() {
 // Wait until all committed bulk groups have completed.
 __device__ __forceinline__ void bulk_wait_all() {
   asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+
+// ----------------------------------------------------------------------------
+// Packed fp32 pairs (sm_100 f32x2 arithmetic) and helpers of the softmax
+// ----------------------------------------------------------------------------
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// 2^x for a pair of floats on the FMA pipe (no MUFU), for x <= 127:
+// x is clamped to >= -126 (so the exponent field cannot underflow), split as x = n + f with n = round(x) (adding and
+// subtracting 1.5 * 2^23 rounds to the nearest integer) and f in [-1/2, 1/2];
+// 2^f comes from a degree-3 polynomial whose coefficients are the
+// relative-error minimax fit on [-1/2, 1/2] computed with the Remez exchange
+// algorithm (max relative error 7.5e-5); 2^n is applied by adding n to the
+// exponent field.  Used for a fixed share of the softmax exponentials so the
+// MUFU unit is not the bottleneck; the result is rounded to bf16 anyway.
+__device__ __forceinline__ uint64_t f2_exp2_poly(uint64_t x) {
+  float x0, x1;
+  f2_unpack(x, x0, x1);
+  const uint64_t xc = f2_pack(fmaxf(x0, -126.0f), fmaxf(x1, -126.0f));
+  const uint64_t magic = f2_pack(12582912.0f, 12582912.0f);
+  const uint64_t neg_magic = f2_pack(-12582912.0f, -12582912.0f);
+  const uint64_t minus_one = f2_pack(-1.0f, -1.0f);
+  const uint64_t j = f2_add(xc, magic);        // round(x) in the low mantissa bits
+  const uint64_t n = f2_add(j, neg_magic);     // round(x) as a float
+  const uint64_t f = f2_fma(n, minus_one, xc); // x - round(x)
+  uint64_t q = f2_fma(f2_pack(0.0551716685295105f, 0.0551716685295105f), f,
+                      f2_pack(0.2426111251115799f, 0.2426111251115799f));
+  q = f2_fma(q, f, f2_pack(0.6932609677314758f, 0.6932609677314758f));
+  q = f2_fma(q, f, f2_pack(0.9999280571937561f, 0.9999280571937561f));
+  float q0, q1, j0, j1;
+  f2_unpack(q, q0, q1);
+  f2_unpack(j, j0, j1);
+  // the integer n sits in the low bits of j; shifted into the exponent field
+  // the constant part of j vanishes (mod 2^32)
+  const float r0 = __int_as_float(__float_as_int(q0) + (__float_as_int(j0) << 23));
+  const float r1 = __int_as_float(__float_as_int(q1) + (__float_as_int(j1) << 23));
+  return f2_pack(r0, r1);
 }
 
 // ----------------------------------------------------------------------------

@@ -54,16 +54,41 @@ def test_tma_load_uses_the_128_byte_swizzle(diag):
     np.testing.assert_array_equal(got, a)
 
 
-@pytest.mark.parametrize("mode", [0, 1, 2, 3])
+@pytest.mark.parametrize("mode", [0, 1, 2, 3, 4, 5, 6, 7])
 def test_tcgen05_operand_forms(diag, mode):
     import torch
     a, b = _bf16_matrix(10 + mode), _bf16_matrix(20 + mode)
     A = bf16_bits_to_f32(a).astype(np.float64)
     B = bf16_bits_to_f32(b).astype(np.float64)
-    ref = {0: A @ B.T, 1: A @ B, 2: A @ B, 3: A.T @ B}[mode]
+    ref = {0: A @ B.T, 1: A @ B, 2: A @ B, 3: A.T @ B}[mode % 4]
     c = torch.zeros(128, 128, dtype=torch.float32, device="cuda")
     assert diag.attn_diag_mma(mode, _dev(a).data_ptr(), _dev(b).data_ptr(), c.data_ptr(), None) == 0
     assert diag.attn_diag_error() == 0
     got = c.cpu().numpy().astype(np.float64)
     err = np.abs(got - ref).max() / np.abs(ref).max()
     assert err < 1e-5, f"mode {mode}: relative error {err:.3e}"
+
+
+def test_polynomial_exp2_against_float64(diag):
+    """The FMA-pipe 2^x used for part of the softmax: relative error within the
+    minimax bound (7.5e-5, plus float32 rounding) on the range the softmax
+    feeds it, and a tiny non-negative value (not garbage) below -126."""
+    import torch
+    diag.attn_diag_exp2.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p]
+    x = np.concatenate([np.linspace(-126.0, 127.0, 2_000_000),
+                        np.random.default_rng(3).uniform(-30, 8, 1_000_000)]).astype(np.float32)
+    xd = torch.from_numpy(x).cuda()
+    yd = torch.empty_like(xd)
+    assert diag.attn_diag_exp2(xd.data_ptr(), yd.data_ptr(), x.size, None) == 0
+    assert diag.attn_diag_error() == 0
+    y = yd.cpu().numpy().astype(np.float64)
+    ref = np.exp2(x.astype(np.float64))
+    normal = x >= -125.0
+    rel = np.abs(y[normal] - ref[normal]) / ref[normal]
+    assert rel.max() < 8e-5, rel.max()
+    low = np.array([-126.5, -200.0, -1e30, -np.inf], dtype=np.float32)
+    ld = torch.from_numpy(low).cuda()
+    lo = torch.empty_like(ld)
+    assert diag.attn_diag_exp2(ld.data_ptr(), lo.data_ptr(), low.size, None) == 0
+    lo = lo.cpu().numpy()
+    assert np.all(lo >= 0) and np.all(lo < 2.0 ** -124)
