@@ -299,7 +299,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   };
 
   if (warp < kDrainWarp0) {
-    regs_inc<kComputeRegs>();
+    regs_realloc<kLaunchRegs, kComputeRegs>();
     // ------------------------------------------------------------ P and dS
     const int quad = warp % 4;
     const int r = quad * 32 + lane;  // key row within the tile
@@ -418,7 +418,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     return;
   }
   if (warp < kMmaWarp) {
-    regs_dec<kDrainRegs>();
+    regs_realloc<kLaunchRegs, kDrainRegs>();
     // ------------------------------------------------------------ dQ drain
     // TMEM -> registers -> the finished Q/dO stage (as four 128x32 fp32 boxes,
     // 128-byte swizzle) -> one TMA reduce-add per box into the fp32 accumulator.
@@ -471,7 +471,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     finish();
     return;
   }
-  regs_dec<kControlRegs>();
+  regs_realloc<kLaunchRegs, kControlRegs>();
   if (warp == kLoadWarp) {
     // ------------------------------------------------------------ loads
     if (lane == 0 && nq > 0) {

@@ -207,7 +207,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   };
 
   if (warp < 8) {
-    regs_inc<kSoftmaxRegs>();
+    regs_realloc<kLaunchRegs, kSoftmaxRegs>();
     // ------------------------------------------------------------ softmax + epilogue
     const int k = warp / 4;            // query tile of this warpgroup
     const int quad = warp % 4;         // TMEM lane quadrant
@@ -368,7 +368,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     return;
   }
 
-  regs_dec<kControlRegs>();
+  regs_realloc<kLaunchRegs, kControlRegs>();
   if (warp == kLoadWarp) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0 && any_work) {

@@ -467,6 +467,19 @@ __device__ __forceinline__ void regs_dec() {
   asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
 }
 
+// Move this warpgroup from `From` registers per thread (its count at launch)
+// to `To`: setmaxnreg.inc to grow, setmaxnreg.dec to shrink, chosen at compile
+// time so the direction can never be wrong.
+template <int From, int To>
+__device__ __forceinline__ void regs_realloc() {
+  static_assert(To % 8 == 0 && To >= 24 && To <= 256, "setmaxnreg count out of range");
+  if constexpr (To > From) {
+    regs_inc<To>();
+  } else if constexpr (To < From) {
+    regs_dec<To>();
+  }
+}
+
 // Named barrier over `count` threads (ids 1..15; id 0 is __syncthreads).
 __device__ __forceinline__ void named_bar_sync(int id, int count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
@@ -526,6 +539,11 @@ __device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
 __device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
   uint64_t d;
   asm("add.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("mul.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
   return d;
 }
 __device__ __forceinline__ float max3f(float a, float b, float c) {
