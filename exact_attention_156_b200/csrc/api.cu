@@ -192,8 +192,8 @@ attn_status launch_fwd(const DeviceState& st, const void* q, const void* k, cons
 
 struct Workspace {
   float* dq_acc;  // [B*H][Sq_pad][D]
-  float* lse2;    // [B*H][Sq_pad]
-  float* delta;   // [B*H][Sq_pad]
+  float* nlse2;   // [B*H][Sq_pad] -LSE * log2(e)
+  float* ndelta;  // [B*H][Sq_pad] -rowsum(dO * O)
   int Sq_pad;
 };
 
@@ -202,8 +202,8 @@ Workspace carve(void* workspace, int B, int Sq, int H, int D) {
   w.Sq_pad = sq_pad(Sq);
   const size_t rows = size_t(B) * H * w.Sq_pad;
   w.dq_acc = static_cast<float*>(workspace);
-  w.lse2 = w.dq_acc + rows * D;
-  w.delta = w.lse2 + rows;
+  w.nlse2 = w.dq_acc + rows * D;
+  w.ndelta = w.nlse2 + rows;
   return w;
 }
 
@@ -213,8 +213,8 @@ attn_status launch_bwd_pre(const void* o, const void* dout, const float* lse, in
   const long long rows = (long long)B * H * w.Sq_pad;
   const unsigned blocks = unsigned((rows + 7) / 8);
   bwd::attn_bwd_pre_kernel<D><<<blocks, 256, 0, stream>>>(
-      static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout), lse, w.lse2,
-      w.delta, w.dq_acc, B, H, Sq, w.Sq_pad);
+      static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout), lse, w.nlse2,
+      w.ndelta, w.dq_acc, B, H, Sq, w.Sq_pad);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_LAUNCH;
 }
 
@@ -231,8 +231,8 @@ attn_status launch_bwd_main(const DeviceState& st, const void* q, const void* k,
   bwd::Params p;
   p.dk = static_cast<__nv_bfloat16*>(dk);
   p.dv = static_cast<__nv_bfloat16*>(dv);
-  p.lse2 = w.lse2;
-  p.delta = w.delta;
+  p.nlse2 = w.nlse2;
+  p.ndelta = w.ndelta;
   p.dq_acc = w.dq_acc;
   p.B = B;
   p.H = H;

@@ -10,18 +10,22 @@
 //   dS = P * (dP - Delta), dK = scale dS^T Q, dQ = scale dS K.
 //
 // Kernels:
-//  1. bwd_pre: Delta_i (fp32), LSE in base 2 (padded rows: +inf so P = 0),
-//     and zeroes the fp32 dQ accumulator.  Memory bound.
+//  1. bwd_pre: -Delta_i (fp32), -LSE in base 2 (padded rows: -inf so P = 0),
+//     and zeroes the fp32 dQ accumulator.  Memory bound.  Both row values are
+//     stored negated so the main kernel adds them with packed fp32 pairs.
 //  2. bwd_main: one CTA per (128-key tile, head, batch); K_j and V_j stay in
 //     shared memory while the CTA streams the query tiles that can see them.
 //     Transposed products put the key index on tensor-memory lanes:
 //       S^T = K Q^T  and  dP^T = V dO^T   (M = keys, N = queries, K = D)
 //       dV += P^T dO  (A = P^T from tensor memory)
 //       dK += dS^T Q  (A = dS^T from shared memory, K-major)
-//       dQ_tile = dS K (A = the same dS^T buffer read MN-major) -> fp32 atomics
-//     warps 0-3: P and dS (one thread = one key row); warps 4-7: drain dQ
-//     from tensor memory into the fp32 accumulator with vector reductions;
-//     warp 8: MMA issue; warp 9: TMA / bulk loads.
+//       dQ_tile = dS K (A = the same dS^T buffer read MN-major) -> fp32 TMA
+//       bulk reduce-add through a dedicated two-slot staging ring
+//     warps 0-3: P and dS (one thread = one key row); warps 4-7: drain dQ;
+//     warp 8: MMA issue; warp 9: Q loads; warp 10: dO loads.
+//     Q (with its row values) is double buffered, dO single buffered; the MMA
+//     order dV(t), S(t+1), dQ(t), dK(t), dP(t+1) lets the next tile's P run
+//     while the tensor core finishes this tile's gradients.
 //  3. bwd_dq_finalize: dQ = bf16(scale * accumulator).
 // Tensor memory (512 columns): dK [0,D) dV [D,2D) S^T/P^T [2D,2D+128)
 // dP^T / dQ [2D+128, 2D+256).
@@ -38,39 +42,44 @@ namespace bwd {
 
 constexpr int BM = 128;  // query rows per tile
 constexpr int BN = 128;  // key rows per CTA
-constexpr int kThreads = 384;  // compute WG, dQ-drain WG, control WG {MMA, TMA, 2 idle}
+constexpr int kThreads = 384;  // compute WG, dQ-drain WG, control WG {MMA, Q load, dO load, idle}
 constexpr int kDrainWarp0 = 4;
 constexpr int kMmaWarp = 8;
-constexpr int kLoadWarp = 9;
-constexpr int kStages = 2;
+constexpr int kLoadQWarp = 9;
+constexpr int kLoadDOWarp = 10;
+constexpr int kQStages = 2;
 // Register split after launch (168 per thread at launch: 384 x 168 = 64512):
-// compute 128 x 240 + drain 128 x 144 + control 128 x 120 = 64512.
+// compute 128 x 256 + drain 128 x 152 + control 128 x 96 = 64512.
 constexpr int kLaunchRegs = 168;
-constexpr int kComputeRegs = 240;
-constexpr int kDrainRegs = 144;
-constexpr int kControlRegs = 120;
+constexpr int kComputeRegs = 256;
+constexpr int kDrainRegs = 152;
+constexpr int kControlRegs = 96;
 static_assert(128 * (kComputeRegs + kDrainRegs + kControlRegs) <= kThreads * kLaunchRegs,
               "register split exceeds the launch allocation");
 
 template <int D>
 struct Cfg {
-  static constexpr int kBoxBytes = 128 * 128;
+  static constexpr int kBoxBytes = 128 * 128;  // one 64-column bf16 box of 128 rows
   static constexpr int kBoxes = D / 64;
   static constexpr int kTileBytes = 128 * D * 2;
+  static constexpr int kDQChunk = 32;                 // fp32 columns per reduce-add box
+  static constexpr int kDQChunks = D / kDQChunk;
+  static constexpr int kDQBufBytes = BM * kDQChunk * 4;  // 16 KB, 128-byte rows
   static constexpr int kKOff = 0;
   static constexpr int kVOff = kKOff + kTileBytes;
-  // stage s = [Q_s | dO_s]; once the MMAs of a stage are done, the whole stage
-  // (128 x D fp32 bytes) holds the dQ tile on its way to the TMA reduce-add.
-  static constexpr int kStageOff = kVOff + kTileBytes;
-  static constexpr int kStageBytes = 2 * kTileBytes;
-  static constexpr int kDSOff = kStageOff + kStages * kStageBytes;  // dS^T, 128 x 128 bf16
-  static constexpr int kLseOff = kDSOff + BN * BM * 2;             // [kStages][BM] fp32
-  static constexpr int kDeltaOff = kLseOff + kStages * BM * 4;     // [kStages][BM] fp32
-  static constexpr int kBarOff = kDeltaOff + kStages * BM * 4;
+  static constexpr int kQOff = kVOff + kTileBytes;                  // [kQStages] Q tiles
+  static constexpr int kDOOff = kQOff + kQStages * kTileBytes;      // one dO tile
+  static constexpr int kDSOff = kDOOff + kTileBytes;                // dS^T, 128 x 128 bf16
+  static constexpr int kDQOff = kDSOff + BN * BM * 2;               // [2] dQ staging boxes
+  static constexpr int kLseOff = kDQOff + 2 * kDQBufBytes;          // [kQStages][BM] -LSE*log2e
+  static constexpr int kDeltaOff = kLseOff + kQStages * BM * 4;     // [kQStages][BM] -Delta
+  static constexpr int kBarOff = kDeltaOff + kQStages * BM * 4;
   static constexpr int kBarKV = 0;
-  static constexpr int kBarFull = 1;
-  static constexpr int kBarEmpty = kBarFull + kStages;
-  static constexpr int kBarS = kBarEmpty + kStages;
+  static constexpr int kBarQFull = 1;
+  static constexpr int kBarQEmpty = kBarQFull + kQStages;
+  static constexpr int kBarDOFull = kBarQEmpty + kQStages;
+  static constexpr int kBarDOEmpty = kBarDOFull + 1;
+  static constexpr int kBarS = kBarDOEmpty + 1;
   static constexpr int kBarDP = kBarS + 1;
   static constexpr int kBarP = kBarDP + 1;
   static constexpr int kBarDS = kBarP + 1;
@@ -85,14 +94,16 @@ struct Cfg {
   static constexpr uint32_t kColDV = D;
   static constexpr uint32_t kColS = 2 * D;
   static constexpr uint32_t kColDP = 2 * D + 128;
-  static_assert(kStageBytes == BM * D * 4, "a stage must hold one fp32 dQ tile");
+  static_assert(kSmemBytes <= 232448, "shared memory exceeds the 227 KB per block of sm_100");
+  static_assert(kDQOff % 1024 == 0 && kDOOff % 1024 == 0 && kDSOff % 1024 == 0,
+                "128-byte-swizzled buffers need 1024-byte alignment");
 };
 
 struct Params {
   __nv_bfloat16* dk;
   __nv_bfloat16* dv;
-  const float* lse2;   // [B*H][Sq_pad] LSE * log2(e); +inf for padding rows
-  const float* delta;  // [B*H][Sq_pad]
+  const float* nlse2;   // [B*H][Sq_pad] -LSE * log2(e); -inf for padding rows
+  const float* ndelta;  // [B*H][Sq_pad] -Delta
   float* dq_acc;       // [B*H][Sq_pad][D]
   int B, H, Sq, Sk, Sq_pad;
   float scale;
@@ -108,7 +119,7 @@ struct Params {
 template <int D>
 __global__ void __launch_bounds__(256) attn_bwd_pre_kernel(
     const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* __restrict__ dout,
-    const float* __restrict__ lse, float* __restrict__ lse2, float* __restrict__ delta,
+    const float* __restrict__ lse, float* __restrict__ nlse2, float* __restrict__ ndelta,
     float* __restrict__ dq_acc, int B, int H, int Sq, int Sq_pad) {
   const long long gw = (long long)blockIdx.x * 8 + threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
@@ -147,13 +158,13 @@ __global__ void __launch_bounds__(256) attn_bwd_pre_kernel(
   for (int off = 16; off > 0; off >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, off);
   if (lane == 0) {
     const size_t r = size_t(bh) * Sq_pad + i;
-    float l2 = INFINITY;  // padding rows and rows that see no key: P = 0
+    float nl2 = -INFINITY;  // padding rows and rows that see no key: P = 0
     if (i < Sq) {
       const float l = lse[size_t(bh) * Sq + i];
-      if (l != -INFINITY) l2 = l * 1.4426950408889634f;
+      if (l != -INFINITY) nl2 = -l * 1.4426950408889634f;
     }
-    lse2[r] = l2;
-    delta[r] = dot;
+    nlse2[r] = nl2;
+    ndelta[r] = -dot;
   }
   float4* acc = reinterpret_cast<float4*>(dq_acc + (size_t(bh) * Sq_pad + i) * D);
   for (int c = lane; c < D / 4; c += 32) acc[c] = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -254,13 +265,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   Bounded bw{abort_flag, p.err, p.timeout_ns};
-  auto stage_addr = [&](int s) { return sbase + C::kStageOff + s * C::kStageBytes; };
-  auto q_addr = [&](int s) { return stage_addr(s); };
-  auto do_addr = [&](int s) { return stage_addr(s) + C::kTileBytes; };
+  auto q_addr = [&](int s) { return sbase + C::kQOff + s * C::kTileBytes; };
+  const uint32_t do_addr = sbase + C::kDOOff;
   const uint32_t k_addr = sbase + C::kKOff;
   const uint32_t v_addr = sbase + C::kVOff;
   const uint32_t ds_addr = sbase + C::kDSOff;
-  int load_count[kStages] = {0, 0};
+  int q_loads0 = 0, q_loads1 = 0;  // Q loads issued per slot (slot 0, slot 1)
+  int do_loads = 0;
   bool drain_issued = false;
 
   // ------------------------------------------------------------ teardown
@@ -272,22 +283,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     if (*abort_flag) {
       const uint64_t drain_ns = 2000000000ull;
-      if (warp == kLoadWarp && lane == 0 && nq > 0) {
-        for (int s = 0; s < kStages; ++s) {
-          if (load_count[s] == 0) continue;
-          const uint64_t t0 = globaltimer_ns();
-          while (!mbar_try_wait(bar(C::kBarFull + s), (load_count[s] - 1) & 1))
-            if (globaltimer_ns() - t0 > drain_ns) break;
-        }
+      auto settle = [&](uint32_t bb, uint32_t parity) {
         const uint64_t t0 = globaltimer_ns();
-        while (!mbar_try_wait(bar(C::kBarKV), 0))
+        while (!mbar_try_wait(bb, parity))
           if (globaltimer_ns() - t0 > drain_ns) break;
+      };
+      if (warp == kLoadQWarp && lane == 0 && nq > 0) {
+        if (q_loads0 > 0) settle(bar(C::kBarQFull + 0), (q_loads0 - 1) & 1);
+        if (q_loads1 > 0) settle(bar(C::kBarQFull + 1), (q_loads1 - 1) & 1);
+        settle(bar(C::kBarKV), 0);
       }
+      if (warp == kLoadDOWarp && lane == 0 && do_loads > 0)
+        settle(bar(C::kBarDOFull), (do_loads - 1) & 1);
       if (warp == kMmaWarp && lane == 0) {
         tc_commit(bar(C::kBarDone));
-        const uint64_t t0 = globaltimer_ns();
-        while (!mbar_try_wait(bar(C::kBarDone), 0))
-          if (globaltimer_ns() - t0 > drain_ns) break;
+        settle(bar(C::kBarDone), 0);
       }
       tc_fence_before();
       __syncthreads();
@@ -307,7 +317,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t lane_off = uint32_t(quad * 32) << 16;
     const uint32_t tS = tmem + lane_off + C::kColS;
     const uint32_t tDP = tmem + lane_off + C::kColDP;
-    const float sl2 = p.scale_log2;
+    const uint64_t sl2 = f2_pack(p.scale_log2, p.scale_log2);
     const int qmin_k = g.qmin(kk_idx);
     const int qmax_k = min(g.qmax(kk_idx), p.Sq - 1);
     const bool key_ok = kk_idx < p.Sk;
@@ -316,74 +326,102 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t sw = uint32_t(r & 7);
     bool ok = true;
     for (int t = 0; t < nq; ++t) {
-      const int s = t % kStages;
+      const int s = t % kQStages;
       const int i0 = (qlo + t) * BM;
-      const float4* lse2 = reinterpret_cast<const float4*>(smem + C::kLseOff + s * BM * 4);
-      const float4* dlt = reinterpret_cast<const float4*>(smem + C::kDeltaOff + s * BM * 4);
+      const float4* nl = reinterpret_cast<const float4*>(smem + C::kLseOff + s * BM * 4);
+      const float4* nd = reinterpret_cast<const float4*>(smem + C::kDeltaOff + s * BM * 4);
+      // P = 2^(scale*log2e*S - LSE*log2e), kept as bf16 pairs (what dV uses) for dS too
       if (!bw.wait_warp(bar(C::kBarS), t & 1, 27)) { ok = false; break; }
       tc_fence_after();
-      float pr[BM];
+      uint32_t pw[BM / 2];
       {
         uint32_t rr[BM];
         tmem_ld128(tS, rr);
+        const bool full = key_ok && n0 + BN - 1 <= p.Sk - 1 && i0 + BM - 1 <= p.Sq - 1 &&
+                          i0 >= g.qmin(n0 + BN - 1) && i0 + BM - 1 <= g.qmax(n0);
+        if (full) {
+          // every entry visible: a quarter of the exponentials on the FMA pipe
 #pragma unroll
-        for (int c = 0; c < BM; c += 4) {
-          const float4 l4 = lse2[c / 4];
-          pr[c + 0] = ex2_approx(fmaf(__uint_as_float(rr[c + 0]), sl2, -l4.x));
-          pr[c + 1] = ex2_approx(fmaf(__uint_as_float(rr[c + 1]), sl2, -l4.y));
-          pr[c + 2] = ex2_approx(fmaf(__uint_as_float(rr[c + 2]), sl2, -l4.z));
-          pr[c + 3] = ex2_approx(fmaf(__uint_as_float(rr[c + 3]), sl2, -l4.w));
+          for (int c = 0; c < BM; c += 4) {
+            const float4 l4 = nl[c / 4];
+            const uint64_t x0 = f2_fma(f2_pack(__uint_as_float(rr[c]), __uint_as_float(rr[c + 1])),
+                                       sl2, f2_pack(l4.x, l4.y));
+            const uint64_t x1 = f2_fma(
+                f2_pack(__uint_as_float(rr[c + 2]), __uint_as_float(rr[c + 3])), sl2,
+                f2_pack(l4.z, l4.w));
+            float a0, a1, a2, a3;
+            f2_unpack(x0, a0, a1);
+            pw[c / 2] = pack_bf16x2(ex2_approx(a0), ex2_approx(a1));
+            if ((c & 7) == 4) {
+              f2_unpack(f2_exp2_poly(x1), a2, a3);
+            } else {
+              f2_unpack(x1, a2, a3);
+              a2 = ex2_approx(a2);
+              a3 = ex2_approx(a3);
+            }
+            pw[c / 2 + 1] = pack_bf16x2(a2, a3);
+          }
+        } else {
+          const int c_lo = key_ok ? qmin_k - i0 : (1 << 30);
+          const int c_hi = qmax_k - i0;
+#pragma unroll
+          for (int c = 0; c < BM; c += 4) {
+            const float4 l4 = nl[c / 4];
+            const uint64_t x0 = f2_fma(f2_pack(__uint_as_float(rr[c]), __uint_as_float(rr[c + 1])),
+                                       sl2, f2_pack(l4.x, l4.y));
+            const uint64_t x1 = f2_fma(
+                f2_pack(__uint_as_float(rr[c + 2]), __uint_as_float(rr[c + 3])), sl2,
+                f2_pack(l4.z, l4.w));
+            float a[4];
+            f2_unpack(x0, a[0], a[1]);
+            f2_unpack(x1, a[2], a[3]);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              a[e] = ex2_approx(a[e]);
+              if (c + e < c_lo || c + e > c_hi) a[e] = 0.f;
+            }
+            pw[c / 2] = pack_bf16x2(a[0], a[1]);
+            pw[c / 2 + 1] = pack_bf16x2(a[2], a[3]);
+          }
         }
       }
-      const bool full = key_ok && n0 + BN - 1 <= p.Sk - 1 && i0 + BM - 1 <= p.Sq - 1 &&
-                        i0 >= g.qmin(n0 + BN - 1) && i0 + BM - 1 <= g.qmax(n0);
-      if (!full) {
-        const int c_lo = key_ok ? qmin_k - i0 : (1 << 30);
-        const int c_hi = qmax_k - i0;
-#pragma unroll
-        for (int c = 0; c < BM; ++c)
-          if (c < c_lo || c > c_hi) pr[c] = 0.f;
-      }
-      {
-        uint32_t w[BM / 2];
-#pragma unroll
-        for (int c = 0; c < BM / 2; ++c) w[c] = pack_bf16x2(pr[2 * c], pr[2 * c + 1]);
-        tmem_st64(tS, w);
-      }
+      tmem_st64(tS, pw);
       tc_fence_before();
       mbar_arrive(bar(C::kBarP));
 
+      // dS = P * (dP - Delta) -> bf16, written swizzled for the dK and dQ products
       if (!bw.wait_warp(bar(C::kBarDP), t & 1, 28)) { ok = false; break; }
-      if (t > 0 && !bw.wait_warp(bar(C::kBarDSEmpty), (t - 1) & 1, 29)) { ok = false; break; }
       tc_fence_after();
+      uint32_t rr[BM];
+      tmem_ld128(tDP, rr);
+      if (t > 0 && !bw.wait_warp(bar(C::kBarDSEmpty), (t - 1) & 1, 29)) { ok = false; break; }
 #pragma unroll
-      for (int c0 = 0; c0 < BM; c0 += 64) {
-        uint32_t rr[64];
-        tmem_ld64(tDP + c0, rr);
+      for (int c = 0; c < BM; c += 8) {
+        const float4 d0 = nd[c / 4];
+        const float4 d1 = nd[c / 4 + 1];
+        const float dl[8] = {d0.x, d0.y, d0.z, d0.w, d1.x, d1.y, d1.z, d1.w};
+        uint32_t w[4];
 #pragma unroll
-        for (int cc = 0; cc < 64; cc += 8) {
-          const float4 d0 = dlt[(c0 + cc) / 4];
-          const float4 d1 = dlt[(c0 + cc) / 4 + 1];
-          const float dl[8] = {d0.x, d0.y, d0.z, d0.w, d1.x, d1.y, d1.z, d1.w};
-          uint32_t w[4];
-#pragma unroll
-          for (int e = 0; e < 8; e += 2) {
-            const float a0 = pr[c0 + cc + e] * (__uint_as_float(rr[cc + e]) - dl[e]);
-            const float a1 = pr[c0 + cc + e + 1] * (__uint_as_float(rr[cc + e + 1]) - dl[e + 1]);
-            w[e / 2] = pack_bf16x2(a0, a1);
-          }
-          const int col = c0 + cc;  // first of 8 columns in this 16-byte chunk
-          const uint32_t box = uint32_t(col / 64);
-          const uint32_t chunk = uint32_t((col % 64) / 8);
-          st_shared_v4(ds_row + box * C::kBoxBytes + ((chunk ^ sw) << 4), w[0], w[1], w[2], w[3]);
+        for (int e = 0; e < 4; ++e) {
+          const uint32_t pp = pw[c / 2 + e];
+          const uint64_t p2 = f2_pack(__uint_as_float(pp << 16), __uint_as_float(pp & 0xffff0000u));
+          const uint64_t gd = f2_add(
+              f2_pack(__uint_as_float(rr[c + 2 * e]), __uint_as_float(rr[c + 2 * e + 1])),
+              f2_pack(dl[2 * e], dl[2 * e + 1]));
+          float a0, a1;
+          f2_unpack(f2_mul(p2, gd), a0, a1);
+          w[e] = pack_bf16x2(a0, a1);
         }
+        const uint32_t box = uint32_t(c / 64);
+        const uint32_t chunk = uint32_t((c % 64) / 8);
+        st_shared_v4(ds_row + box * C::kBoxBytes + ((chunk ^ sw) << 4), w[0], w[1], w[2], w[3]);
       }
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(bar(C::kBarDS));
     }
-    // epilogue: dK = scale * acc, dV = acc (bf16)
-    if (ok && nq > 0) ok = bw.wait_warp(bar(C::kBarDQFull), (nq - 1) & 1, 30);
+    // epilogue: dK = scale * acc, dV = acc (bf16), once the last dK product is done
+    if (ok && nq > 0) ok = bw.wait_warp(bar(C::kBarDSEmpty), (nq - 1) & 1, 30);
     if (ok) {
       tc_fence_after();
       const size_t orow = ((size_t(b) * p.Sk + size_t(kk_idx)) * p.H + h) * D;
@@ -420,51 +458,48 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp < kMmaWarp) {
     regs_realloc<kLaunchRegs, kDrainRegs>();
     // ------------------------------------------------------------ dQ drain
-    // TMEM -> registers -> the finished Q/dO stage (as four 128x32 fp32 boxes,
-    // 128-byte swizzle) -> one TMA reduce-add per box into the fp32 accumulator.
+    // TMEM -> registers (then the tensor memory is handed back at once) ->
+    // 32-column fp32 boxes (128-byte swizzle) in a two-slot staging ring ->
+    // one TMA reduce-add per box into the fp32 accumulator.
     const int quad = warp % 4;
     const int r = quad * 32 + lane;  // query row within the tile
     const uint32_t tDQ = tmem + (uint32_t(quad * 32) << 16) + C::kColDP;
     const uint32_t sw = uint32_t(r & 7);
     const bool leader = (warp == kDrainWarp0 && lane == 0);
     if (leader) tma_prefetch_desc(&tmDQ);
+    int n = 0;  // boxes issued so far
     for (int t = 0; t < nq; ++t) {
-      const int s = t % kStages;
       // all four drain warps continue or stop together (they meet at named barriers)
       if (!named_bar_and(1, 128, bw.wait(bar(C::kBarDQFull), t & 1, 31))) break;
       tc_fence_after();
-      const uint32_t stg = stage_addr(s) + uint32_t(r) * 128;
-      auto stage_cols = [&](const uint32_t(&rr)[64], int c_base) {
-#pragma unroll
-        for (int c = 0; c < 64; c += 4) {
-          const int col = c_base + c;
-          const uint32_t box = uint32_t(col / 32);
-          const uint32_t chunk = uint32_t((col % 32) / 4);
-          st_shared_v4(stg + box * (128 * 128) + ((chunk ^ sw) << 4), rr[c], rr[c + 1],
-                       rr[c + 2], rr[c + 3]);
-        }
-      };
-      uint32_t rr[64];
-      tmem_ld64(tDQ, rr);
+      uint32_t rr[D];
       if constexpr (D == 128) {
-        stage_cols(rr, 0);
-        tmem_ld64(tDQ + 64, rr);
+        tmem_ld128(tDQ, rr);
+      } else {
+        tmem_ld64(tDQ, rr);
       }
       // tensor memory is free again: the MMA warp may start dP of the next tile
       tc_fence_before();
       mbar_arrive(bar(C::kBarDQEmpty));
-      stage_cols(rr, D - 64);
-      fence_proxy_async_smem();
-      named_bar_sync(1, 128);
-      if (leader) {
-        const int row0 = bh * p.Sq_pad + (qlo + t) * BM;
+      const int row0 = bh * p.Sq_pad + (qlo + t) * BM;
 #pragma unroll
-        for (int box = 0; box < D / 32; ++box)
-          tma_reduce_add_2d(&tmDQ, stage_addr(s) + box * (128 * 128), box * 32, row0);
-        bulk_commit();
-        bulk_wait_read_all();  // the stage may be refilled once the reduce has read it
-        mbar_arrive(bar(C::kBarEmpty + s));
-        drain_issued = true;
+      for (int c = 0; c < C::kDQChunks; ++c, ++n) {
+        const uint32_t buf = sbase + C::kDQOff + uint32_t(n & 1) * C::kDQBufBytes;
+        // the reduce that last read this slot (two boxes ago) must have finished reading
+        if (leader && n >= 2) bulk_wait_read<1>();
+        named_bar_sync(1, 128);
+        const uint32_t row = buf + uint32_t(r) * 128;
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          st_shared_v4(row + ((uint32_t(k) ^ sw) << 4), rr[c * 32 + 4 * k], rr[c * 32 + 4 * k + 1],
+                       rr[c * 32 + 4 * k + 2], rr[c * 32 + 4 * k + 3]);
+        fence_proxy_async_smem();
+        named_bar_sync(1, 128);
+        if (leader) {
+          tma_reduce_add_2d(&tmDQ, buf, c * C::kDQChunk, row0);
+          bulk_commit();
+          drain_issued = true;
+        }
       }
     }
     if (leader && drain_issued) bulk_wait_all();
@@ -472,33 +507,43 @@ __global__ void __launch_bounds__(kThreads, 1)
     return;
   }
   regs_realloc<kLaunchRegs, kControlRegs>();
-  if (warp == kLoadWarp) {
-    // ------------------------------------------------------------ loads
+  if (warp == kLoadQWarp) {
+    // ------------------------------------------------------------ K, V, Q (+ row values)
     if (lane == 0 && nq > 0) {
       tma_prefetch_desc(&tmQ);
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
-      tma_prefetch_desc(&tmDO);
       mbar_arrive_expect_tx(bar(C::kBarKV), 2 * C::kTileBytes);
       for (int x = 0; x < C::kBoxes; ++x) {
         tma_load_4d(k_addr + x * C::kBoxBytes, &tmK, bar(C::kBarKV), x * 64, h, n0, b);
         tma_load_4d(v_addr + x * C::kBoxBytes, &tmV, bar(C::kBarKV), x * 64, h, n0, b);
       }
       for (int t = 0; t < nq; ++t) {
-        const int s = t % kStages;
-        const int u = t / kStages;
-        if (u > 0 && !bw.wait(bar(C::kBarEmpty + s), (u - 1) & 1, 20)) break;
+        const int s = t % kQStages;
+        const int u = t / kQStages;
+        if (u > 0 && !bw.wait(bar(C::kBarQEmpty + s), (u - 1) & 1, 20)) break;
         const int i0 = (qlo + t) * BM;
-        const uint32_t fb = bar(C::kBarFull + s);
-        mbar_arrive_expect_tx(fb, 2 * C::kTileBytes + 2 * BM * 4);
-        for (int x = 0; x < C::kBoxes; ++x) {
+        const uint32_t fb = bar(C::kBarQFull + s);
+        mbar_arrive_expect_tx(fb, C::kTileBytes + 2 * BM * 4);
+        for (int x = 0; x < C::kBoxes; ++x)
           tma_load_4d(q_addr(s) + x * C::kBoxBytes, &tmQ, fb, x * 64, h, i0, b);
-          tma_load_4d(do_addr(s) + x * C::kBoxBytes, &tmDO, fb, x * 64, h, i0, b);
-        }
         const size_t roff = size_t(bh) * p.Sq_pad + i0;
-        bulk_load(sbase + C::kLseOff + s * BM * 4, p.lse2 + roff, BM * 4, fb);
-        bulk_load(sbase + C::kDeltaOff + s * BM * 4, p.delta + roff, BM * 4, fb);
-        load_count[s]++;
+        bulk_load(sbase + C::kLseOff + s * BM * 4, p.nlse2 + roff, BM * 4, fb);
+        bulk_load(sbase + C::kDeltaOff + s * BM * 4, p.ndelta + roff, BM * 4, fb);
+        if (s == 0) ++q_loads0; else ++q_loads1;
+      }
+    }
+  } else if (warp == kLoadDOWarp) {
+    // ------------------------------------------------------------ dO
+    if (lane == 0 && nq > 0) {
+      tma_prefetch_desc(&tmDO);
+      for (int t = 0; t < nq; ++t) {
+        if (t > 0 && !bw.wait(bar(C::kBarDOEmpty), (t - 1) & 1, 32)) break;
+        const int i0 = (qlo + t) * BM;
+        mbar_arrive_expect_tx(bar(C::kBarDOFull), C::kTileBytes);
+        for (int x = 0; x < C::kBoxes; ++x)
+          tma_load_4d(do_addr + x * C::kBoxBytes, &tmDO, bar(C::kBarDOFull), x * 64, h, i0, b);
+        do_loads++;
       }
     }
   } else if (warp == kMmaWarp) {
@@ -514,44 +559,52 @@ __global__ void __launch_bounds__(kThreads, 1)
           mma_chain_kk4(tmem + d_col, sdesc_sw128(a_base, 16), sdesc_sw128(b_base, 16), id_s, 0u);
       };
       bool ok = bw.wait(bar(C::kBarKV), 0, 21);
-      if (ok) ok = bw.wait(bar(C::kBarFull + 0), 0, 22);
+      if (ok) ok = bw.wait(bar(C::kBarQFull + 0), 0, 22);
       if (ok) {
         tc_fence_after();
         issue_kmajor(C::kColS, k_addr, q_addr(0));
         tc_commit(bar(C::kBarS));
-        issue_kmajor(C::kColDP, v_addr, do_addr(0));
+        ok = bw.wait(bar(C::kBarDOFull), 0, 33);
+      }
+      if (ok) {
+        tc_fence_after();
+        issue_kmajor(C::kColDP, v_addr, do_addr);
         tc_commit(bar(C::kBarDP));
       }
       for (int t = 0; ok && t < nq; ++t) {
-        const int s = t % kStages;
+        const int s = t % kQStages;
+        const bool more = t + 1 < nq;
         // dV += P^T dO   (A = P^T in tensor memory, K = query index)
         if (!bw.wait(bar(C::kBarP), t & 1, 23)) { ok = false; break; }
         tc_fence_after();
         mma_chain_ts_mn8(tmem + C::kColDV, tmem + C::kColS,
-                         sdesc_sw128(do_addr(s), C::kBoxBytes), id_dv, t > 0 ? 1u : 0u);
-        // dK += dS^T Q   (A = dS^T in shared memory, K-major over the query index)
-        if (!bw.wait(bar(C::kBarDS), t & 1, 24)) { ok = false; break; }
-        tc_fence_after();
-        mma_chain_kmn8(tmem + C::kColDK, sdesc_sw128(ds_addr, 16),
-                       sdesc_sw128(q_addr(s), C::kBoxBytes), id_dv, t > 0 ? 1u : 0u);
-        // next S^T while this tile's dQ is formed and drained
-        const bool more = t + 1 < nq;
-        const int s1 = (t + 1) % kStages;
+                         sdesc_sw128(do_addr, C::kBoxBytes), id_dv, t > 0 ? 1u : 0u);
+        tc_commit(bar(C::kBarDOEmpty));
+        // next S^T: overwrites P^T only after dV has read it (same issue order)
         if (more) {
-          if (!bw.wait(bar(C::kBarFull + s1), ((t + 1) / kStages) & 1, 25)) { ok = false; break; }
+          const int s1 = (t + 1) % kQStages;
+          if (!bw.wait(bar(C::kBarQFull + s1), ((t + 1) / kQStages) & 1, 25)) { ok = false; break; }
           tc_fence_after();
           issue_kmajor(C::kColS, k_addr, q_addr(s1));
           tc_commit(bar(C::kBarS));
         }
+        if (!bw.wait(bar(C::kBarDS), t & 1, 24)) { ok = false; break; }
+        tc_fence_after();
         // dQ_tile = dS K  (A = dS read MN-major: rows of the buffer are keys = K index)
         mma_chain_mnmn8(tmem + C::kColDP, sdesc_sw128(ds_addr, C::kBoxBytes),
                         sdesc_sw128(k_addr, C::kBoxBytes), id_dq, 0u);
         tc_commit(bar(C::kBarDQFull));
+        // dK += dS^T Q   (A = dS^T in shared memory, K-major over the query index)
+        mma_chain_kmn8(tmem + C::kColDK, sdesc_sw128(ds_addr, 16),
+                       sdesc_sw128(q_addr(s), C::kBoxBytes), id_dv, t > 0 ? 1u : 0u);
+        tc_commit(bar(C::kBarQEmpty + s));
         tc_commit(bar(C::kBarDSEmpty));
         if (more) {
+          // dP^T of the next tile reuses the dQ columns once the drain has read them
           if (!bw.wait(bar(C::kBarDQEmpty), t & 1, 26)) { ok = false; break; }
+          if (!bw.wait(bar(C::kBarDOFull), (t + 1) & 1, 34)) { ok = false; break; }
           tc_fence_after();
-          issue_kmajor(C::kColDP, v_addr, do_addr(s1));
+          issue_kmajor(C::kColDP, v_addr, do_addr);
           tc_commit(bar(C::kBarDP));
         }
       }
