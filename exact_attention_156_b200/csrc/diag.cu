@@ -9,6 +9,13 @@
 //       mode 3: C = A^T B, A MN-major, B MN-major        (dQ = dS K)
 //       modes 4-7: the same four products through the fused multi-step
 //       chains the kernels issue (mma_chain_*)
+//   attn_diag_mma_pair: one 256x128x128 bf16 product issued for a pair of
+//     CTAs (a cluster of two, tcgen05 cta_group::2); CTA r holds rows
+//     [128 r, 128 r + 128) of A and C, and rows [64 r, 64 r + 64) of B (N x K):
+//       mode 8:  C = A B^T, A and B K-major, placed by plain stores
+//       mode 9:  C = A B,   A from tensor memory, B MN-major (CTA r: columns [64 r, +64))
+//       mode 10: as mode 8, operands brought in by the pair's TMA loads whose
+//                bytes are counted on the even CTA's mbarrier
 //   attn_diag_tma: a TMA load of a (1, 128, 1, 128) bf16 tensor with the
 //     same 4-D map and 128-byte swizzle as the kernels; the raw shared-memory
 //     bytes are copied out so the test can check the placement.
@@ -153,6 +160,129 @@ __global__ void __launch_bounds__(128, 1)
   }
 }
 
+// ---------------------------------------------------------------- CTA pair
+// A is 256 x 128 (row-major), B is 128 x 128 (row-major: N x K for modes 8/10,
+// K x N for mode 9), C is 256 x 128 fp32.
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(128, 1)
+    diag_mma_pair_kernel(int mode, const __nv_bfloat16* A, const __nv_bfloat16* Bm, float* C,
+                         const __grid_constant__ CUtensorMap mapA,
+                         const __grid_constant__ CUtensorMap mapB) {
+  extern __shared__ __align__(1024) uint8_t smem[];
+  // [A half: 2 boxes of 128 rows x 64 cols][B half: K-major 2 boxes of 64 rows, or one
+  //  MN-major box of 128 K rows x 64 N cols][bars]
+  constexpr int kAOff = 0, kBOff = 2 * kBox, kBarOff = 4 * kBox;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kBarOff);  // 0: loads, 1: product done
+  uint32_t& tslot = *reinterpret_cast<uint32_t*>(smem + kBarOff + 16);
+  int& abort_flag = *reinterpret_cast<int*>(smem + kBarOff + 20);
+  const int tid = threadIdx.x;
+  const int warp = tid / 32;
+  const uint32_t rank = cluster_ctarank();
+  const uint32_t sa_u = smem_u32(smem + kAOff), sb_u = smem_u32(smem + kBOff);
+  if ((sa_u & 1023u) != 0) return;
+  const int row = warp * 32 + (tid % 32);  // this CTA's row of A / C
+  if (tid == 0) {
+    mbar_init(smem_u32(&bars[0]), 1);
+    mbar_init(smem_u32(&bars[1]), 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (mode == 8 || mode == 9) {
+    // A half: rows [128 rank, +128) of A, K-major, two 64-column boxes
+    for (int e = tid; e < 128 * N; e += blockDim.x) {
+      const int r = e / N, c = e % N;
+      if (mode == 8)
+        *reinterpret_cast<__nv_bfloat16*>(smem + kAOff + swz(r, c)) = A[(128 * rank + r) * N + c];
+    }
+    if (mode == 8) {
+      // B half, K-major: rows [64 rank, +64) of B (N x K); boxes of 64 rows (8 KB)
+      for (int e = tid; e < 64 * N; e += blockDim.x) {
+        const int r = e / N, c = e % N;
+        const uint32_t off = uint32_t(c / 64) * 8192 + uint32_t(r) * 128 +
+                             ((uint32_t((c % 64) / 8) ^ uint32_t(r & 7)) << 4) + uint32_t(c % 8) * 2;
+        *reinterpret_cast<__nv_bfloat16*>(smem + kBOff + off) = Bm[(64 * rank + r) * N + c];
+      }
+    } else {
+      // B half, MN-major: all 128 K rows, N columns [64 rank, +64): one 128 x 64 box
+      for (int e = tid; e < 128 * 64; e += blockDim.x) {
+        const int r = e / 64, c = e % 64;
+        *reinterpret_cast<__nv_bfloat16*>(smem + kBOff + swz(r, c)) = Bm[r * N + 64 * rank + c];
+      }
+    }
+    fence_proxy_async_smem();
+  }
+  if (warp == 0) {
+    tmem_alloc_pair(smem_u32(&tslot), 256);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  cluster_sync();  // barriers initialised and operands placed in both CTAs
+  tc_fence_after();
+  const uint32_t tmem = tslot;
+  const uint32_t lane_off = uint32_t(warp * 32) << 16;
+  if (mode == 9) {
+    // A rows of this CTA into tensor memory columns [128, 192) as bf16 pairs
+    uint32_t w[32];
+    for (int half = 0; half < 2; ++half) {
+#pragma unroll
+      for (int c = 0; c < 32; ++c) {
+        const int k = half * 64 + 2 * c;
+        w[c] = pack_bf16x2(__bfloat162float(A[(128 * rank + row) * N + k]),
+                           __bfloat162float(A[(128 * rank + row) * N + k + 1]));
+      }
+      tmem_st32(tmem + lane_off + 128 + half * 32, w);
+    }
+    tc_fence_before();
+  }
+  Bounded bw{&abort_flag, &g_diag_err, 1000000000ull};
+  const uint32_t leader_load_bar = mapa_shared(smem_u32(&bars[0]), 0);
+  if (mode == 10 && tid == 0) {
+    if (rank == 0) mbar_arrive_expect_tx(smem_u32(&bars[0]), 2 * (2 * kBox + 2 * 8192));
+    for (int x = 0; x < 2; ++x) {
+      tma_load_4d_pair(sa_u + x * kBox, &mapA, leader_load_bar, x * 64, 0, 128 * int(rank), 0);
+      tma_load_4d_pair(sb_u + x * 8192, &mapB, leader_load_bar, x * 64, 0, 64 * int(rank), 0);
+    }
+  }
+  cluster_sync();  // mode 9: both CTAs' A rows are in tensor memory
+  tc_fence_after();
+  bool ok = true;
+  if (rank == 0 && tid == 0) {
+    if (mode == 10) ok = bw.wait(smem_u32(&bars[0]), 0, 3);
+    if (ok) {
+      tc_fence_after();
+      const uint32_t id_kk = idesc_bf16_f32(256, 128, false, false);
+      const uint32_t id_ts = idesc_bf16_f32(256, 128, false, true);
+      for (int kk = 0; kk < 8; ++kk) {
+        const uint32_t acc = kk > 0 ? 1u : 0u;
+        if (mode == 9) {
+          mma2_bf16_ts(tmem, tmem + 128 + kk * 8, sdesc_sw128(sb_u + kk * 16 * 128, kBox), id_ts, acc);
+        } else {
+          const uint32_t a_off = (kk / 4) * kBox + (kk % 4) * 32;
+          const uint32_t b_off = (kk / 4) * 8192 + (kk % 4) * 32;
+          mma2_bf16_ss(tmem, sdesc_sw128(sa_u + a_off, 16), sdesc_sw128(sb_u + b_off, 16), id_kk, acc);
+        }
+      }
+    }
+    tc_commit_pair(smem_u32(&bars[1]), 0x3);
+  }
+  __syncwarp();
+  ok = bw.wait_warp(smem_u32(&bars[1]), 0, 4);
+  tc_fence_after();
+  if (ok) {
+    for (int c0 = 0; c0 < N; c0 += 32) {
+      uint32_t r[32];
+      tmem_ld32(tmem + lane_off + c0, r);
+#pragma unroll
+      for (int c = 0; c < 32; ++c) C[(128 * rank + row) * N + c0 + c] = __uint_as_float(r[c]);
+    }
+  }
+  tc_fence_before();
+  cluster_sync();  // no CTA leaves while its peer may still use its memory
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem, 256);
+  }
+}
+
 __global__ void __launch_bounds__(32, 1)
     diag_tma_kernel(const __grid_constant__ CUtensorMap map, uint8_t* out) {
   extern __shared__ __align__(1024) uint8_t smem[];
@@ -206,6 +336,42 @@ __attribute__((visibility("default"))) int attn_diag_mma(int mode, const void* A
   diag_mma_kernel<<<1, 128, smem, static_cast<cudaStream_t>(stream)>>>(
       mode, static_cast<const __nv_bfloat16*>(A), static_cast<const __nv_bfloat16*>(B), C);
   return cudaGetLastError() == cudaSuccess ? 0 : 3;
+}
+
+// C (256 x 128 fp32) = the pair product of `mode` (8, 9 or 10) of A (256 x 128)
+// and B (128 x 128), both row-major bf16.
+__attribute__((visibility("default"))) int attn_diag_mma_pair(int mode, const void* A,
+                                                              const void* B, float* C,
+                                                              void* stream) {
+  if (mode < 8 || mode > 10 || !A || !B || !C) return 1;
+  void* fn = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) !=
+          cudaSuccess ||
+      fn == nullptr)
+    return 2;
+  // A as (D=128, H=1, S=256, B=1) with 128 x 64 boxes; B as (128, 1, 128, 1) with 64 x 64 boxes
+  alignas(64) CUtensorMap mapA, mapB;
+  const cuuint64_t dA[4] = {128, 1, 256, 1}, dB[4] = {128, 1, 128, 1};
+  const cuuint64_t sA[3] = {256, 256, 256 * 256}, sB[3] = {256, 256, 128 * 256};
+  const cuuint32_t bA[4] = {64, 1, 128, 1}, bB[4] = {64, 1, 64, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  auto enc = reinterpret_cast<EncodeTiledFn>(fn);
+  if (enc(&mapA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(A), dA, sA, bA, estr,
+          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS ||
+      enc(&mapB, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(B), dB, sB, bB, estr,
+          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return 3;
+  const int smem = 4 * kBox + 64;
+  if (cudaFuncSetAttribute(diag_mma_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           smem) != cudaSuccess)
+    return 4;
+  diag_mma_pair_kernel<<<2, 128, smem, static_cast<cudaStream_t>(stream)>>>(
+      mode, static_cast<const __nv_bfloat16*>(A), static_cast<const __nv_bfloat16*>(B), C, mapA,
+      mapB);
+  return cudaGetLastError() == cudaSuccess ? 0 : 5;
 }
 
 __attribute__((visibility("default"))) int attn_diag_tma(const void* A, void* out, void* stream) {

@@ -92,3 +92,25 @@ def test_polynomial_exp2_against_float64(diag):
     assert diag.attn_diag_exp2(ld.data_ptr(), lo.data_ptr(), low.size, None) == 0
     lo = lo.cpu().numpy()
     assert np.all(lo >= 0) and np.all(lo < 2.0 ** -124)
+
+
+@pytest.mark.parametrize("mode", [8, 9, 10])
+def test_tcgen05_cta_pair_products(diag, mode):
+    """One 256 x 128 x 128 product shared by a pair of CTAs (cta_group::2): each CTA
+    holds half of A's rows and half of B's rows; mode 10 brings the operands in with
+    the pair's TMA loads counted on the even CTA's barrier."""
+    import torch
+    diag.attn_diag_mma_pair.argtypes = [ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p,
+                                        ctypes.c_void_p, ctypes.c_void_p]
+    rng = np.random.default_rng(30 + mode)
+    a = f32_to_bf16_bits(rng.standard_normal((256, 128)).astype(np.float32))
+    b = _bf16_matrix(40 + mode)
+    A = bf16_bits_to_f32(a).astype(np.float64)
+    B = bf16_bits_to_f32(b).astype(np.float64)
+    ref = A @ B if mode == 9 else A @ B.T
+    c = torch.zeros(256, 128, dtype=torch.float32, device="cuda")
+    assert diag.attn_diag_mma_pair(mode, _dev(a).data_ptr(), _dev(b).data_ptr(), c.data_ptr(), None) == 0
+    assert diag.attn_diag_error() == 0
+    got = c.cpu().numpy().astype(np.float64)
+    err = np.abs(got - ref).max() / np.abs(ref).max()
+    assert err < 1e-5, f"mode {mode}: relative error {err:.3e}"
