@@ -7,10 +7,12 @@ code with it.
 from .attn_ref import (  # noqa: F401
     attention_backward,
     attention_backward_head,
+    attention_backward_kv_head,
     attention_backward_rows,
     attention_backward_rows_dq,
     attention_forward,
     attention_forward_rows,
+    kv_head,
     online_softmax_forward,
     visible_mask,
 )

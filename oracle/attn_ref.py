@@ -28,6 +28,12 @@ Readings of points the pages leave open (each listed in the design doc):
     scores: LSE_i = m_i + ln(sum_j exp(S_ij - m_i)).
   * a query row with no visible key has O_i = 0, LSE_i = -inf and zero
     gradient contributions.
+  * K and V may have fewer heads Hk than Q (H a multiple of Hk): the pages'
+    Transformers snippet (FlashAttention-2 overview, lshu.cn, section 3.3)
+    shapes Q with num_heads and K, V with num_kv_heads for the same call.
+    Query head h attends with key/value head h // (H / Hk) (consecutive query
+    heads share one K/V head; Hk = 1 is multi-query attention), and the
+    gradient of a shared K/V head is the sum over its query heads.
   * the backward is the analytic gradient of that definition (the pages say
     only that the backward recomputes the scores, yfxerp.com section 1):
     dV = P^T dO; dP = dO V^T; Delta_i = sum_j P_ij dP_ij; dS = P * (dP - Delta);
@@ -38,6 +44,13 @@ Arrays use the pages' layout (batch, seqlen, nheads, head_dim).
 from __future__ import annotations
 
 import numpy as np
+
+
+def kv_head(h: int, H: int, Hk: int) -> int:
+    """Key/value head used by query head h when K and V have Hk of H heads."""
+    if Hk < 1 or H % Hk != 0:
+        raise ValueError(f"query heads {H} not a multiple of key/value heads {Hk}")
+    return h // (H // Hk)
 
 
 def _f64(x):
@@ -95,8 +108,8 @@ def attention_forward(q, k, v, scale: float, causal: int = 0,
                       win_left: int = -1, win_right: int = -1):
     """O and LSE of exact attention, the three standard steps in float64.
 
-    q: (B, Sq, H, D); k, v: (B, Sk, H, D).  Returns o (B, Sq, H, D) float64
-    and lse (B, H, Sq) float64 (natural log).
+    q: (B, Sq, H, D); k, v: (B, Sk, Hk, D) with H a multiple of Hk.  Returns
+    o (B, Sq, H, D) float64 and lse (B, H, Sq) float64 (natural log).
     FlashAttention-2 overview (lshu.cn), section 2.1: S = Q K^T, row softmax,
     weighted sum of V.
     """
@@ -106,12 +119,14 @@ def attention_forward(q, k, v, scale: float, causal: int = 0,
     o = np.zeros((B, Sq, H, D), dtype=np.float64)
     lse = np.zeros((B, H, Sq), dtype=np.float64)
     rows = np.arange(Sq)
+    Hk = k.shape[2]
     for b in range(B):
         for h in range(H):
-            S = _scores(q[b, :, h, :], k[b, :, h, :], scale, rows, Sq, Sk,
+            g = kv_head(h, H, Hk)
+            S = _scores(q[b, :, h, :], k[b, :, g, :], scale, rows, Sq, Sk,
                         causal, win_left, win_right)
             P, l = _softmax_rows(S)
-            o[b, :, h, :] = P @ v[b, :, h, :]
+            o[b, :, h, :] = P @ v[b, :, g, :]
             lse[b, h, :] = l
     return o, lse
 
@@ -135,8 +150,9 @@ def attention_forward_rows(q, k, v, triples, scale: float, causal: int = 0,
     for bh in np.unique(keys):
         sel = np.nonzero(keys == bh)[0]
         b, h = int(bh // H), int(bh % H)
-        kh = _f64(k[b, :, h, :])
-        vh = _f64(v[b, :, h, :])
+        g = kv_head(h, H, k.shape[2])
+        kh = _f64(k[b, :, g, :])
+        vh = _f64(v[b, :, g, :])
         for c0 in range(0, len(sel), 1024):
             s = sel[c0:c0 + 1024]
             rows = triples[s, 2]
@@ -163,7 +179,8 @@ def attention_backward(q, k, v, do, scale: float, causal: int = 0,
                        win_left: int = -1, win_right: int = -1):
     """Analytic gradient of L = sum(O * dO) with respect to Q, K and V.
 
-    Returns a dict with o, lse, delta (B, H, Sq), dq, dk, dv (float64).
+    Returns a dict with o, lse, delta (B, H, Sq), dq, dk, dv (float64); with
+    fewer K/V heads, dk and dv of a K/V head sum over its query heads.
     dV = P^T dO; dP = dO V^T; Delta = rowsum(P * dP) (= rowsum(dO * O));
     dS = P * (dP - Delta); dQ = scale dS K; dK = scale dS^T Q.
     """
@@ -175,17 +192,19 @@ def attention_backward(q, k, v, do, scale: float, causal: int = 0,
     out["lse"] = np.zeros((B, H, Sq))
     out["delta"] = np.zeros((B, H, Sq))
     rows = np.arange(Sq)
+    Hk = k.shape[2]
     for b in range(B):
         for h in range(H):
-            qh, kh, vh, doh = q[b, :, h], k[b, :, h], v[b, :, h], do[b, :, h]
+            g = kv_head(h, H, Hk)
+            qh, kh, vh, doh = q[b, :, h], k[b, :, g], v[b, :, g], do[b, :, h]
             O, lse, delta, P, dS = _head_backward(qh, kh, vh, doh, scale, rows,
                                                   Sq, Sk, causal, win_left, win_right)
             out["o"][b, :, h] = O
             out["lse"][b, h] = lse
             out["delta"][b, h] = delta
-            out["dv"][b, :, h] = P.T @ doh
+            out["dv"][b, :, g] += P.T @ doh
             out["dq"][b, :, h] = scale * (dS @ kh)
-            out["dk"][b, :, h] = scale * (dS.T @ qh)
+            out["dk"][b, :, g] += scale * (dS.T @ qh)
     return out
 
 
@@ -205,7 +224,8 @@ def attention_backward_rows_dq(q, k, v, do, triples, scale: float, causal: int =
     for bh in np.unique(keys):
         sel = np.nonzero(keys == bh)[0]
         b, h = int(bh // H), int(bh % H)
-        kh, vh = _f64(k[b, :, h]), _f64(v[b, :, h])
+        g = kv_head(h, H, k.shape[2])
+        kh, vh = _f64(k[b, :, g]), _f64(v[b, :, g])
         for c0 in range(0, len(sel), 1024):
             s = sel[c0:c0 + 1024]
             rows = triples[s, 2]
@@ -229,7 +249,8 @@ def attention_backward_rows(q, k, v, do, b: int, h: int, rows, scale: float,
     rows = np.asarray(rows, dtype=np.int64)
     Sq = q.shape[1]
     Sk = k.shape[1]
-    kh, vh = _f64(k[b, :, h]), _f64(v[b, :, h])
+    g = kv_head(h, q.shape[2], k.shape[2])
+    kh, vh = _f64(k[b, :, g]), _f64(v[b, :, g])
     qh, doh = _f64(q[b, rows, h]), _f64(do[b, rows, h])
     O, lse, _, P, dS = _head_backward(qh, kh, vh, doh, scale, rows, Sq, Sk,
                                       causal, win_left, win_right)
@@ -239,7 +260,9 @@ def attention_backward_rows(q, k, v, do, b: int, h: int, rows, scale: float,
 def attention_backward_head(q, k, v, do, b: int, h: int, scale: float,
                             causal: int = 0, win_left: int = -1, win_right: int = -1,
                             row_chunk: int = 1024):
-    """dK and dV (Sk, D) of one (batch, head); query rows are taken in chunks.
+    """Query head h's share of dK and dV (Sk, D) of its (batch, K/V head);
+    query rows are taken in chunks.  With as many K/V heads as query heads
+    this is the head's dK and dV.
 
     dK and dV sum over every query row, so every row's softmax and Delta is
     evaluated; chunking the rows only bounds memory.
@@ -255,6 +278,23 @@ def attention_backward_head(q, k, v, do, b: int, h: int, scale: float,
                                                     causal, win_left, win_right)
         dk += dkp
         dv += dvp
+    return dk, dv
+
+
+def attention_backward_kv_head(q, k, v, do, b: int, g: int, scale: float,
+                               causal: int = 0, win_left: int = -1, win_right: int = -1,
+                               row_chunk: int = 1024):
+    """dK and dV (Sk, D) of K/V head g of batch b: the sum over the query
+    heads that share it (just one when the head counts are equal)."""
+    H, Hk = q.shape[2], k.shape[2]
+    dk = np.zeros((k.shape[1], k.shape[3]))
+    dv = np.zeros_like(dk)
+    for h in range(H):
+        if kv_head(h, H, Hk) == g:
+            dkh, dvh = attention_backward_head(q, k, v, do, b, h, scale, causal,
+                                               win_left, win_right, row_chunk)
+            dk += dkh
+            dv += dvh
     return dk, dv
 
 
@@ -280,13 +320,14 @@ def online_softmax_forward(q, k, v, scale: float, tile: int, causal: int = 0,
     lse = np.zeros((B, H, Sq))
     for b in range(B):
         for h in range(H):
+            g = kv_head(h, H, k.shape[2])
             for i in range(Sq):
                 m_i = -np.inf
                 l_i = 0.0
                 acc = np.zeros(D)
                 for j0 in range(0, Sk, tile):
                     j1 = min(Sk, j0 + tile)
-                    s = scale * (k[b, j0:j1, h] @ q[b, i, h])
+                    s = scale * (k[b, j0:j1, g] @ q[b, i, h])
                     s = np.where(vis[i, j0:j1], s, -np.inf)
                     m_new = max(m_i, float(np.max(s)))
                     if m_new == -np.inf:
@@ -294,7 +335,7 @@ def online_softmax_forward(q, k, v, scale: float, tile: int, causal: int = 0,
                     alpha = np.exp(m_i - m_new)  # exp(-inf) = 0 on the first visible tile
                     p = np.exp(s - m_new)
                     l_i = l_i * alpha + float(np.sum(p))
-                    acc = acc * alpha + p @ v[b, j0:j1, h]
+                    acc = acc * alpha + p @ v[b, j0:j1, g]
                     m_i = m_new
                 if l_i > 0.0:
                     o[b, i, h] = acc / l_i
