@@ -35,8 +35,12 @@ sys.path.insert(0, ROOT)
 
 METRIC = "attention fwd/bwd TFLOPS at seq 8K–32K, D=128, bf16 vs B200 dense BF16 peak"
 UNIT = "TFLOP/s"
-WORKLOAD = dict(name="c5_b1h32s8192d128_fwdbwd", B=1, H=32, Sq=8192, Sk=8192, D=128,
+WORKLOAD = dict(name="c5_b1h32s8192d128_fwdbwd", B=1, H=32, Hk=32, Sq=8192, Sk=8192, D=128,
                 causal=1, win_left=-1, win_right=-1, input_scale=0.5, seed=1005)
+# grouped K/V heads (GQA, 4 query heads per K/V head) at the same sizes
+GQA_WORKLOAD = dict(name="gqa_b1h32hk8s8192d128_fwdbwd", B=1, H=32, Hk=8, Sq=8192, Sk=8192,
+                    D=128, causal=1, win_left=-1, win_right=-1, input_scale=0.5, seed=1006)
+WORKLOADS = {"fwdbwd": WORKLOAD, "gqa": GQA_WORKLOAD}
 FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "hbm_gbs": 6650.0, "source": "fallback"}
 BWD_KERNEL_SOURCES = ["bwd_sm100.cuh", "ptx.cuh", "common.cuh"]
 FWD_KERNEL_SOURCES = ["fwd_sm100.cuh", "ptx.cuh", "common.cuh"]
@@ -127,6 +131,12 @@ def sources_sha(files) -> str:
     return h.hexdigest()[:12]
 
 
+def traffic_key(kernel: str, w) -> str:
+    """Name of a kernel's line in profiles/traffic_per_launch.txt: the kernel for
+    the headline workload, kernel@workload for the others."""
+    return kernel if w is WORKLOAD else f"{kernel}@{w['name']}"
+
+
 def committed_traffic(kernel: str, sha: str):
     """DRAM bytes per launch recorded from an ncu capture, if the kernel's
     sources have not changed since (profiles/traffic_per_launch.txt)."""
@@ -196,7 +206,7 @@ class ClockSampler:
 def oracle_sample_inputs(w):
     from synth import bf16_bits_to_f32, make_inputs
     bits = make_inputs(w["B"], w["Sq"], w["Sk"], w["H"], w["D"], w["seed"], w["input_scale"],
-                       with_dout=True)
+                       with_dout=True, Hk=w["Hk"])
     return {n: bf16_bits_to_f32(bits[n]) for n in ("q", "k", "v", "do")}
 
 
@@ -246,7 +256,7 @@ def run_reference(args):
     rank, world, _ = dist_env()
     if rank != 0:
         return 0
-    w = WORKLOAD
+    w = WORKLOADS[args.workload]
     inputs = oracle_sample_inputs(w)
     for i in range(args.warmup):
         oracle_sample(inputs, w, 1000 + i)
@@ -272,11 +282,16 @@ def run_reference(args):
 
 
 def config_dict(w):
-    return {"workload": f"{w['name']}: fwd+bwd, B={w['B']} H={w['H']} Sq=Sk={w['Sq']} "
-                        f"D={w['D']} causal bf16, inputs N(0,1)*{w['input_scale']}",
-            "B": w["B"], "H": w["H"], "Sq": w["Sq"], "Sk": w["Sk"], "D": w["D"],
-            "causal": bool(w["causal"]),
-            "l2": "no flush: inputs (Q,K,V,dO 256 MiB) and outputs exceed the 126 MB L2"}
+    heads = f"H={w['H']}" + (f" Hk={w['Hk']}" if w["Hk"] != w["H"] else "")
+    in_mib = 2 * w["B"] * w["D"] * 2 * (w["Sq"] * w["H"] + w["Sk"] * w["Hk"]) / 2**20
+    d = {"workload": f"{w['name']}: fwd+bwd, B={w['B']} {heads} Sq=Sk={w['Sq']} "
+                     f"D={w['D']} causal bf16, inputs N(0,1)*{w['input_scale']}",
+         "B": w["B"], "H": w["H"], "Sq": w["Sq"], "Sk": w["Sk"], "D": w["D"],
+         "causal": bool(w["causal"]),
+         "l2": f"no flush: inputs (Q,K,V,dO {in_mib:.0f} MiB) and outputs exceed the 126 MB L2"}
+    if w["Hk"] != w["H"]:
+        d["Hk"] = w["Hk"]
+    return d
 
 
 # ---------------------------------------------------------------------------
@@ -296,11 +311,12 @@ def run_gpu(args):
                                           get_last_device_error)
     from synth import make_inputs
 
-    w = WORKLOAD
+    w = WORKLOADS[args.workload]
     B, H, Sq, Sk, D = w["B"], w["H"], w["Sq"], w["Sk"], w["D"]
     causal = bool(w["causal"])
     win = (w["win_left"], w["win_right"])
-    bits = make_inputs(B, Sq, Sk, H, D, w["seed"] + rank, w["input_scale"], with_dout=True)
+    bits = make_inputs(B, Sq, Sk, H, D, w["seed"] + rank, w["input_scale"], with_dout=True,
+                       Hk=w["Hk"])
     host = {n: torch.from_numpy(bits[n].view("int16")).view(torch.bfloat16).pin_memory()
             for n in ("q", "k", "v", "do")}
     dev = {n: t.to(device) for n, t in host.items()}
@@ -403,13 +419,13 @@ def run_gpu(args):
                      "achieved": bwd_main_tflops, "peak": peak, "unit": "TFLOP/s",
                      "frac": bwd_main_tflops / peak,
                      "peak_source": f"{peaks.get('source')} bf16_tflops (burst)",
-                     "traffic": committed_traffic("attn_bwd_main_kernel",
+                     "traffic": committed_traffic(traffic_key("attn_bwd_main_kernel", w),
                                                   sources_sha(BWD_KERNEL_SOURCES))},
         "kernels": kernels,
         "fwd_roofline": {"bound": "tensor", "kernel": "attn_fwd_kernel<128>",
                          "achieved": fwd_tflops, "peak": peak, "unit": "TFLOP/s",
                          "frac": fwd_tflops / peak,
-                         "traffic": committed_traffic("attn_fwd_kernel",
+                         "traffic": committed_traffic(traffic_key("attn_fwd_kernel", w),
                                                       sources_sha(FWD_KERNEL_SOURCES))},
         "e2e": e2e,
         "gpu_launches": launches,
@@ -431,6 +447,9 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="fwdbwd",
+                    help="fwdbwd: the headline fwd+bwd workload (default); gqa: the same sizes "
+                         "with 8 K/V heads for 32 query heads")
     ap.add_argument("--no-cpu-baseline", action="store_true",
                     help="skip the timed oracle sample (it adds ~15 s of CPU time)")
     ap.add_argument("--no-e2e", action="store_true",

@@ -48,6 +48,14 @@ def _load() -> ctypes.CDLL:
     lib.attn_bwd_main.restype = i
     lib.attn_bwd_dq_finalize.argtypes = [vp, i, i, i, i, f, vp, sz, vp]
     lib.attn_bwd_dq_finalize.restype = i
+    lib.attn_fwd_gqa.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, i, i, vp]
+    lib.attn_fwd_gqa.restype = i
+    lib.attn_bwd_gqa.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, i,
+                                 i, vp, sz, vp]
+    lib.attn_bwd_gqa.restype = i
+    lib.attn_bwd_main_gqa.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, i, i, vp,
+                                      sz, vp]
+    lib.attn_bwd_main_gqa.restype = i
     lib.attn_bwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, i,
                                      i, vp]
     lib.attn_bwd_noalloc.restype = i
@@ -90,6 +98,15 @@ def _check(t, name, dtype, ndim):
         raise ValueError(f"{name} must be contiguous (batch, seqlen, nheads, head_dim)")
 
 
+def _kv_heads(q, k, v):
+    """K/V head count; fewer than q's heads selects grouped K/V heads (GQA/MQA)."""
+    H, Hk = q.shape[2], k.shape[2]
+    if v.shape[2] != Hk or Hk < 1 or H % Hk != 0:
+        raise ValueError(f"k and v must have the same number of heads, dividing q's {H}: "
+                         f"k {tuple(k.shape)}, v {tuple(v.shape)}")
+    return Hk
+
+
 def _scale(softmax_scale, D):
     return float(1.0 / math.sqrt(D)) if softmax_scale is None else float(softmax_scale)
 
@@ -102,8 +119,10 @@ def _window(causal, window_size):
 def attn_fwd(q, k, v, softmax_scale: Optional[float] = None, causal: bool = False,
              window_size: Optional[Tuple[int, int]] = None, out=None, lse=None,
              stream=None):
-    """O, LSE = exact attention of q (B,Sq,H,D), k, v (B,Sk,H,D), all bf16 CUDA.
+    """O, LSE = exact attention of q (B,Sq,H,D), k, v (B,Sk,Hk,D), all bf16 CUDA.
 
+    Hk = H is ordinary multi-head attention; Hk < H (a divisor of H) shares each
+    K/V head among H/Hk consecutive query heads (GQA; MQA when Hk = 1).
     ``softmax_scale=None`` means 1/sqrt(D).  ``window_size=(left, right)`` with
     -1 for an unbounded side.  Returns (o bf16 (B,Sq,H,D), lse fp32 (B,H,Sq)).
     """
@@ -119,11 +138,15 @@ def attn_fwd(q, k, v, softmax_scale: Optional[float] = None, causal: bool = Fals
     _check(out, "out", torch.bfloat16, 4)
     _check(lse, "lse", torch.float32, 3)
     c, wl, wr = _window(causal, window_size)
-    st = lib.attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
-                      B, Sq, Sk, H, D, _scale(softmax_scale, D), c, wl, wr,
-                      _stream_handle(stream, q.device))
+    Hk = _kv_heads(q, k, v)
+    args = (q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(), B, Sq, Sk)
+    tail = (D, _scale(softmax_scale, D), c, wl, wr, _stream_handle(stream, q.device))
+    if Hk == H:
+        st, name = lib.attn_fwd(*args, H, *tail), "attn_fwd"
+    else:
+        st, name = lib.attn_fwd_gqa(*args, H, Hk, *tail), "attn_fwd_gqa"
     if st != 0:
-        raise AttnError(st, "attn_fwd")
+        raise AttnError(st, name)
     return out, lse
 
 
@@ -152,13 +175,17 @@ def attn_bwd(q, k, v, out, dout, lse, softmax_scale: Optional[float] = None,
     if workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     c, wl, wr = _window(causal, window_size)
-    st = lib.attn_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), dout.data_ptr(),
-                      lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
-                      B, Sq, Sk, H, D, _scale(softmax_scale, D), c, wl, wr,
-                      workspace.data_ptr(), workspace.numel() * workspace.element_size(),
-                      _stream_handle(stream, q.device))
+    Hk = _kv_heads(q, k, v)
+    args = (q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), dout.data_ptr(),
+            lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, Sq, Sk)
+    tail = (D, _scale(softmax_scale, D), c, wl, wr, workspace.data_ptr(),
+            workspace.numel() * workspace.element_size(), _stream_handle(stream, q.device))
+    if Hk == H:
+        st, name = lib.attn_bwd(*args, H, *tail), "attn_bwd"
+    else:
+        st, name = lib.attn_bwd_gqa(*args, H, Hk, *tail), "attn_bwd_gqa"
     if st != 0:
-        raise AttnError(st, "attn_bwd")
+        raise AttnError(st, name)
     return dq, dk, dv
 
 
@@ -185,10 +212,16 @@ def attn_bwd_stages(q, k, v, out, dout, lse, dq, dk, dv, workspace,
         raise AttnError(st, "attn_bwd_preprocess")
     if between:
         between(1)
-    st = lib.attn_bwd_main(q.data_ptr(), k.data_ptr(), v.data_ptr(), dout.data_ptr(),
-                           dk.data_ptr(), dv.data_ptr(), B, Sq, Sk, H, D, sc, c, wl, wr, wp, wb, hs)
+    Hk = _kv_heads(q, k, v)
+    args = (q.data_ptr(), k.data_ptr(), v.data_ptr(), dout.data_ptr(), dk.data_ptr(),
+            dv.data_ptr(), B, Sq, Sk)
+    if Hk == H:
+        st, name = lib.attn_bwd_main(*args, H, D, sc, c, wl, wr, wp, wb, hs), "attn_bwd_main"
+    else:
+        st, name = (lib.attn_bwd_main_gqa(*args, H, Hk, D, sc, c, wl, wr, wp, wb, hs),
+                    "attn_bwd_main_gqa")
     if st != 0:
-        raise AttnError(st, "attn_bwd_main")
+        raise AttnError(st, name)
     if between:
         between(2)
     st = lib.attn_bwd_dq_finalize(dq.data_ptr(), B, Sq, H, D, sc, wp, wb, hs)

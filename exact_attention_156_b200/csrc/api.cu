@@ -116,12 +116,13 @@ bool on_current_device(const void* p) {
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 attn_status check_common(int B, int Sq, int Sk, int H, int D, float scale, int win_left,
-                         int win_right) {
+                         int win_right, int Hk = -1) {
+  if (Hk < 0) Hk = H;
   if (B < 1 || Sq < 1 || Sk < 1 || H < 1) return ATTN_ERR_SHAPE;
   if (B > 65535 || H > 65535) return ATTN_ERR_SHAPE;
+  if (Hk < 1 || Hk > H || H % Hk != 0) return ATTN_ERR_SHAPE;
   if (D != 64 && D != 128) return ATTN_ERR_HEADDIM;
-  const long long row = (long long)H * D;
-  if ((long long)B * Sq * row >= (1ll << 31) || (long long)B * Sk * row >= (1ll << 31))
+  if ((long long)B * Sq * H * D >= (1ll << 31) || (long long)B * Sk * Hk * D >= (1ll << 31))
     return ATTN_ERR_SHAPE;
   if (!(scale > 0.f) || !isfinite(scale)) return ATTN_ERR_SHAPE;
   if (win_left < -1 || win_right < -1) return ATTN_ERR_WINDOW;
@@ -165,17 +166,18 @@ size_t workspace_bytes(int B, int Sq, int H, int D) {
 
 template <int D>
 attn_status launch_fwd(const DeviceState& st, const void* q, const void* k, const void* v, void* o,
-                       float* lse, int B, int Sq, int Sk, int H, float scale, int causal,
+                       float* lse, int B, int Sq, int Sk, int H, int Hk, float scale, int causal,
                        int win_left, int win_right, cudaStream_t stream) {
   alignas(64) CUtensorMap mq, mk, mv;
-  if (make_map(&mq, q, B, Sq, H, D) != ATTN_OK || make_map(&mk, k, B, Sk, H, D) != ATTN_OK ||
-      make_map(&mv, v, B, Sk, H, D) != ATTN_OK)
+  if (make_map(&mq, q, B, Sq, H, D) != ATTN_OK || make_map(&mk, k, B, Sk, Hk, D) != ATTN_OK ||
+      make_map(&mv, v, B, Sk, Hk, D) != ATTN_OK)
     return ATTN_ERR_LAUNCH;
   fwd::Params p;
   p.o = static_cast<__nv_bfloat16*>(o);
   p.lse = lse;
   p.B = B;
   p.H = H;
+  p.Hk = Hk;
   p.Sq = Sq;
   p.Sk = Sk;
   p.scale_log2 = scale * 1.4426950408889634f;
@@ -221,11 +223,11 @@ attn_status launch_bwd_pre(const void* o, const void* dout, const float* lse, in
 template <int D>
 attn_status launch_bwd_main(const DeviceState& st, const void* q, const void* k, const void* v,
                             const void* dout, void* dk, void* dv, int B, int Sq, int Sk, int H,
-                            float scale, int causal, int win_left, int win_right,
+                            int Hk, float scale, int causal, int win_left, int win_right,
                             const Workspace& w, cudaStream_t stream) {
   alignas(64) CUtensorMap mq, mk, mv, mdo, mdq;
-  if (make_map(&mq, q, B, Sq, H, D) != ATTN_OK || make_map(&mk, k, B, Sk, H, D) != ATTN_OK ||
-      make_map(&mv, v, B, Sk, H, D) != ATTN_OK || make_map(&mdo, dout, B, Sq, H, D) != ATTN_OK ||
+  if (make_map(&mq, q, B, Sq, H, D) != ATTN_OK || make_map(&mk, k, B, Sk, Hk, D) != ATTN_OK ||
+      make_map(&mv, v, B, Sk, Hk, D) != ATTN_OK || make_map(&mdo, dout, B, Sq, H, D) != ATTN_OK ||
       make_dq_map(&mdq, w.dq_acc, (long long)B * H * w.Sq_pad, D) != ATTN_OK)
     return ATTN_ERR_LAUNCH;
   bwd::Params p;
@@ -239,6 +241,7 @@ attn_status launch_bwd_main(const DeviceState& st, const void* q, const void* k,
   p.Sq = Sq;
   p.Sk = Sk;
   p.Sq_pad = w.Sq_pad;
+  p.Hk = Hk;
   p.scale = scale;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.causal = causal ? 1 : 0;
@@ -246,7 +249,7 @@ attn_status launch_bwd_main(const DeviceState& st, const void* q, const void* k,
   p.win_right = win_right;
   p.err = st.err;
   p.timeout_ns = kTimeoutNs;
-  dim3 grid((Sk + bwd::BN - 1) / bwd::BN, H, B);
+  dim3 grid((Sk + bwd::BN - 1) / bwd::BN, Hk, B);
   bwd::attn_bwd_main_kernel<D>
       <<<grid, bwd::kThreads, bwd::Cfg<D>::kSmemBytes, stream>>>(mq, mk, mv, mdo, mdq, p);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_LAUNCH;
@@ -343,11 +346,11 @@ const char* attn_status_string(attn_status s) {
   return "unknown status";
 }
 
-attn_status attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B,
-                     int Sq, int Sk, int H, int D, float scale, int causal, int win_left,
-                     int win_right, void* stream) {
+attn_status attn_fwd_gqa(const void* q, const void* k, const void* v, void* o, float* lse,
+                         int B, int Sq, int Sk, int H, int Hk, int D, float scale, int causal,
+                         int win_left, int win_right, void* stream) {
   if (!q || !k || !v || !o || !lse) return ATTN_ERR_NULLPTR;
-  attn_status s = check_common(B, Sq, Sk, H, D, scale, win_left, win_right);
+  attn_status s = check_common(B, Sq, Sk, H, D, scale, win_left, win_right, Hk);
   if (s != ATTN_OK) return s;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) ||
       (reinterpret_cast<uintptr_t>(lse) & 3u))
@@ -360,8 +363,17 @@ attn_status attn_fwd(const void* q, const void* k, const void* v, void* o, float
     return ATTN_ERR_DEVICE;
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
   if (D == 64)
-    return launch_fwd<64>(*st, q, k, v, o, lse, B, Sq, Sk, H, scale, causal, win_left, win_right, cs);
-  return launch_fwd<128>(*st, q, k, v, o, lse, B, Sq, Sk, H, scale, causal, win_left, win_right, cs);
+    return launch_fwd<64>(*st, q, k, v, o, lse, B, Sq, Sk, H, Hk, scale, causal, win_left,
+                          win_right, cs);
+  return launch_fwd<128>(*st, q, k, v, o, lse, B, Sq, Sk, H, Hk, scale, causal, win_left,
+                         win_right, cs);
+}
+
+attn_status attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                     int Sq, int Sk, int H, int D, float scale, int causal, int win_left,
+                     int win_right, void* stream) {
+  return attn_fwd_gqa(q, k, v, o, lse, B, Sq, Sk, H, H, D, scale, causal, win_left, win_right,
+                      stream);
 }
 
 size_t attn_bwd_workspace_size(int B, int Sq, int H, int D) {
@@ -369,12 +381,13 @@ size_t attn_bwd_workspace_size(int B, int Sq, int H, int D) {
   return workspace_bytes(B, Sq, H, D);
 }
 
-attn_status attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
-                     const float* lse, void* dq, void* dk, void* dv, int B, int Sq, int Sk, int H,
-                     int D, float scale, int causal, int win_left, int win_right, void* workspace,
-                     size_t workspace_size, void* stream) {
+attn_status attn_bwd_gqa(const void* q, const void* k, const void* v, const void* o,
+                         const void* dout, const float* lse, void* dq, void* dk, void* dv, int B,
+                         int Sq, int Sk, int H, int Hk, int D, float scale, int causal,
+                         int win_left, int win_right, void* workspace, size_t workspace_size,
+                         void* stream) {
   if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv) return ATTN_ERR_NULLPTR;
-  attn_status s = check_common(B, Sq, Sk, H, D, scale, win_left, win_right);
+  attn_status s = check_common(B, Sq, Sk, H, D, scale, win_left, win_right, Hk);
   if (s != ATTN_OK) return s;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) ||
       !aligned16(dq) || !aligned16(dk) || !aligned16(dv) ||
@@ -391,17 +404,25 @@ attn_status attn_bwd(const void* q, const void* k, const void* v, const void* o,
   if (D == 64) {
     s = launch_bwd_pre<64>(o, dout, lse, B, Sq, H, w, cs);
     if (s == ATTN_OK)
-      s = launch_bwd_main<64>(*st, q, k, v, dout, dk, dv, B, Sq, Sk, H, scale, causal, win_left,
-                              win_right, w, cs);
+      s = launch_bwd_main<64>(*st, q, k, v, dout, dk, dv, B, Sq, Sk, H, Hk, scale, causal,
+                              win_left, win_right, w, cs);
     if (s == ATTN_OK) s = launch_bwd_dq<64>(dq, B, Sq, H, scale, w, cs);
   } else {
     s = launch_bwd_pre<128>(o, dout, lse, B, Sq, H, w, cs);
     if (s == ATTN_OK)
-      s = launch_bwd_main<128>(*st, q, k, v, dout, dk, dv, B, Sq, Sk, H, scale, causal, win_left,
-                               win_right, w, cs);
+      s = launch_bwd_main<128>(*st, q, k, v, dout, dk, dv, B, Sq, Sk, H, Hk, scale, causal,
+                               win_left, win_right, w, cs);
     if (s == ATTN_OK) s = launch_bwd_dq<128>(dq, B, Sq, H, scale, w, cs);
   }
   return s;
+}
+
+attn_status attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                     const float* lse, void* dq, void* dk, void* dv, int B, int Sq, int Sk, int H,
+                     int D, float scale, int causal, int win_left, int win_right, void* workspace,
+                     size_t workspace_size, void* stream) {
+  return attn_bwd_gqa(q, k, v, o, dout, lse, dq, dk, dv, B, Sq, Sk, H, H, D, scale, causal,
+                      win_left, win_right, workspace, workspace_size, stream);
 }
 
 attn_status attn_bwd_preprocess(const void* o, const void* dout, const float* lse, int B, int Sq,
@@ -424,12 +445,12 @@ attn_status attn_bwd_preprocess(const void* o, const void* dout, const float* ls
                  : launch_bwd_pre<128>(o, dout, lse, B, Sq, H, w, cs);
 }
 
-attn_status attn_bwd_main(const void* q, const void* k, const void* v, const void* dout,
-                          void* dk, void* dv, int B, int Sq, int Sk, int H, int D, float scale,
-                          int causal, int win_left, int win_right, void* workspace,
-                          size_t workspace_size, void* stream) {
+attn_status attn_bwd_main_gqa(const void* q, const void* k, const void* v, const void* dout,
+                              void* dk, void* dv, int B, int Sq, int Sk, int H, int Hk, int D,
+                              float scale, int causal, int win_left, int win_right,
+                              void* workspace, size_t workspace_size, void* stream) {
   if (!q || !k || !v || !dout || !dk || !dv) return ATTN_ERR_NULLPTR;
-  attn_status s = check_common(B, Sq, Sk, H, D, scale, win_left, win_right);
+  attn_status s = check_common(B, Sq, Sk, H, D, scale, win_left, win_right, Hk);
   if (s != ATTN_OK) return s;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dout) || !aligned16(dk) ||
       !aligned16(dv))
@@ -442,10 +463,18 @@ attn_status attn_bwd_main(const void* q, const void* k, const void* v, const voi
   if (!all_on_device({q, k, v, dout, dk, dv, workspace})) return ATTN_ERR_DEVICE;
   const Workspace w = carve(workspace, B, Sq, H, D);
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
-  return D == 64 ? launch_bwd_main<64>(*st, q, k, v, dout, dk, dv, B, Sq, Sk, H, scale, causal,
-                                       win_left, win_right, w, cs)
-                 : launch_bwd_main<128>(*st, q, k, v, dout, dk, dv, B, Sq, Sk, H, scale, causal,
-                                        win_left, win_right, w, cs);
+  return D == 64 ? launch_bwd_main<64>(*st, q, k, v, dout, dk, dv, B, Sq, Sk, H, Hk, scale,
+                                       causal, win_left, win_right, w, cs)
+                 : launch_bwd_main<128>(*st, q, k, v, dout, dk, dv, B, Sq, Sk, H, Hk, scale,
+                                        causal, win_left, win_right, w, cs);
+}
+
+attn_status attn_bwd_main(const void* q, const void* k, const void* v, const void* dout,
+                          void* dk, void* dv, int B, int Sq, int Sk, int H, int D, float scale,
+                          int causal, int win_left, int win_right, void* workspace,
+                          size_t workspace_size, void* stream) {
+  return attn_bwd_main_gqa(q, k, v, dout, dk, dv, B, Sq, Sk, H, H, D, scale, causal, win_left,
+                           win_right, workspace, workspace_size, stream);
 }
 
 attn_status attn_bwd_dq_finalize(void* dq, int B, int Sq, int H, int D, float scale,
@@ -492,14 +521,14 @@ attn_status attn_bwd_noalloc(const void* q, const void* k, const void* v, const 
   if (D == 64) {
     s = launch_bwd_pre<64>(o, dout, lse, B, Sq, H, w, cs);
     if (s == ATTN_OK)
-      s = launch_bwd_main<64>(*st, q, k, v, dout, dk, dv, B, Sq, Sk, H, scale, causal, win_left,
-                              win_right, w, cs);
+      s = launch_bwd_main<64>(*st, q, k, v, dout, dk, dv, B, Sq, Sk, H, H, scale, causal,
+                              win_left, win_right, w, cs);
     if (s == ATTN_OK) s = launch_bwd_dq<64>(dq, B, Sq, H, scale, w, cs);
   } else {
     s = launch_bwd_pre<128>(o, dout, lse, B, Sq, H, w, cs);
     if (s == ATTN_OK)
-      s = launch_bwd_main<128>(*st, q, k, v, dout, dk, dv, B, Sq, Sk, H, scale, causal, win_left,
-                               win_right, w, cs);
+      s = launch_bwd_main<128>(*st, q, k, v, dout, dk, dv, B, Sq, Sk, H, H, scale, causal,
+                               win_left, win_right, w, cs);
     if (s == ATTN_OK) s = launch_bwd_dq<128>(dq, B, Sq, H, scale, w, cs);
   }
   return s;

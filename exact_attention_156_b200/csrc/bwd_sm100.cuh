@@ -13,8 +13,10 @@
 //  1. bwd_pre: -Delta_i (fp32), -LSE in base 2 (padded rows: -inf so P = 0),
 //     and zeroes the fp32 dQ accumulator.  Memory bound.  Both row values are
 //     stored negated so the main kernel adds them with packed fp32 pairs.
-//  2. bwd_main: one CTA per (128-key tile, head, batch); K_j and V_j stay in
-//     shared memory while the CTA streams the query tiles that can see them.
+//  2. bwd_main: one CTA per (128-key tile, key/value head, batch); K_j and V_j
+//     stay in shared memory while the CTA streams the query tiles that can see
+//     them, for every query head that reads this K/V head (one, or H / Hk with
+//     grouped K/V heads), so dK_j and dV_j accumulate in tensor memory.
 //     Transposed products put the key index on tensor-memory lanes:
 //       S^T = K Q^T  and  dP^T = V dO^T   (M = keys, N = queries, K = D)
 //       dV += P^T dO  (A = P^T from tensor memory)
@@ -106,6 +108,7 @@ struct Params {
   const float* ndelta;  // [B*H][Sq_pad] -Delta
   float* dq_acc;       // [B*H][Sq_pad][D]
   int B, H, Sq, Sk, Sq_pad;
+  int Hk;  // key/value heads: the CTA's K/V head is shared by H / Hk query heads
   float scale;
   float scale_log2;
   int causal, win_left, win_right;
@@ -237,15 +240,20 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 
   const int kt = blockIdx.x;  // key tile; low indices see the most query tiles when causal
-  const int h = blockIdx.y;
+  const int hk = blockIdx.y;  // key/value head
   const int b = blockIdx.z;
-  const int bh = b * p.H + h;
+  const int group = p.H / p.Hk;  // query heads sharing this K/V head
   const MaskGeom g = MaskGeom::make(p.Sq, p.Sk, p.causal, p.win_left, p.win_right);
   const int n0 = kt * BN;
   const int n1 = min(n0 + BN - 1, p.Sk - 1);
   int qlo, qhi;
   qtile_range(g, n0, n1, qlo, qhi);
-  const int nq = qhi - qlo;
+  const int nq_head = qhi - qlo;  // query tiles per query head
+  // Work item t of this CTA: query head hk * group + t / nq_head, query tile
+  // qlo + t % nq_head.  dK and dV of the K/V head accumulate over all of them.
+  const int nq = nq_head * group;
+  auto item_head = [&](int t) { return hk * group + t / nq_head; };
+  auto item_row0 = [&](int t) { return (qlo + t % nq_head) * BM; };
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::kNumBars; ++i) {
@@ -327,7 +335,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     for (int t = 0; t < nq; ++t) {
       const int s = t % kQStages;
-      const int i0 = (qlo + t) * BM;
+      const int i0 = item_row0(t);
       const float4* nl = reinterpret_cast<const float4*>(smem + C::kLseOff + s * BM * 4);
       const float4* nd = reinterpret_cast<const float4*>(smem + C::kDeltaOff + s * BM * 4);
       // P = 2^(scale*log2e*S - LSE*log2e), kept as bf16 pairs (what dV uses) for dS too
@@ -424,7 +432,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (ok && nq > 0) ok = bw.wait_warp(bar(C::kBarDSEmpty), (nq - 1) & 1, 30);
     if (ok) {
       tc_fence_after();
-      const size_t orow = ((size_t(b) * p.Sk + size_t(kk_idx)) * p.H + h) * D;
+      const size_t orow = ((size_t(b) * p.Sk + size_t(kk_idx)) * p.Hk + hk) * D;
 #pragma unroll 1
       for (int which = 0; which < 2; ++which) {
         const uint32_t col = which == 0 ? C::kColDK : C::kColDV;
@@ -481,7 +489,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // tensor memory is free again: the MMA warp may start dP of the next tile
       tc_fence_before();
       mbar_arrive(bar(C::kBarDQEmpty));
-      const int row0 = bh * p.Sq_pad + (qlo + t) * BM;
+      const int row0 = (b * p.H + item_head(t)) * p.Sq_pad + item_row0(t);
 #pragma unroll
       for (int c = 0; c < C::kDQChunks; ++c, ++n) {
         const uint32_t buf = sbase + C::kDQOff + uint32_t(n & 1) * C::kDQBufBytes;
@@ -515,19 +523,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_prefetch_desc(&tmV);
       mbar_arrive_expect_tx(bar(C::kBarKV), 2 * C::kTileBytes);
       for (int x = 0; x < C::kBoxes; ++x) {
-        tma_load_4d(k_addr + x * C::kBoxBytes, &tmK, bar(C::kBarKV), x * 64, h, n0, b);
-        tma_load_4d(v_addr + x * C::kBoxBytes, &tmV, bar(C::kBarKV), x * 64, h, n0, b);
+        tma_load_4d(k_addr + x * C::kBoxBytes, &tmK, bar(C::kBarKV), x * 64, hk, n0, b);
+        tma_load_4d(v_addr + x * C::kBoxBytes, &tmV, bar(C::kBarKV), x * 64, hk, n0, b);
       }
       for (int t = 0; t < nq; ++t) {
         const int s = t % kQStages;
         const int u = t / kQStages;
         if (u > 0 && !bw.wait(bar(C::kBarQEmpty + s), (u - 1) & 1, 20)) break;
-        const int i0 = (qlo + t) * BM;
+        const int i0 = item_row0(t);
+        const int h = item_head(t);
         const uint32_t fb = bar(C::kBarQFull + s);
         mbar_arrive_expect_tx(fb, C::kTileBytes + 2 * BM * 4);
         for (int x = 0; x < C::kBoxes; ++x)
           tma_load_4d(q_addr(s) + x * C::kBoxBytes, &tmQ, fb, x * 64, h, i0, b);
-        const size_t roff = size_t(bh) * p.Sq_pad + i0;
+        const size_t roff = size_t(b * p.H + h) * p.Sq_pad + i0;
         bulk_load(sbase + C::kLseOff + s * BM * 4, p.nlse2 + roff, BM * 4, fb);
         bulk_load(sbase + C::kDeltaOff + s * BM * 4, p.ndelta + roff, BM * 4, fb);
         if (s == 0) ++q_loads0; else ++q_loads1;
@@ -539,10 +548,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_prefetch_desc(&tmDO);
       for (int t = 0; t < nq; ++t) {
         if (t > 0 && !bw.wait(bar(C::kBarDOEmpty), (t - 1) & 1, 32)) break;
-        const int i0 = (qlo + t) * BM;
+        const int i0 = item_row0(t);
         mbar_arrive_expect_tx(bar(C::kBarDOFull), C::kTileBytes);
         for (int x = 0; x < C::kBoxes; ++x)
-          tma_load_4d(do_addr + x * C::kBoxBytes, &tmDO, bar(C::kBarDOFull), x * 64, h, i0, b);
+          tma_load_4d(do_addr + x * C::kBoxBytes, &tmDO, bar(C::kBarDOFull), x * 64, item_head(t),
+                      i0, b);
         do_loads++;
       }
     }

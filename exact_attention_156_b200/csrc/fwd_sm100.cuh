@@ -81,6 +81,7 @@ struct Params {
   __nv_bfloat16* o;
   float* lse;
   int B, H, Sq, Sk;
+  int Hk;            // key/value heads (H a multiple of Hk; query head h reads h / (H / Hk))
   float scale_log2;  // scale * log2(e)
   int causal, win_left, win_right;
   int num_mblocks;   // ceil(Sq / (NQ * BM))
@@ -124,6 +125,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int mb = p.causal ? (p.num_mblocks - 1 - int(blockIdx.x)) : int(blockIdx.x);
   const int h = blockIdx.y;
+  const int hk = h / (p.H / p.Hk);  // the key/value head this query head reads
   const int b = blockIdx.z;
   const MaskGeom g = MaskGeom::make(p.Sq, p.Sk, p.causal, p.win_left, p.win_right);
 
@@ -392,7 +394,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const void* map = (L & 1) ? static_cast<const void*>(&tmV) : static_cast<const void*>(&tmK);
         mbar_arrive_expect_tx(bar(C::kBarFull + s), C::kTileBytes);
         for (int x = 0; x < C::kBoxes; ++x)
-          tma_load_4d(kv_addr(s) + x * C::kBoxBytes, map, bar(C::kBarFull + s), x * 64, h, j * BN,
+          tma_load_4d(kv_addr(s) + x * C::kBoxBytes, map, bar(C::kBarFull + s), x * 64, hk, j * BN,
                       b);
         load_count[s]++;
       }

@@ -127,7 +127,7 @@ ATTN_API attn_status attn_bwd(const void* q, const void* k, const void* v, const
  * attn_bwd_main - for every 128-key tile: recomputes P from Q, K and the
  *   workspace LSE, accumulates dV = P^T dO and dK = scale dS^T Q in tensor
  *   memory and writes them (bf16), and adds dS K into the workspace dQ
- *   accumulator with float32 atomic reductions.
+ *   accumulator with float32 bulk reduce-adds.
  * attn_bwd_dq_finalize - dq = bf16(scale * accumulator).
  */
 ATTN_API attn_status attn_bwd_preprocess(const void* o, const void* dout, const float* lse,
@@ -139,6 +139,36 @@ ATTN_API attn_status attn_bwd_main(const void* q, const void* k, const void* v, 
                                    void* workspace, size_t workspace_bytes, void* stream);
 ATTN_API attn_status attn_bwd_dq_finalize(void* dq, int B, int Sq, int H, int D, float scale,
                                           void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Grouped K/V heads (GQA; MQA when Hk == 1).  The pages' Transformers snippet
+ * (FlashAttention-2 overview, lshu.cn, section 3.3) shapes Q with num_heads and
+ * K, V with num_kv_heads for the same call.  K and V (and dK, dV) have Hk heads,
+ * Q, O, dO, dQ and lse have H heads, H a multiple of Hk; query head h attends
+ * with key/value head h / (H / Hk) (consecutive query heads share one K/V head).
+ * dK and dV of a shared head are the sums over its query heads (accumulated in
+ * the kernel, no atomics).  The workspace is sized by H, as for attn_bwd.
+ *
+ *   k, v [B, Sk, Hk, D] bf16 (in)     dk, dv [B, Sk, Hk, D] bf16 (out)
+ *   every other argument as in attn_fwd / attn_bwd / attn_bwd_main.
+ * Errors: as the entry points they extend; ATTN_ERR_SHAPE also if Hk < 1,
+ * Hk > H or H is not a multiple of Hk.  With Hk == H they equal attn_fwd,
+ * attn_bwd and attn_bwd_main.
+ */
+ATTN_API attn_status attn_fwd_gqa(const void* q, const void* k, const void* v, void* o,
+                                  float* lse, int B, int Sq, int Sk, int H, int Hk, int D,
+                                  float scale, int causal, int win_left, int win_right,
+                                  void* stream);
+ATTN_API attn_status attn_bwd_gqa(const void* q, const void* k, const void* v, const void* o,
+                                  const void* dout, const float* lse, void* dq, void* dk,
+                                  void* dv, int B, int Sq, int Sk, int H, int Hk, int D,
+                                  float scale, int causal, int win_left, int win_right,
+                                  void* workspace, size_t workspace_bytes, void* stream);
+ATTN_API attn_status attn_bwd_main_gqa(const void* q, const void* k, const void* v,
+                                       const void* dout, void* dk, void* dv, int B, int Sq,
+                                       int Sk, int H, int Hk, int D, float scale, int causal,
+                                       int win_left, int win_right, void* workspace,
+                                       size_t workspace_bytes, void* stream);
 
 /*
  * attn_bwd_noalloc - attn_bwd for callers that cannot allocate device memory.

@@ -10,7 +10,8 @@ section 4.4).  Some workloads scale the draws by 0.5.
 Recipe (fixed here, the pages only say "random"):
   * generator: numpy ``Generator(PCG64(seed))``;
   * draw order: Q, K, V, dO, each ``standard_normal`` in float32 of shape
-    (B, S, H, D), multiplied by the workload's input scale;
+    (B, S, H, D) (K and V with Hk heads when the key/value heads are
+    grouped), multiplied by the workload's input scale;
   * round every value to bfloat16 with round-to-nearest-even;
   * the CUDA path receives the bf16 bit patterns; the oracle receives the
     same values widened to float64.
@@ -107,19 +108,21 @@ def bf16_bits_to_f32(b: np.ndarray) -> np.ndarray:
 
 
 def make_inputs(B: int, Sq: int, Sk: int, H: int, D: int, seed: int,
-                input_scale: float = 1.0, with_dout: bool = False):
+                input_scale: float = 1.0, with_dout: bool = False, Hk: Optional[int] = None):
     """Draw Q, K, V (and dO) for one workload.
 
     Returns a dict of bf16 bit arrays (uint16) with keys 'q', 'k', 'v' and,
-    if requested, 'do'; every array has shape (B, S, H, D).
+    if requested, 'do'; Q and dO have shape (B, Sq, H, D), K and V
+    (B, Sk, Hk, D) with Hk = H unless given (grouped K/V heads).
     """
     rng = np.random.Generator(np.random.PCG64(seed))
     out = {}
-    shapes = [("q", Sq), ("k", Sk), ("v", Sk)]
+    Hk = H if Hk is None else Hk
+    shapes = [("q", Sq, H), ("k", Sk, Hk), ("v", Sk, Hk)]
     if with_dout:
-        shapes.append(("do", Sq))
-    for name, S in shapes:
-        x = rng.standard_normal((B, S, H, D), dtype=np.float32)
+        shapes.append(("do", Sq, H))
+    for name, S, heads in shapes:
+        x = rng.standard_normal((B, S, heads, D), dtype=np.float32)
         if input_scale != 1.0:
             x *= np.float32(input_scale)
         out[name] = f32_to_bf16_bits(x)

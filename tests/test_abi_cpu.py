@@ -103,3 +103,36 @@ def test_binding_refuses_cpu_tensors():
     q = torch.zeros(1, 128, 2, 64, dtype=torch.bfloat16)
     with pytest.raises(ValueError, match="CUDA"):
         attn_fwd(q, q, q)
+
+
+def test_grouped_head_counts_are_validated():
+    from exact_attention_156_b200 import lib
+
+    def fwd(H, Hk, D=128):
+        return lib.attn_fwd_gqa(0x1000, 0x2000, 0x3000, 0x4000, 0x5000, 1, 128, 128, H, Hk, D,
+                                0.125, 1, -1, -1, None)
+    assert fwd(8, 0) == SHAPE
+    assert fwd(8, 16) == SHAPE
+    assert fwd(8, 3) == SHAPE
+    assert fwd(6, 4) == SHAPE
+    assert fwd(8, 2, D=96) == HEADDIM
+    assert fwd(8, 2) in (ARCH, DEVICE)       # well-formed: stops at the device checks
+    assert fwd(8, 1) in (ARCH, DEVICE)
+    p = [0x1000 * (i + 1) for i in range(9)]
+    ws = lib.attn_bwd_workspace_size(1, 128, 8, 128)
+    assert lib.attn_bwd_gqa(*p, 1, 128, 128, 8, 3, 128, 0.1, 1, -1, -1, 0x100000, ws, None) == SHAPE
+    assert lib.attn_bwd_main_gqa(*p[:6], 1, 128, 128, 8, 0, 128, 0.1, 1, -1, -1, 0x100000, ws,
+                                 None) == SHAPE
+    assert lib.attn_bwd_gqa(*p, 1, 128, 128, 8, 2, 128, 0.1, 1, -1, -1, None, ws, None) == 10
+
+
+def test_binding_checks_key_value_heads():
+    from types import SimpleNamespace
+
+    from exact_attention_156_b200._binding import _kv_heads
+    t = lambda *shape: SimpleNamespace(shape=shape)
+    assert _kv_heads(t(1, 8, 8, 64), t(1, 8, 8, 64), t(1, 8, 8, 64)) == 8
+    assert _kv_heads(t(1, 8, 8, 64), t(1, 8, 2, 64), t(1, 8, 2, 64)) == 2
+    for k, v in ((t(1, 8, 3, 64), t(1, 8, 3, 64)), (t(1, 8, 2, 64), t(1, 8, 4, 64))):
+        with pytest.raises(ValueError):
+            _kv_heads(t(1, 8, 8, 64), k, v)
