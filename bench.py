@@ -131,10 +131,12 @@ def sources_sha(files) -> str:
     return h.hexdigest()[:12]
 
 
-def traffic_key(kernel: str, w) -> str:
+def traffic_key(kernel: str, w, fmt: str = "bf16") -> str:
     """Name of a kernel's line in profiles/traffic_per_launch.txt: the kernel for
-    the headline workload, kernel@workload for the others."""
-    return kernel if w is WORKLOAD else f"{kernel}@{w['name']}"
+    the headline workload in bf16, kernel@workload[/f16] for the others."""
+    if w is WORKLOAD and fmt == "bf16":
+        return kernel
+    return f"{kernel}@{w['name']}" + ("/f16" if fmt == "f16" else "")
 
 
 def committed_traffic(kernel: str, sha: str):
@@ -316,8 +318,9 @@ def run_gpu(args):
     causal = bool(w["causal"])
     win = (w["win_left"], w["win_right"])
     bits = make_inputs(B, Sq, Sk, H, D, w["seed"] + rank, w["input_scale"], with_dout=True,
-                       Hk=w["Hk"])
-    host = {n: torch.from_numpy(bits[n].view("int16")).view(torch.bfloat16).pin_memory()
+                       Hk=w["Hk"], fmt=args.dtype)
+    tdtype = torch.float16 if args.dtype == "f16" else torch.bfloat16
+    host = {n: torch.from_numpy(bits[n].view("int16")).view(tdtype).pin_memory()
             for n in ("q", "k", "v", "do")}
     dev = {n: t.to(device) for n, t in host.items()}
     q, k, v, do = dev["q"], dev["k"], dev["v"], dev["do"]
@@ -413,19 +416,19 @@ def run_gpu(args):
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "scaling": "weak", "vs_baseline": None, "dtype": args.dtype, "data": "synthetic",
         "config": config_dict(w),
         "roofline": {"bound": "tensor", "kernel": "attn_bwd_main_kernel<128>",
                      "achieved": bwd_main_tflops, "peak": peak, "unit": "TFLOP/s",
                      "frac": bwd_main_tflops / peak,
                      "peak_source": f"{peaks.get('source')} bf16_tflops (burst)",
-                     "traffic": committed_traffic(traffic_key("attn_bwd_main_kernel", w),
+                     "traffic": committed_traffic(traffic_key("attn_bwd_main_kernel", w, args.dtype),
                                                   sources_sha(BWD_KERNEL_SOURCES))},
         "kernels": kernels,
         "fwd_roofline": {"bound": "tensor", "kernel": "attn_fwd_kernel<128>",
                          "achieved": fwd_tflops, "peak": peak, "unit": "TFLOP/s",
                          "frac": fwd_tflops / peak,
-                         "traffic": committed_traffic(traffic_key("attn_fwd_kernel", w),
+                         "traffic": committed_traffic(traffic_key("attn_fwd_kernel", w, args.dtype),
                                                       sources_sha(FWD_KERNEL_SOURCES))},
         "e2e": e2e,
         "gpu_launches": launches,
@@ -447,6 +450,8 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--dtype", choices=["bf16", "f16"], default="bf16",
+                    help="element format of the 16-bit tensors (default bf16)")
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="fwdbwd",
                     help="fwdbwd: the headline fwd+bwd workload (default); gqa: the same sizes "
                          "with 8 K/V heads for 32 query heads")

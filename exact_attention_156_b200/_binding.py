@@ -19,8 +19,9 @@ ATTN_STATUS = {
     0: "ATTN_OK", 1: "ATTN_ERR_NULLPTR", 2: "ATTN_ERR_SHAPE", 3: "ATTN_ERR_HEADDIM",
     4: "ATTN_ERR_ALIGN", 5: "ATTN_ERR_WINDOW", 6: "ATTN_ERR_ARCH", 7: "ATTN_ERR_DEVICE",
     8: "ATTN_ERR_LAUNCH", 9: "ATTN_ERR_TIMEOUT", 10: "ATTN_ERR_WORKSPACE",
-    11: "ATTN_ERR_SCRATCH",
+    11: "ATTN_ERR_SCRATCH", 12: "ATTN_ERR_DTYPE",
 }
+ATTN_DTYPE_BF16, ATTN_DTYPE_F16 = 0, 1
 
 
 class AttnError(RuntimeError):
@@ -48,14 +49,18 @@ def _load() -> ctypes.CDLL:
     lib.attn_bwd_main.restype = i
     lib.attn_bwd_dq_finalize.argtypes = [vp, i, i, i, i, f, vp, sz, vp]
     lib.attn_bwd_dq_finalize.restype = i
-    lib.attn_fwd_gqa.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, i, i, vp]
-    lib.attn_fwd_gqa.restype = i
-    lib.attn_bwd_gqa.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, i,
-                                 i, vp, sz, vp]
-    lib.attn_bwd_gqa.restype = i
-    lib.attn_bwd_main_gqa.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, i, i, vp,
-                                      sz, vp]
-    lib.attn_bwd_main_gqa.restype = i
+    lib.attn_fwd_ex.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, i, f, i, i, i, vp]
+    lib.attn_fwd_ex.restype = i
+    lib.attn_bwd_ex.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, f, i, i,
+                                i, vp, sz, vp]
+    lib.attn_bwd_ex.restype = i
+    lib.attn_bwd_preprocess_ex.argtypes = [vp, vp, vp, i, i, i, i, i, vp, sz, vp]
+    lib.attn_bwd_preprocess_ex.restype = i
+    lib.attn_bwd_main_ex.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, f, i, i, i, vp,
+                                     sz, vp]
+    lib.attn_bwd_main_ex.restype = i
+    lib.attn_bwd_dq_finalize_ex.argtypes = [vp, i, i, i, i, i, f, vp, sz, vp]
+    lib.attn_bwd_dq_finalize_ex.restype = i
     lib.attn_bwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, i,
                                      i, vp]
     lib.attn_bwd_noalloc.restype = i
@@ -98,6 +103,17 @@ def _check(t, name, dtype, ndim):
         raise ValueError(f"{name} must be contiguous (batch, seqlen, nheads, head_dim)")
 
 
+def _dtype_code(t) -> int:
+    """attn_dtype of a bf16 or f16 tensor (the format every 16-bit tensor of a call shares)."""
+    import torch
+    dtype = getattr(t, "dtype", None)
+    if dtype == torch.bfloat16:
+        return ATTN_DTYPE_BF16
+    if dtype == torch.float16:
+        return ATTN_DTYPE_F16
+    raise TypeError(f"tensors must be torch.bfloat16 or torch.float16, got {dtype}")
+
+
 def _kv_heads(q, k, v):
     """K/V head count; fewer than q's heads selects grouped K/V heads (GQA/MQA)."""
     H, Hk = q.shape[2], k.shape[2]
@@ -119,7 +135,8 @@ def _window(causal, window_size):
 def attn_fwd(q, k, v, softmax_scale: Optional[float] = None, causal: bool = False,
              window_size: Optional[Tuple[int, int]] = None, out=None, lse=None,
              stream=None):
-    """O, LSE = exact attention of q (B,Sq,H,D), k, v (B,Sk,Hk,D), all bf16 CUDA.
+    """O, LSE = exact attention of q (B,Sq,H,D), k, v (B,Sk,Hk,D), all bf16 (or all
+    float16) CUDA tensors.
 
     Hk = H is ordinary multi-head attention; Hk < H (a divisor of H) shares each
     K/V head among H/Hk consecutive query heads (GQA; MQA when Hk = 1).
@@ -127,24 +144,25 @@ def attn_fwd(q, k, v, softmax_scale: Optional[float] = None, causal: bool = Fals
     -1 for an unbounded side.  Returns (o bf16 (B,Sq,H,D), lse fp32 (B,H,Sq)).
     """
     import torch
+    dt = _dtype_code(q)
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
-        _check(t, n, torch.bfloat16, 4)
+        _check(t, n, q.dtype, 4)
     B, Sq, H, D = q.shape
     Sk = k.shape[1]
     if out is None:
         out = torch.empty_like(q)
     if lse is None:
         lse = torch.empty((B, H, Sq), dtype=torch.float32, device=q.device)
-    _check(out, "out", torch.bfloat16, 4)
+    _check(out, "out", q.dtype, 4)
     _check(lse, "lse", torch.float32, 3)
     c, wl, wr = _window(causal, window_size)
     Hk = _kv_heads(q, k, v)
     args = (q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(), B, Sq, Sk)
-    tail = (D, _scale(softmax_scale, D), c, wl, wr, _stream_handle(stream, q.device))
-    if Hk == H:
-        st, name = lib.attn_fwd(*args, H, *tail), "attn_fwd"
+    tail = (_scale(softmax_scale, D), c, wl, wr, _stream_handle(stream, q.device))
+    if Hk == H and dt == ATTN_DTYPE_BF16:
+        st, name = lib.attn_fwd(*args, H, D, *tail), "attn_fwd"
     else:
-        st, name = lib.attn_fwd_gqa(*args, H, Hk, *tail), "attn_fwd_gqa"
+        st, name = lib.attn_fwd_ex(*args, H, Hk, D, dt, *tail), "attn_fwd_ex"
     if st != 0:
         raise AttnError(st, name)
     return out, lse
@@ -163,8 +181,9 @@ def attn_bwd(q, k, v, out, dout, lse, softmax_scale: Optional[float] = None,
     bytes) is allocated by torch when not given.  Returns (dq, dk, dv) bf16.
     """
     import torch
+    dt = _dtype_code(q)
     for t, n in ((q, "q"), (k, "k"), (v, "v"), (out, "out"), (dout, "dout")):
-        _check(t, n, torch.bfloat16, 4)
+        _check(t, n, q.dtype, 4)
     _check(lse, "lse", torch.float32, 3)
     B, Sq, H, D = q.shape
     Sk = k.shape[1]
@@ -178,12 +197,12 @@ def attn_bwd(q, k, v, out, dout, lse, softmax_scale: Optional[float] = None,
     Hk = _kv_heads(q, k, v)
     args = (q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), dout.data_ptr(),
             lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, Sq, Sk)
-    tail = (D, _scale(softmax_scale, D), c, wl, wr, workspace.data_ptr(),
+    tail = (_scale(softmax_scale, D), c, wl, wr, workspace.data_ptr(),
             workspace.numel() * workspace.element_size(), _stream_handle(stream, q.device))
-    if Hk == H:
-        st, name = lib.attn_bwd(*args, H, *tail), "attn_bwd"
+    if Hk == H and dt == ATTN_DTYPE_BF16:
+        st, name = lib.attn_bwd(*args, H, D, *tail), "attn_bwd"
     else:
-        st, name = lib.attn_bwd_gqa(*args, H, Hk, *tail), "attn_bwd_gqa"
+        st, name = lib.attn_bwd_ex(*args, H, Hk, D, dt, *tail), "attn_bwd_ex"
     if st != 0:
         raise AttnError(st, name)
     return dq, dk, dv
@@ -200,33 +219,44 @@ def attn_bwd_stages(q, k, v, out, dout, lse, dq, dk, dv, workspace,
     """
     B, Sq, H, D = q.shape
     Sk = k.shape[1]
+    dt = _dtype_code(q)
     c, wl, wr = _window(causal, window_size)
     sc = _scale(softmax_scale, D)
     hs = _stream_handle(stream, q.device)
     wp, wb = workspace.data_ptr(), workspace.numel() * workspace.element_size()
+    Hk = _kv_heads(q, k, v)
+    plain = Hk == H and dt == ATTN_DTYPE_BF16
     if between:
         between(0)
-    st = lib.attn_bwd_preprocess(out.data_ptr(), dout.data_ptr(), lse.data_ptr(), B, Sq, H, D,
-                                 wp, wb, hs)
+    if plain:
+        st, name = lib.attn_bwd_preprocess(out.data_ptr(), dout.data_ptr(), lse.data_ptr(), B, Sq,
+                                           H, D, wp, wb, hs), "attn_bwd_preprocess"
+    else:
+        st, name = lib.attn_bwd_preprocess_ex(out.data_ptr(), dout.data_ptr(), lse.data_ptr(), B,
+                                              Sq, H, D, dt, wp, wb, hs), "attn_bwd_preprocess_ex"
     if st != 0:
-        raise AttnError(st, "attn_bwd_preprocess")
+        raise AttnError(st, name)
     if between:
         between(1)
-    Hk = _kv_heads(q, k, v)
     args = (q.data_ptr(), k.data_ptr(), v.data_ptr(), dout.data_ptr(), dk.data_ptr(),
             dv.data_ptr(), B, Sq, Sk)
-    if Hk == H:
+    if plain:
         st, name = lib.attn_bwd_main(*args, H, D, sc, c, wl, wr, wp, wb, hs), "attn_bwd_main"
     else:
-        st, name = (lib.attn_bwd_main_gqa(*args, H, Hk, D, sc, c, wl, wr, wp, wb, hs),
-                    "attn_bwd_main_gqa")
+        st, name = (lib.attn_bwd_main_ex(*args, H, Hk, D, dt, sc, c, wl, wr, wp, wb, hs),
+                    "attn_bwd_main_ex")
     if st != 0:
         raise AttnError(st, name)
     if between:
         between(2)
-    st = lib.attn_bwd_dq_finalize(dq.data_ptr(), B, Sq, H, D, sc, wp, wb, hs)
+    if plain:
+        st, name = lib.attn_bwd_dq_finalize(dq.data_ptr(), B, Sq, H, D, sc, wp, wb, hs), \
+            "attn_bwd_dq_finalize"
+    else:
+        st, name = lib.attn_bwd_dq_finalize_ex(dq.data_ptr(), B, Sq, H, D, dt, sc, wp, wb, hs), \
+            "attn_bwd_dq_finalize_ex"
     if st != 0:
-        raise AttnError(st, "attn_bwd_dq_finalize")
+        raise AttnError(st, name)
     if between:
         between(3)
     return dq, dk, dv

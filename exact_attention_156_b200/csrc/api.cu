@@ -10,6 +10,7 @@
 #include <mutex>
 #include <stdint.h>
 #include <string.h>
+#include <type_traits>
 
 #include "../../include/attn.h"
 #include "bwd_sm100.cuh"
@@ -69,19 +70,23 @@ attn_status device_state(DeviceState** out) {
     if (s.arch_ok) {
       if (cudaGetSymbolAddress(reinterpret_cast<void**>(&s.err), g_attn_err) != cudaSuccess)
         return ATTN_ERR_LAUNCH;
-      if (set_smem(fwd::attn_fwd_kernel<64>, fwd::Cfg<64>::kSmemBytes) != cudaSuccess ||
-          set_smem(fwd::attn_fwd_kernel<128>, fwd::Cfg<128>::kSmemBytes) != cudaSuccess ||
-          set_smem(bwd::attn_bwd_main_kernel<64>, bwd::Cfg<64>::kSmemBytes) != cudaSuccess ||
-          set_smem(bwd::attn_bwd_main_kernel<128>, bwd::Cfg<128>::kSmemBytes) != cudaSuccess)
-        return ATTN_ERR_LAUNCH;
       // The warp-specialised kernels hand registers between warpgroups with
       // setmaxnreg; the split is sized for exactly kLaunchRegs per thread at
       // launch.  Refuse to launch a build whose allocation differs.
-      if (regs_of(fwd::attn_fwd_kernel<64>) != fwd::kLaunchRegs ||
-          regs_of(fwd::attn_fwd_kernel<128>) != fwd::kLaunchRegs ||
-          regs_of(bwd::attn_bwd_main_kernel<64>) != bwd::kLaunchRegs ||
-          regs_of(bwd::attn_bwd_main_kernel<128>) != bwd::kLaunchRegs)
-        return ATTN_ERR_LAUNCH;
+      bool ok = true;
+      auto prepare = [&](auto d, auto e) {
+        constexpr int D = decltype(d)::value;
+        using E = decltype(e);
+        ok = ok && set_smem(fwd::attn_fwd_kernel<D, E>, fwd::Cfg<D>::kSmemBytes) == cudaSuccess &&
+             set_smem(bwd::attn_bwd_main_kernel<D, E>, bwd::Cfg<D>::kSmemBytes) == cudaSuccess &&
+             regs_of(fwd::attn_fwd_kernel<D, E>) == fwd::kLaunchRegs &&
+             regs_of(bwd::attn_bwd_main_kernel<D, E>) == bwd::kLaunchRegs;
+      };
+      prepare(std::integral_constant<int, 64>{}, ElemBF16{});
+      prepare(std::integral_constant<int, 128>{}, ElemBF16{});
+      prepare(std::integral_constant<int, 64>{}, ElemF16{});
+      prepare(std::integral_constant<int, 128>{}, ElemF16{});
+      if (!ok) return ATTN_ERR_LAUNCH;
       if (g_encode == nullptr) {
         void* fn = nullptr;
         cudaDriverEntryPointQueryResult q;
@@ -129,15 +134,24 @@ attn_status check_common(int B, int Sq, int Sk, int H, int D, float scale, int w
   return ATTN_OK;
 }
 
-// 4-D bf16 map over a (B, S, H, D) tensor, box = 64 x 1 x 128 x 1, 128-byte swizzle.
-attn_status make_map(CUtensorMap* map, const void* base, int B, int S, int H, int D) {
+// TMA element type of a kernel element format.
+template <class E>
+constexpr CUtensorMapDataType tmap_type() {
+  return std::is_same<E, ElemF16>::value ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
+                                          : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+}
+
+// 4-D map over a (B, S, H, D) tensor of 16-bit elements, box = 64 x 1 x 128 x 1,
+// 128-byte swizzle.
+attn_status make_map(CUtensorMap* map, const void* base, int B, int S, int H, int D,
+                     CUtensorMapDataType dtype) {
   const cuuint64_t dims[4] = {cuuint64_t(D), cuuint64_t(H), cuuint64_t(S), cuuint64_t(B)};
   const cuuint64_t strides[3] = {cuuint64_t(D) * 2, cuuint64_t(H) * D * 2,
                                  cuuint64_t(S) * H * D * 2};
   const cuuint32_t box[4] = {64, 1, 128, 1};
   const cuuint32_t estr[4] = {1, 1, 1, 1};
   const CUresult r =
-      g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides,
+      g_encode(map, dtype, 4, const_cast<void*>(base), dims, strides,
                box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? ATTN_OK : ATTN_ERR_LAUNCH;
@@ -164,16 +178,17 @@ size_t workspace_bytes(int B, int Sq, int H, int D) {
   return rows * D * 4 + rows * 4 * 2;
 }
 
-template <int D>
+template <int D, class E>
 attn_status launch_fwd(const DeviceState& st, const void* q, const void* k, const void* v, void* o,
                        float* lse, int B, int Sq, int Sk, int H, int Hk, float scale, int causal,
                        int win_left, int win_right, cudaStream_t stream) {
+  constexpr CUtensorMapDataType dt = tmap_type<E>();
   alignas(64) CUtensorMap mq, mk, mv;
-  if (make_map(&mq, q, B, Sq, H, D) != ATTN_OK || make_map(&mk, k, B, Sk, Hk, D) != ATTN_OK ||
-      make_map(&mv, v, B, Sk, Hk, D) != ATTN_OK)
+  if (make_map(&mq, q, B, Sq, H, D, dt) != ATTN_OK || make_map(&mk, k, B, Sk, Hk, D, dt) != ATTN_OK ||
+      make_map(&mv, v, B, Sk, Hk, D, dt) != ATTN_OK)
     return ATTN_ERR_LAUNCH;
   fwd::Params p;
-  p.o = static_cast<__nv_bfloat16*>(o);
+  p.o = static_cast<uint16_t*>(o);
   p.lse = lse;
   p.B = B;
   p.H = H;
@@ -188,7 +203,8 @@ attn_status launch_fwd(const DeviceState& st, const void* q, const void* k, cons
   p.err = st.err;
   p.timeout_ns = kTimeoutNs;
   dim3 grid(p.num_mblocks, H, B);
-  fwd::attn_fwd_kernel<D><<<grid, fwd::kThreads, fwd::Cfg<D>::kSmemBytes, stream>>>(mq, mk, mv, p);
+  fwd::attn_fwd_kernel<D, E><<<grid, fwd::kThreads, fwd::Cfg<D>::kSmemBytes, stream>>>(mq, mk, mv,
+                                                                                       p);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_LAUNCH;
 }
 
@@ -209,30 +225,32 @@ Workspace carve(void* workspace, int B, int Sq, int H, int D) {
   return w;
 }
 
-template <int D>
+template <int D, class E>
 attn_status launch_bwd_pre(const void* o, const void* dout, const float* lse, int B, int Sq,
                            int H, const Workspace& w, cudaStream_t stream) {
   const long long rows = (long long)B * H * w.Sq_pad;
   const unsigned blocks = unsigned((rows + 7) / 8);
-  bwd::attn_bwd_pre_kernel<D><<<blocks, 256, 0, stream>>>(
-      static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout), lse, w.nlse2,
+  bwd::attn_bwd_pre_kernel<D, E><<<blocks, 256, 0, stream>>>(
+      static_cast<const uint16_t*>(o), static_cast<const uint16_t*>(dout), lse, w.nlse2,
       w.ndelta, w.dq_acc, B, H, Sq, w.Sq_pad);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_LAUNCH;
 }
 
-template <int D>
+template <int D, class E>
 attn_status launch_bwd_main(const DeviceState& st, const void* q, const void* k, const void* v,
                             const void* dout, void* dk, void* dv, int B, int Sq, int Sk, int H,
                             int Hk, float scale, int causal, int win_left, int win_right,
                             const Workspace& w, cudaStream_t stream) {
+  constexpr CUtensorMapDataType dt = tmap_type<E>();
   alignas(64) CUtensorMap mq, mk, mv, mdo, mdq;
-  if (make_map(&mq, q, B, Sq, H, D) != ATTN_OK || make_map(&mk, k, B, Sk, Hk, D) != ATTN_OK ||
-      make_map(&mv, v, B, Sk, Hk, D) != ATTN_OK || make_map(&mdo, dout, B, Sq, H, D) != ATTN_OK ||
+  if (make_map(&mq, q, B, Sq, H, D, dt) != ATTN_OK || make_map(&mk, k, B, Sk, Hk, D, dt) != ATTN_OK ||
+      make_map(&mv, v, B, Sk, Hk, D, dt) != ATTN_OK ||
+      make_map(&mdo, dout, B, Sq, H, D, dt) != ATTN_OK ||
       make_dq_map(&mdq, w.dq_acc, (long long)B * H * w.Sq_pad, D) != ATTN_OK)
     return ATTN_ERR_LAUNCH;
   bwd::Params p;
-  p.dk = static_cast<__nv_bfloat16*>(dk);
-  p.dv = static_cast<__nv_bfloat16*>(dv);
+  p.dk = static_cast<uint16_t*>(dk);
+  p.dv = static_cast<uint16_t*>(dv);
   p.nlse2 = w.nlse2;
   p.ndelta = w.ndelta;
   p.dq_acc = w.dq_acc;
@@ -250,19 +268,52 @@ attn_status launch_bwd_main(const DeviceState& st, const void* q, const void* k,
   p.err = st.err;
   p.timeout_ns = kTimeoutNs;
   dim3 grid((Sk + bwd::BN - 1) / bwd::BN, Hk, B);
-  bwd::attn_bwd_main_kernel<D>
+  bwd::attn_bwd_main_kernel<D, E>
       <<<grid, bwd::kThreads, bwd::Cfg<D>::kSmemBytes, stream>>>(mq, mk, mv, mdo, mdq, p);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_LAUNCH;
 }
 
-template <int D>
+template <int D, class E>
 attn_status launch_bwd_dq(void* dq, int B, int Sq, int H, float scale, const Workspace& w,
                           cudaStream_t stream) {
   const long long total = (long long)B * Sq * H * (D / 8);
   const unsigned blocks = unsigned((total + 255) / 256);
-  bwd::attn_bwd_dq_kernel<D><<<blocks, 256, 0, stream>>>(
-      w.dq_acc, static_cast<__nv_bfloat16*>(dq), B, H, Sq, w.Sq_pad, scale);
+  bwd::attn_bwd_dq_kernel<D, E><<<blocks, 256, 0, stream>>>(
+      w.dq_acc, static_cast<uint16_t*>(dq), B, H, Sq, w.Sq_pad, scale);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_LAUNCH;
+}
+
+// Calls f(integral_constant<int, D>, element format) for the (head_dim, dtype)
+// of a call; both were validated before.
+template <class F>
+attn_status dispatch(int D, int dtype, F&& f) {
+  if (dtype == ATTN_DTYPE_F16)
+    return D == 64 ? f(std::integral_constant<int, 64>{}, ElemF16{})
+                   : f(std::integral_constant<int, 128>{}, ElemF16{});
+  return D == 64 ? f(std::integral_constant<int, 64>{}, ElemBF16{})
+                 : f(std::integral_constant<int, 128>{}, ElemBF16{});
+}
+
+attn_status check_dtype(int dtype) {
+  return (dtype == ATTN_DTYPE_BF16 || dtype == ATTN_DTYPE_F16) ? ATTN_OK : ATTN_ERR_DTYPE;
+}
+
+// The three backward stages on one stream through workspace `w`.
+attn_status run_backward(const DeviceState& st, const void* q, const void* k, const void* v,
+                         const void* o, const void* dout, const float* lse, void* dq, void* dk,
+                         void* dv, int B, int Sq, int Sk, int H, int Hk, int D, int dtype,
+                         float scale, int causal, int win_left, int win_right, const Workspace& w,
+                         cudaStream_t cs) {
+  return dispatch(D, dtype, [&](auto d, auto e) {
+    constexpr int DD = decltype(d)::value;
+    using E = decltype(e);
+    attn_status s = launch_bwd_pre<DD, E>(o, dout, lse, B, Sq, H, w, cs);
+    if (s == ATTN_OK)
+      s = launch_bwd_main<DD, E>(st, q, k, v, dout, dk, dv, B, Sq, Sk, H, Hk, scale, causal,
+                                 win_left, win_right, w, cs);
+    if (s == ATTN_OK) s = launch_bwd_dq<DD, E>(dq, B, Sq, H, scale, w, cs);
+    return s;
+  });
 }
 
 attn_status check_workspace(const void* workspace, size_t bytes, int B, int Sq, int H, int D) {
@@ -342,38 +393,37 @@ const char* attn_status_string(attn_status s) {
     case ATTN_ERR_SCRATCH:
       return "backward scratch for this problem exceeds the 64 MiB built into attn_bwd_noalloc "
              "(call attn_bwd with a workspace instead)";
+    case ATTN_ERR_DTYPE: return "dtype must be ATTN_DTYPE_BF16 (0) or ATTN_DTYPE_F16 (1)";
   }
   return "unknown status";
 }
 
-attn_status attn_fwd_gqa(const void* q, const void* k, const void* v, void* o, float* lse,
-                         int B, int Sq, int Sk, int H, int Hk, int D, float scale, int causal,
-                         int win_left, int win_right, void* stream) {
+attn_status attn_fwd_ex(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                        int Sq, int Sk, int H, int Hk, int D, int dtype, float scale, int causal,
+                        int win_left, int win_right, void* stream) {
   if (!q || !k || !v || !o || !lse) return ATTN_ERR_NULLPTR;
   attn_status s = check_common(B, Sq, Sk, H, D, scale, win_left, win_right, Hk);
   if (s != ATTN_OK) return s;
+  if ((s = check_dtype(dtype)) != ATTN_OK) return s;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) ||
       (reinterpret_cast<uintptr_t>(lse) & 3u))
     return ATTN_ERR_ALIGN;
   DeviceState* st = nullptr;
   s = device_state(&st);
   if (s != ATTN_OK) return s;
-  if (!on_current_device(q) || !on_current_device(k) || !on_current_device(v) ||
-      !on_current_device(o) || !on_current_device(lse))
-    return ATTN_ERR_DEVICE;
+  if (!all_on_device({q, k, v, o, lse})) return ATTN_ERR_DEVICE;
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
-  if (D == 64)
-    return launch_fwd<64>(*st, q, k, v, o, lse, B, Sq, Sk, H, Hk, scale, causal, win_left,
-                          win_right, cs);
-  return launch_fwd<128>(*st, q, k, v, o, lse, B, Sq, Sk, H, Hk, scale, causal, win_left,
-                         win_right, cs);
+  return dispatch(D, dtype, [&](auto d, auto e) {
+    return launch_fwd<decltype(d)::value, decltype(e)>(*st, q, k, v, o, lse, B, Sq, Sk, H, Hk,
+                                                       scale, causal, win_left, win_right, cs);
+  });
 }
 
 attn_status attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B,
                      int Sq, int Sk, int H, int D, float scale, int causal, int win_left,
                      int win_right, void* stream) {
-  return attn_fwd_gqa(q, k, v, o, lse, B, Sq, Sk, H, H, D, scale, causal, win_left, win_right,
-                      stream);
+  return attn_fwd_ex(q, k, v, o, lse, B, Sq, Sk, H, H, D, ATTN_DTYPE_BF16, scale, causal,
+                     win_left, win_right, stream);
 }
 
 size_t attn_bwd_workspace_size(int B, int Sq, int H, int D) {
@@ -381,14 +431,15 @@ size_t attn_bwd_workspace_size(int B, int Sq, int H, int D) {
   return workspace_bytes(B, Sq, H, D);
 }
 
-attn_status attn_bwd_gqa(const void* q, const void* k, const void* v, const void* o,
-                         const void* dout, const float* lse, void* dq, void* dk, void* dv, int B,
-                         int Sq, int Sk, int H, int Hk, int D, float scale, int causal,
-                         int win_left, int win_right, void* workspace, size_t workspace_size,
-                         void* stream) {
+attn_status attn_bwd_ex(const void* q, const void* k, const void* v, const void* o,
+                        const void* dout, const float* lse, void* dq, void* dk, void* dv, int B,
+                        int Sq, int Sk, int H, int Hk, int D, int dtype, float scale, int causal,
+                        int win_left, int win_right, void* workspace, size_t workspace_size,
+                        void* stream) {
   if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv) return ATTN_ERR_NULLPTR;
   attn_status s = check_common(B, Sq, Sk, H, D, scale, win_left, win_right, Hk);
   if (s != ATTN_OK) return s;
+  if ((s = check_dtype(dtype)) != ATTN_OK) return s;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) ||
       !aligned16(dq) || !aligned16(dk) || !aligned16(dv) ||
       (reinterpret_cast<uintptr_t>(lse) & 3u))
@@ -399,38 +450,26 @@ attn_status attn_bwd_gqa(const void* q, const void* k, const void* v, const void
   s = device_state(&st);
   if (s != ATTN_OK) return s;
   if (!all_on_device({q, k, v, o, dout, lse, dq, dk, dv, workspace})) return ATTN_ERR_DEVICE;
-  cudaStream_t cs = static_cast<cudaStream_t>(stream);
-  const Workspace w = carve(workspace, B, Sq, H, D);
-  if (D == 64) {
-    s = launch_bwd_pre<64>(o, dout, lse, B, Sq, H, w, cs);
-    if (s == ATTN_OK)
-      s = launch_bwd_main<64>(*st, q, k, v, dout, dk, dv, B, Sq, Sk, H, Hk, scale, causal,
-                              win_left, win_right, w, cs);
-    if (s == ATTN_OK) s = launch_bwd_dq<64>(dq, B, Sq, H, scale, w, cs);
-  } else {
-    s = launch_bwd_pre<128>(o, dout, lse, B, Sq, H, w, cs);
-    if (s == ATTN_OK)
-      s = launch_bwd_main<128>(*st, q, k, v, dout, dk, dv, B, Sq, Sk, H, Hk, scale, causal,
-                               win_left, win_right, w, cs);
-    if (s == ATTN_OK) s = launch_bwd_dq<128>(dq, B, Sq, H, scale, w, cs);
-  }
-  return s;
+  return run_backward(*st, q, k, v, o, dout, lse, dq, dk, dv, B, Sq, Sk, H, Hk, D, dtype, scale,
+                      causal, win_left, win_right, carve(workspace, B, Sq, H, D),
+                      static_cast<cudaStream_t>(stream));
 }
 
 attn_status attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
                      const float* lse, void* dq, void* dk, void* dv, int B, int Sq, int Sk, int H,
                      int D, float scale, int causal, int win_left, int win_right, void* workspace,
                      size_t workspace_size, void* stream) {
-  return attn_bwd_gqa(q, k, v, o, dout, lse, dq, dk, dv, B, Sq, Sk, H, H, D, scale, causal,
-                      win_left, win_right, workspace, workspace_size, stream);
+  return attn_bwd_ex(q, k, v, o, dout, lse, dq, dk, dv, B, Sq, Sk, H, H, D, ATTN_DTYPE_BF16,
+                     scale, causal, win_left, win_right, workspace, workspace_size, stream);
 }
 
-attn_status attn_bwd_preprocess(const void* o, const void* dout, const float* lse, int B, int Sq,
-                                int H, int D, void* workspace, size_t workspace_size,
-                                void* stream) {
+attn_status attn_bwd_preprocess_ex(const void* o, const void* dout, const float* lse, int B,
+                                   int Sq, int H, int D, int dtype, void* workspace,
+                                   size_t workspace_size, void* stream) {
   if (!o || !dout || !lse) return ATTN_ERR_NULLPTR;
   attn_status s = check_common(B, Sq, 1, H, D, 1.0f, -1, -1);
   if (s != ATTN_OK) return s;
+  if ((s = check_dtype(dtype)) != ATTN_OK) return s;
   if (!aligned16(o) || !aligned16(dout) || (reinterpret_cast<uintptr_t>(lse) & 3u))
     return ATTN_ERR_ALIGN;
   s = check_workspace(workspace, workspace_size, B, Sq, H, D);
@@ -441,17 +480,26 @@ attn_status attn_bwd_preprocess(const void* o, const void* dout, const float* ls
   if (!all_on_device({o, dout, lse, workspace})) return ATTN_ERR_DEVICE;
   const Workspace w = carve(workspace, B, Sq, H, D);
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
-  return D == 64 ? launch_bwd_pre<64>(o, dout, lse, B, Sq, H, w, cs)
-                 : launch_bwd_pre<128>(o, dout, lse, B, Sq, H, w, cs);
+  return dispatch(D, dtype, [&](auto d, auto e) {
+    return launch_bwd_pre<decltype(d)::value, decltype(e)>(o, dout, lse, B, Sq, H, w, cs);
+  });
 }
 
-attn_status attn_bwd_main_gqa(const void* q, const void* k, const void* v, const void* dout,
-                              void* dk, void* dv, int B, int Sq, int Sk, int H, int Hk, int D,
-                              float scale, int causal, int win_left, int win_right,
-                              void* workspace, size_t workspace_size, void* stream) {
+attn_status attn_bwd_preprocess(const void* o, const void* dout, const float* lse, int B, int Sq,
+                                int H, int D, void* workspace, size_t workspace_size,
+                                void* stream) {
+  return attn_bwd_preprocess_ex(o, dout, lse, B, Sq, H, D, ATTN_DTYPE_BF16, workspace,
+                                workspace_size, stream);
+}
+
+attn_status attn_bwd_main_ex(const void* q, const void* k, const void* v, const void* dout,
+                             void* dk, void* dv, int B, int Sq, int Sk, int H, int Hk, int D,
+                             int dtype, float scale, int causal, int win_left, int win_right,
+                             void* workspace, size_t workspace_size, void* stream) {
   if (!q || !k || !v || !dout || !dk || !dv) return ATTN_ERR_NULLPTR;
   attn_status s = check_common(B, Sq, Sk, H, D, scale, win_left, win_right, Hk);
   if (s != ATTN_OK) return s;
+  if ((s = check_dtype(dtype)) != ATTN_OK) return s;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dout) || !aligned16(dk) ||
       !aligned16(dv))
     return ATTN_ERR_ALIGN;
@@ -463,25 +511,28 @@ attn_status attn_bwd_main_gqa(const void* q, const void* k, const void* v, const
   if (!all_on_device({q, k, v, dout, dk, dv, workspace})) return ATTN_ERR_DEVICE;
   const Workspace w = carve(workspace, B, Sq, H, D);
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
-  return D == 64 ? launch_bwd_main<64>(*st, q, k, v, dout, dk, dv, B, Sq, Sk, H, Hk, scale,
-                                       causal, win_left, win_right, w, cs)
-                 : launch_bwd_main<128>(*st, q, k, v, dout, dk, dv, B, Sq, Sk, H, Hk, scale,
-                                        causal, win_left, win_right, w, cs);
+  return dispatch(D, dtype, [&](auto d, auto e) {
+    return launch_bwd_main<decltype(d)::value, decltype(e)>(*st, q, k, v, dout, dk, dv, B, Sq,
+                                                            Sk, H, Hk, scale, causal, win_left,
+                                                            win_right, w, cs);
+  });
 }
 
 attn_status attn_bwd_main(const void* q, const void* k, const void* v, const void* dout,
                           void* dk, void* dv, int B, int Sq, int Sk, int H, int D, float scale,
                           int causal, int win_left, int win_right, void* workspace,
                           size_t workspace_size, void* stream) {
-  return attn_bwd_main_gqa(q, k, v, dout, dk, dv, B, Sq, Sk, H, H, D, scale, causal, win_left,
-                           win_right, workspace, workspace_size, stream);
+  return attn_bwd_main_ex(q, k, v, dout, dk, dv, B, Sq, Sk, H, H, D, ATTN_DTYPE_BF16, scale,
+                          causal, win_left, win_right, workspace, workspace_size, stream);
 }
 
-attn_status attn_bwd_dq_finalize(void* dq, int B, int Sq, int H, int D, float scale,
-                                 void* workspace, size_t workspace_size, void* stream) {
+attn_status attn_bwd_dq_finalize_ex(void* dq, int B, int Sq, int H, int D, int dtype,
+                                    float scale, void* workspace, size_t workspace_size,
+                                    void* stream) {
   if (!dq) return ATTN_ERR_NULLPTR;
   attn_status s = check_common(B, Sq, 1, H, D, scale, -1, -1);
   if (s != ATTN_OK) return s;
+  if ((s = check_dtype(dtype)) != ATTN_OK) return s;
   if (!aligned16(dq)) return ATTN_ERR_ALIGN;
   s = check_workspace(workspace, workspace_size, B, Sq, H, D);
   if (s != ATTN_OK) return s;
@@ -491,8 +542,15 @@ attn_status attn_bwd_dq_finalize(void* dq, int B, int Sq, int H, int D, float sc
   if (!all_on_device({dq, workspace})) return ATTN_ERR_DEVICE;
   const Workspace w = carve(workspace, B, Sq, H, D);
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
-  return D == 64 ? launch_bwd_dq<64>(dq, B, Sq, H, scale, w, cs)
-                 : launch_bwd_dq<128>(dq, B, Sq, H, scale, w, cs);
+  return dispatch(D, dtype, [&](auto d, auto e) {
+    return launch_bwd_dq<decltype(d)::value, decltype(e)>(dq, B, Sq, H, scale, w, cs);
+  });
+}
+
+attn_status attn_bwd_dq_finalize(void* dq, int B, int Sq, int H, int D, float scale,
+                                 void* workspace, size_t workspace_size, void* stream) {
+  return attn_bwd_dq_finalize_ex(dq, B, Sq, H, D, ATTN_DTYPE_BF16, scale, workspace,
+                                 workspace_size, stream);
 }
 
 attn_status attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* o,
@@ -514,24 +572,11 @@ attn_status attn_bwd_noalloc(const void* q, const void* k, const void* v, const 
   void* scratch = nullptr;
   s = noalloc_scratch(&scratch);
   if (s != ATTN_OK) return s;
-  cudaStream_t cs = static_cast<cudaStream_t>(stream);
   // The preprocess kernel rewrites Delta and LSE rows and zeroes the dQ
   // accumulator, so nothing left in the scratch by an earlier call is read.
-  const Workspace w = carve(scratch, B, Sq, H, D);
-  if (D == 64) {
-    s = launch_bwd_pre<64>(o, dout, lse, B, Sq, H, w, cs);
-    if (s == ATTN_OK)
-      s = launch_bwd_main<64>(*st, q, k, v, dout, dk, dv, B, Sq, Sk, H, H, scale, causal,
-                              win_left, win_right, w, cs);
-    if (s == ATTN_OK) s = launch_bwd_dq<64>(dq, B, Sq, H, scale, w, cs);
-  } else {
-    s = launch_bwd_pre<128>(o, dout, lse, B, Sq, H, w, cs);
-    if (s == ATTN_OK)
-      s = launch_bwd_main<128>(*st, q, k, v, dout, dk, dv, B, Sq, Sk, H, H, scale, causal,
-                               win_left, win_right, w, cs);
-    if (s == ATTN_OK) s = launch_bwd_dq<128>(dq, B, Sq, H, scale, w, cs);
-  }
-  return s;
+  return run_backward(*st, q, k, v, o, dout, lse, dq, dk, dv, B, Sq, Sk, H, H, D,
+                      ATTN_DTYPE_BF16, scale, causal, win_left, win_right,
+                      carve(scratch, B, Sq, H, D), static_cast<cudaStream_t>(stream));
 }
 
 attn_status attn_get_last_device_error(void) {

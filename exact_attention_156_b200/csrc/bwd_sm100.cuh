@@ -28,7 +28,9 @@
 //     Q (with its row values) is double buffered, dO single buffered; the MMA
 //     order dV(t), S(t+1), dQ(t), dK(t), dP(t+1) lets the next tile's P run
 //     while the tensor core finishes this tile's gradients.
-//  3. bwd_dq_finalize: dQ = bf16(scale * accumulator).
+//  3. bwd_dq_finalize: dQ = scale * accumulator, rounded to the input format.
+// Q, K, V, dO, P, dS and the gradients are bf16 or f16 (template parameter E);
+// all accumulation is f32.
 // Tensor memory (512 columns): dK [0,D) dV [D,2D) S^T/P^T [2D,2D+128)
 // dP^T / dQ [2D+128, 2D+256).
 #pragma once
@@ -102,8 +104,8 @@ struct Cfg {
 };
 
 struct Params {
-  __nv_bfloat16* dk;
-  __nv_bfloat16* dv;
+  uint16_t* dk;  // 16-bit elements (bf16 or f16, as the kernel's element format)
+  uint16_t* dv;
   const float* nlse2;   // [B*H][Sq_pad] -LSE * log2(e); -inf for padding rows
   const float* ndelta;  // [B*H][Sq_pad] -Delta
   float* dq_acc;       // [B*H][Sq_pad][D]
@@ -119,9 +121,9 @@ struct Params {
 // ---------------------------------------------------------------------------
 // 1. preprocess: one warp per (b, h, row of the padded query axis)
 // ---------------------------------------------------------------------------
-template <int D>
+template <int D, class E>
 __global__ void __launch_bounds__(256) attn_bwd_pre_kernel(
-    const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* __restrict__ dout,
+    const uint16_t* __restrict__ o, const uint16_t* __restrict__ dout,
     const float* __restrict__ lse, float* __restrict__ nlse2, float* __restrict__ ndelta,
     float* __restrict__ dq_acc, int B, int H, int Sq, int Sq_pad) {
   const long long gw = (long long)blockIdx.x * 8 + threadIdx.x / 32;
@@ -135,26 +137,24 @@ __global__ void __launch_bounds__(256) attn_bwd_pre_kernel(
   float dot = 0.f;
   if (i < Sq) {
     const size_t base = ((size_t(b) * Sq + i) * H + h) * D;
-    constexpr int kPer = D / 32;  // bf16 elements per lane (2 or 4)
+    constexpr int kPer = D / 32;  // 16-bit elements per lane (2 or 4)
+    uint32_t ow[kPer / 2], dw[kPer / 2];
     if constexpr (kPer == 4) {
       const uint2 ov = *reinterpret_cast<const uint2*>(o + base + lane * 4);
       const uint2 dv = *reinterpret_cast<const uint2*>(dout + base + lane * 4);
-      const __nv_bfloat162* o2 = reinterpret_cast<const __nv_bfloat162*>(&ov);
-      const __nv_bfloat162* d2 = reinterpret_cast<const __nv_bfloat162*>(&dv);
-#pragma unroll
-      for (int t = 0; t < 2; ++t) {
-        const float2 a = __bfloat1622float2(o2[t]);
-        const float2 c = __bfloat1622float2(d2[t]);
-        dot = fmaf(a.x, c.x, dot);
-        dot = fmaf(a.y, c.y, dot);
-      }
+      ow[0] = ov.x; ow[1] = ov.y;
+      dw[0] = dv.x; dw[1] = dv.y;
     } else {
-      const __nv_bfloat162 ov = *reinterpret_cast<const __nv_bfloat162*>(o + base + lane * 2);
-      const __nv_bfloat162 dv = *reinterpret_cast<const __nv_bfloat162*>(dout + base + lane * 2);
-      const float2 a = __bfloat1622float2(ov);
-      const float2 c = __bfloat1622float2(dv);
-      dot = fmaf(a.x, c.x, dot);
-      dot = fmaf(a.y, c.y, dot);
+      ow[0] = *reinterpret_cast<const uint32_t*>(o + base + lane * 2);
+      dw[0] = *reinterpret_cast<const uint32_t*>(dout + base + lane * 2);
+    }
+#pragma unroll
+    for (int t = 0; t < kPer / 2; ++t) {
+      float a0, a1, c0, c1;
+      E::unpack2(ow[t], a0, a1);
+      E::unpack2(dw[t], c0, c1);
+      dot = fmaf(a0, c0, dot);
+      dot = fmaf(a1, c1, dot);
     }
   }
 #pragma unroll
@@ -174,11 +174,11 @@ __global__ void __launch_bounds__(256) attn_bwd_pre_kernel(
 }
 
 // ---------------------------------------------------------------------------
-// 3. dQ finalize: dq[b, i, h, :] = bf16(scale * acc[b, h, i, :]); 8 elements per thread
+// 3. dQ finalize: dq[b, i, h, :] = 16-bit(scale * acc[b, h, i, :]); 8 elements per thread
 // ---------------------------------------------------------------------------
-template <int D>
+template <int D, class E>
 __global__ void __launch_bounds__(256) attn_bwd_dq_kernel(const float* __restrict__ dq_acc,
-                                                          __nv_bfloat16* __restrict__ dq, int B,
+                                                          uint16_t* __restrict__ dq, int B,
                                                           int H, int Sq, int Sq_pad, float scale) {
   const long long t = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   constexpr int kVec = D / 8;
@@ -195,10 +195,10 @@ __global__ void __launch_bounds__(256) attn_bwd_dq_kernel(const float* __restric
   const float4 a = src[0];
   const float4 c = src[1];
   uint4 w;
-  w.x = pack_bf16x2(a.x * scale, a.y * scale);
-  w.y = pack_bf16x2(a.z * scale, a.w * scale);
-  w.z = pack_bf16x2(c.x * scale, c.y * scale);
-  w.w = pack_bf16x2(c.z * scale, c.w * scale);
+  w.x = E::pack2(a.x * scale, a.y * scale);
+  w.y = E::pack2(a.z * scale, a.w * scale);
+  w.z = E::pack2(c.x * scale, c.y * scale);
+  w.w = E::pack2(c.z * scale, c.w * scale);
   *reinterpret_cast<uint4*>(dq + ((size_t(b) * Sq + i) * H + h) * D + v * 8) = w;
 }
 
@@ -218,7 +218,8 @@ __device__ __forceinline__ void qtile_range(const MaskGeom& g, int n0, int n1, i
   qhi = z / BM + 1;
 }
 
-template <int D>
+// E: element format of Q, K, V, dO, P, dS and the gradients (ElemBF16 or ElemF16).
+template <int D, class E>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ,
                          const __grid_constant__ CUtensorMap tmK,
@@ -338,7 +339,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int i0 = item_row0(t);
       const float4* nl = reinterpret_cast<const float4*>(smem + C::kLseOff + s * BM * 4);
       const float4* nd = reinterpret_cast<const float4*>(smem + C::kDeltaOff + s * BM * 4);
-      // P = 2^(scale*log2e*S - LSE*log2e), kept as bf16 pairs (what dV uses) for dS too
+      // P = 2^(scale*log2e*S - LSE*log2e), kept as 16-bit pairs (what dV uses) for dS too
       if (!bw.wait_warp(bar(C::kBarS), t & 1, 27)) { ok = false; break; }
       tc_fence_after();
       uint32_t pw[BM / 2];
@@ -359,7 +360,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 f2_pack(l4.z, l4.w));
             float a0, a1, a2, a3;
             f2_unpack(x0, a0, a1);
-            pw[c / 2] = pack_bf16x2(ex2_approx(a0), ex2_approx(a1));
+            pw[c / 2] = E::pack2(ex2_approx(a0), ex2_approx(a1));
             if ((c & 7) == 4) {
               f2_unpack(f2_exp2_poly(x1), a2, a3);
             } else {
@@ -367,7 +368,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               a2 = ex2_approx(a2);
               a3 = ex2_approx(a3);
             }
-            pw[c / 2 + 1] = pack_bf16x2(a2, a3);
+            pw[c / 2 + 1] = E::pack2(a2, a3);
           }
         } else {
           const int c_lo = key_ok ? qmin_k - i0 : (1 << 30);
@@ -388,8 +389,8 @@ __global__ void __launch_bounds__(kThreads, 1)
               a[e] = ex2_approx(a[e]);
               if (c + e < c_lo || c + e > c_hi) a[e] = 0.f;
             }
-            pw[c / 2] = pack_bf16x2(a[0], a[1]);
-            pw[c / 2 + 1] = pack_bf16x2(a[2], a[3]);
+            pw[c / 2] = E::pack2(a[0], a[1]);
+            pw[c / 2 + 1] = E::pack2(a[2], a[3]);
           }
         }
       }
@@ -397,7 +398,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       mbar_arrive(bar(C::kBarP));
 
-      // dS = P * (dP - Delta) -> bf16, written swizzled for the dK and dQ products
+      // dS = P * (dP - Delta) -> 16-bit, written swizzled for the dK and dQ products
       if (!bw.wait_warp(bar(C::kBarDP), t & 1, 28)) { ok = false; break; }
       tc_fence_after();
       uint32_t rr[BM];
@@ -411,14 +412,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t w[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const uint32_t pp = pw[c / 2 + e];
-          const uint64_t p2 = f2_pack(__uint_as_float(pp << 16), __uint_as_float(pp & 0xffff0000u));
+          float pl, ph;
+          E::unpack2(pw[c / 2 + e], pl, ph);
+          const uint64_t p2 = f2_pack(pl, ph);
           const uint64_t gd = f2_add(
               f2_pack(__uint_as_float(rr[c + 2 * e]), __uint_as_float(rr[c + 2 * e + 1])),
               f2_pack(dl[2 * e], dl[2 * e + 1]));
           float a0, a1;
           f2_unpack(f2_mul(p2, gd), a0, a1);
-          w[e] = pack_bf16x2(a0, a1);
+          w[e] = E::pack2(a0, a1);
         }
         const uint32_t box = uint32_t(c / 64);
         const uint32_t chunk = uint32_t((c % 64) / 8);
@@ -428,7 +430,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       mbar_arrive(bar(C::kBarDS));
     }
-    // epilogue: dK = scale * acc, dV = acc (bf16), once the last dK product is done
+    // epilogue: dK = scale * acc, dV = acc (16-bit), once the last dK product is done
     if (ok && nq > 0) ok = bw.wait_warp(bar(C::kBarDSEmpty), (nq - 1) & 1, 30);
     if (ok) {
       tc_fence_after();
@@ -437,7 +439,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int which = 0; which < 2; ++which) {
         const uint32_t col = which == 0 ? C::kColDK : C::kColDV;
         const float mul = which == 0 ? p.scale : 1.0f;
-        __nv_bfloat16* outp = which == 0 ? p.dk : p.dv;
+        uint16_t* outp = which == 0 ? p.dk : p.dv;
 #pragma unroll 1
         for (int c0 = 0; c0 < D; c0 += 32) {
           uint32_t rr[32];
@@ -450,7 +452,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint32_t w[16];
 #pragma unroll
           for (int c = 0; c < 16; ++c)
-            w[c] = pack_bf16x2(__uint_as_float(rr[2 * c]) * mul, __uint_as_float(rr[2 * c + 1]) * mul);
+            w[c] = E::pack2(__uint_as_float(rr[2 * c]) * mul, __uint_as_float(rr[2 * c + 1]) * mul);
           if (key_ok) {
             uint8_t* dst = reinterpret_cast<uint8_t*>(outp + orow + c0);
 #pragma unroll
@@ -559,9 +561,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issue
     if (lane == 0 && nq > 0) {
-      constexpr uint32_t id_s = idesc_bf16_f32(BN, BM, false, false);   // S^T, dP^T
-      constexpr uint32_t id_dv = idesc_bf16_f32(BN, D, false, true);    // dV, dK
-      constexpr uint32_t id_dq = idesc_bf16_f32(BM, D, true, true);     // dQ
+      constexpr uint32_t id_s = idesc_f32acc(BN, BM, false, false, E::kFmt);  // S^T, dP^T
+      constexpr uint32_t id_dv = idesc_f32acc(BN, D, false, true, E::kFmt);   // dV, dK
+      constexpr uint32_t id_dq = idesc_f32acc(BM, D, true, true, E::kFmt);    // dQ
       auto issue_kmajor = [&](uint32_t d_col, uint32_t a_base, uint32_t b_base) {
         if constexpr (D == 128)
           mma_chain_kk8(tmem + d_col, sdesc_sw128(a_base, 16), sdesc_sw128(b_base, 16), id_s, 0u);

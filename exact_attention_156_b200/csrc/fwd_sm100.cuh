@@ -21,9 +21,10 @@
 //    are scaled by scale*log2(e) and exponentiated with ex2.  The running max
 //    is only raised when it grows by more than 2^8 (factor 256), so O is
 //    rescaled rarely; since O and l share the stale max, O/l is unchanged.
-//  * epilogue: O/l in bf16 and LSE = (m + log2 l) * ln 2 (natural log).
+//  * epilogue: O/l in the input format and LSE = (m + log2 l) * ln 2 (natural log).
+//  * Q, K, V, P and O are bf16 or f16 (template parameter E); accumulation is f32.
 // Tensor memory (512 columns): S0 [0,128) S1 [128,256) O0 [256,256+D)
-// O1 [256+D, 256+2D); P_k (bf16 pairs) overwrites the first 64 columns of S_k.
+// O1 [256+D, 256+2D); P_k (16-bit pairs) overwrites the first 64 columns of S_k.
 #pragma once
 
 #include <cuda.h>
@@ -78,7 +79,7 @@ struct Cfg {
 };
 
 struct Params {
-  __nv_bfloat16* o;
+  uint16_t* o;  // 16-bit elements (bf16 or f16, as the kernel's element format)
   float* lse;
   int B, H, Sq, Sk;
   int Hk;            // key/value heads (H a multiple of Hk; query head h reads h / (H / Hk))
@@ -102,7 +103,8 @@ __device__ __forceinline__ void tile_range(const MaskGeom& g, int r0, int r1, in
   jhi = khi / BN + 1;
 }
 
-template <int D>
+// E: element format of Q, K, V, P and O (ElemBF16 or ElemF16).
+template <int D, class E>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const Params p) {
@@ -273,7 +275,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // p = 2^(s * scale * log2(e) - m): pairs in f32x2.  On fully visible
       // tiles one pair in four is exponentiated on the FMA pipe (polynomial),
       // the rest on MUFU; tiles with masked (-inf) scores use MUFU only, whose
-      // ex2(-inf) is exactly 0.  P goes to tensor memory as bf16 pairs in two
+      // ex2(-inf) is exactly 0.  P goes to tensor memory as 16-bit pairs in two
       // 64-column halves (columns [0,32) and [32,64) of S_k).
       auto exp_store = [&](auto use_poly) {
 #pragma unroll
@@ -294,7 +296,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             acc2[c & 3] = f2_add(acc2[c & 3], p2);
             float p0, p1;
             f2_unpack(p2, p0, p1);
-            pk[c] = pack_bf16x2(p0, p1);
+            pk[c] = E::pack2(p0, p1);
           }
           tmem_st32(tS + half * 32, pk);
         }
@@ -330,7 +332,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_arrive(bar(C::kBarP + k));
     }
 
-    // Epilogue: O = O / l (bf16), LSE = (m + log2 l) ln 2.
+    // Epilogue: O = O / l (input format), LSE = (m + log2 l) ln 2.
     if (valid[k] && ok) {
       const bool row_ok = i < p.Sq;
       const size_t orow = ((size_t(b) * p.Sq + size_t(i)) * p.H + h) * D;
@@ -352,7 +354,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint32_t w[16];
 #pragma unroll
           for (int c = 0; c < 16; ++c)
-            w[c] = pack_bf16x2(__uint_as_float(r[2 * c]) * inv_l, __uint_as_float(r[2 * c + 1]) * inv_l);
+            w[c] = E::pack2(__uint_as_float(r[2 * c]) * inv_l, __uint_as_float(r[2 * c + 1]) * inv_l);
           if (row_ok) {
             uint8_t* dst = reinterpret_cast<uint8_t*>(p.o + orow + c0);
 #pragma unroll
@@ -402,8 +404,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0 && any_work) {
-      constexpr uint32_t idesc_qk = idesc_bf16_f32(BM, BN, false, false);
-      constexpr uint32_t idesc_pv = idesc_bf16_f32(BM, D, false, true);
+      constexpr uint32_t idesc_qk = idesc_f32acc(BM, BN, false, false, E::kFmt);
+      constexpr uint32_t idesc_pv = idesc_f32acc(BM, D, false, true, E::kFmt);
       auto in_range = [&](int k, int j) { return j >= jlo[k] && j < jhi[k]; };
       auto issue_s = [&](int k, int s) {
         if constexpr (D == 128)

@@ -348,6 +348,14 @@ __device__ __forceinline__ void mma_chain_ts_mn8(uint32_t d_tmem, uint32_t a_tme
       : "memory");
 }
 
+// Instruction descriptor for kind::f16 with 16-bit A/B of format `fmt`
+// (0 = f16, 1 = bf16; A and B always the same) and f32 accumulate.
+__host__ __device__ constexpr uint32_t idesc_f32acc(int M, int N, bool a_mn_major,
+                                                    bool b_mn_major, uint32_t fmt) {
+  return (1u << 4) | (fmt << 7) | (fmt << 10) | ((a_mn_major ? 1u : 0u) << 15) |
+         ((b_mn_major ? 1u : 0u) << 16) | (uint32_t(N >> 3) << 17) | (uint32_t(M >> 4) << 24);
+}
+
 // Instruction descriptor for kind::f16 with bf16 A/B and f32 accumulate.
 // Fields: [4,6) D format (1 = f32), [7,10) A format (1 = bf16), [10,13) B format,
 // [15] A major (1 = MN-major), [16] B major, [17,23) N>>3, [24,29) M>>4.
@@ -697,6 +705,31 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 __device__ __forceinline__ void red_add_f32(float* gptr, float a) {
   asm volatile("red.global.add.f32 [%0], %1;" ::"l"(gptr), "f"(a) : "memory");
 }
+
+// The two 16-bit element formats of the operands and outputs.  pack2 rounds
+// two floats to nearest-even and puts `lo` in bits 0..15; unpack2 widens a
+// packed pair exactly.
+struct ElemBF16 {
+  static constexpr uint32_t kFmt = 1;  // kind::f16 operand format code
+  __device__ static __forceinline__ uint32_t pack2(float lo, float hi) { return pack_bf16x2(lo, hi); }
+  __device__ static __forceinline__ void unpack2(uint32_t u, float& lo, float& hi) {
+    lo = __uint_as_float(u << 16);
+    hi = __uint_as_float(u & 0xffff0000u);
+  }
+};
+struct ElemF16 {
+  static constexpr uint32_t kFmt = 0;
+  __device__ static __forceinline__ uint32_t pack2(float lo, float hi) {
+    uint32_t r;
+    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+  }
+  __device__ static __forceinline__ void unpack2(uint32_t u, float& lo, float& hi) {
+    asm("{\n\t.reg .f16 l, h;\n\tmov.b32 {l, h}, %2;\n\tcvt.f32.f16 %0, l;\n\tcvt.f32.f16 %1, h;\n\t}"
+        : "=f"(lo), "=f"(hi)
+        : "r"(u));
+  }
+};
 
 __device__ __forceinline__ void red_add_v4(float* gptr, float a, float b, float c, float d) {
   asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(gptr), "f"(a), "f"(b), "f"(c),

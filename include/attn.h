@@ -17,7 +17,8 @@
  * attention scores instead of storing them.
  *
  * Conventions for every entry point:
- *   - Tensors Q, K, V, O, dO, dQ, dK, dV are bfloat16, row-major
+ *   - Tensors Q, K, V, O, dO, dQ, dK, dV are bfloat16 (float16 through the
+ *     _ex entry points), row-major
  *     (batch, seqlen, nheads, head_dim) with head_dim contiguous and no padding
  *     between rows ("BSHD"), 16-byte aligned.  Q, O, dO, dQ have seqlen Sq;
  *     K, V, dK, dV have seqlen Sk.
@@ -71,8 +72,18 @@ typedef enum {
     ATTN_ERR_LAUNCH = 8,    /* a CUDA call (descriptor build, launch) failed      */
     ATTN_ERR_TIMEOUT = 9,   /* a device-side bounded wait ran out                 */
     ATTN_ERR_WORKSPACE = 10, /* workspace NULL, misaligned or smaller than needed */
-    ATTN_ERR_SCRATCH = 11    /* problem too large for attn_bwd_noalloc's scratch  */
+    ATTN_ERR_SCRATCH = 11,   /* problem too large for attn_bwd_noalloc's scratch  */
+    ATTN_ERR_DTYPE = 12      /* element format not one of attn_dtype              */
 } attn_status;
+
+/* Element format of the 16-bit tensors (Q, K, V, O, dO, dQ, dK, dV): the RTX
+ * 5060 flash-attention page (pptc.cn), section 6.1, names fp16 and bf16 as the
+ * mature input types and its section 4.4 test draws float16 tensors.
+ * Accumulation is float32 in both. */
+typedef enum {
+    ATTN_DTYPE_BF16 = 0,
+    ATTN_DTYPE_F16 = 1
+} attn_dtype;
 
 /*
  * attn_fwd - O and LSE of exact attention (FlashAttention-2 overview, section 2.2:
@@ -141,7 +152,9 @@ ATTN_API attn_status attn_bwd_dq_finalize(void* dq, int B, int Sq, int H, int D,
                                           void* workspace, size_t workspace_bytes, void* stream);
 
 /*
- * Grouped K/V heads (GQA; MQA when Hk == 1).  The pages' Transformers snippet
+ * The extended forms: grouped K/V heads and the element format.
+ *
+ * Grouped K/V heads (GQA; MQA when Hk == 1): the pages' Transformers snippet
  * (FlashAttention-2 overview, lshu.cn, section 3.3) shapes Q with num_heads and
  * K, V with num_kv_heads for the same call.  K and V (and dK, dV) have Hk heads,
  * Q, O, dO, dQ and lse have H heads, H a multiple of Hk; query head h attends
@@ -149,26 +162,38 @@ ATTN_API attn_status attn_bwd_dq_finalize(void* dq, int B, int Sq, int H, int D,
  * dK and dV of a shared head are the sums over its query heads (accumulated in
  * the kernel, no atomics).  The workspace is sized by H, as for attn_bwd.
  *
- *   k, v [B, Sk, Hk, D] bf16 (in)     dk, dv [B, Sk, Hk, D] bf16 (out)
- *   every other argument as in attn_fwd / attn_bwd / attn_bwd_main.
+ * dtype (attn_dtype): the format of every 16-bit tensor of the call; P and dS
+ * are rounded to that format before their products, outputs are rounded from
+ * float32 accumulators.
+ *
+ *   k, v [B, Sk, Hk, D] (in)     dk, dv [B, Sk, Hk, D] (out)
+ *   every other argument as in attn_fwd / attn_bwd and its three stages.
  * Errors: as the entry points they extend; ATTN_ERR_SHAPE also if Hk < 1,
- * Hk > H or H is not a multiple of Hk.  With Hk == H they equal attn_fwd,
- * attn_bwd and attn_bwd_main.
+ * Hk > H or H is not a multiple of Hk; ATTN_ERR_DTYPE for an unknown dtype.
+ * With Hk == H and ATTN_DTYPE_BF16 they equal attn_fwd, attn_bwd,
+ * attn_bwd_preprocess, attn_bwd_main and attn_bwd_dq_finalize.
  */
-ATTN_API attn_status attn_fwd_gqa(const void* q, const void* k, const void* v, void* o,
-                                  float* lse, int B, int Sq, int Sk, int H, int Hk, int D,
-                                  float scale, int causal, int win_left, int win_right,
-                                  void* stream);
-ATTN_API attn_status attn_bwd_gqa(const void* q, const void* k, const void* v, const void* o,
-                                  const void* dout, const float* lse, void* dq, void* dk,
-                                  void* dv, int B, int Sq, int Sk, int H, int Hk, int D,
-                                  float scale, int causal, int win_left, int win_right,
-                                  void* workspace, size_t workspace_bytes, void* stream);
-ATTN_API attn_status attn_bwd_main_gqa(const void* q, const void* k, const void* v,
-                                       const void* dout, void* dk, void* dv, int B, int Sq,
-                                       int Sk, int H, int Hk, int D, float scale, int causal,
-                                       int win_left, int win_right, void* workspace,
-                                       size_t workspace_bytes, void* stream);
+ATTN_API attn_status attn_fwd_ex(const void* q, const void* k, const void* v, void* o,
+                                 float* lse, int B, int Sq, int Sk, int H, int Hk, int D,
+                                 int dtype, float scale, int causal, int win_left, int win_right,
+                                 void* stream);
+ATTN_API attn_status attn_bwd_ex(const void* q, const void* k, const void* v, const void* o,
+                                 const void* dout, const float* lse, void* dq, void* dk,
+                                 void* dv, int B, int Sq, int Sk, int H, int Hk, int D,
+                                 int dtype, float scale, int causal, int win_left, int win_right,
+                                 void* workspace, size_t workspace_bytes, void* stream);
+ATTN_API attn_status attn_bwd_preprocess_ex(const void* o, const void* dout, const float* lse,
+                                            int B, int Sq, int H, int D, int dtype,
+                                            void* workspace, size_t workspace_bytes,
+                                            void* stream);
+ATTN_API attn_status attn_bwd_main_ex(const void* q, const void* k, const void* v,
+                                      const void* dout, void* dk, void* dv, int B, int Sq,
+                                      int Sk, int H, int Hk, int D, int dtype, float scale,
+                                      int causal, int win_left, int win_right, void* workspace,
+                                      size_t workspace_bytes, void* stream);
+ATTN_API attn_status attn_bwd_dq_finalize_ex(void* dq, int B, int Sq, int H, int D, int dtype,
+                                             float scale, void* workspace,
+                                             size_t workspace_bytes, void* stream);
 
 /*
  * attn_bwd_noalloc - attn_bwd for callers that cannot allocate device memory.

@@ -12,7 +12,8 @@ Recipe (fixed here, the pages only say "random"):
   * draw order: Q, K, V, dO, each ``standard_normal`` in float32 of shape
     (B, S, H, D) (K and V with Hk heads when the key/value heads are
     grouped), multiplied by the workload's input scale;
-  * round every value to bfloat16 with round-to-nearest-even;
+  * round every value to bfloat16 (or IEEE float16 for the float16 tests)
+    with round-to-nearest-even;
   * the CUDA path receives the bf16 bit patterns; the oracle receives the
     same values widened to float64.
 """
@@ -107,14 +108,32 @@ def bf16_bits_to_f32(b: np.ndarray) -> np.ndarray:
     return (b.astype(np.uint32) << np.uint32(16)).view(np.float32)
 
 
+def f32_to_f16_bits(x: np.ndarray) -> np.ndarray:
+    """Round float32 values to IEEE float16 (nearest, ties to even); return the bit patterns as uint16."""
+    return np.ascontiguousarray(x, dtype=np.float32).astype(np.float16).view(np.uint16)
+
+
+def f16_bits_to_f32(b: np.ndarray) -> np.ndarray:
+    """Widen float16 bit patterns (uint16) to float32 exactly."""
+    return np.ascontiguousarray(b, dtype=np.uint16).view(np.float16).astype(np.float32)
+
+
+def bits_to_f32(b: np.ndarray, fmt: str = "bf16") -> np.ndarray:
+    return f16_bits_to_f32(b) if fmt == "f16" else bf16_bits_to_f32(b)
+
+
 def make_inputs(B: int, Sq: int, Sk: int, H: int, D: int, seed: int,
-                input_scale: float = 1.0, with_dout: bool = False, Hk: Optional[int] = None):
+                input_scale: float = 1.0, with_dout: bool = False, Hk: Optional[int] = None,
+                fmt: str = "bf16"):
     """Draw Q, K, V (and dO) for one workload.
 
-    Returns a dict of bf16 bit arrays (uint16) with keys 'q', 'k', 'v' and,
-    if requested, 'do'; Q and dO have shape (B, Sq, H, D), K and V
-    (B, Sk, Hk, D) with Hk = H unless given (grouped K/V heads).
+    Returns a dict of 16-bit bit arrays (uint16; bfloat16, or IEEE float16 when
+    fmt == "f16") with keys 'q', 'k', 'v' and, if requested, 'do'; Q and dO have
+    shape (B, Sq, H, D), K and V (B, Sk, Hk, D) with Hk = H unless given
+    (grouped K/V heads).  The float32 draws do not depend on fmt.
     """
+    if fmt not in ("bf16", "f16"):
+        raise ValueError(fmt)
     rng = np.random.Generator(np.random.PCG64(seed))
     out = {}
     Hk = H if Hk is None else Hk
@@ -125,7 +144,7 @@ def make_inputs(B: int, Sq: int, Sk: int, H: int, D: int, seed: int,
         x = rng.standard_normal((B, S, heads, D), dtype=np.float32)
         if input_scale != 1.0:
             x *= np.float32(input_scale)
-        out[name] = f32_to_bf16_bits(x)
+        out[name] = f32_to_f16_bits(x) if fmt == "f16" else f32_to_bf16_bits(x)
     return out
 
 

@@ -1,12 +1,12 @@
-"""Shared helpers of the tests: device transfer of the seeded bf16 inputs and
-the parity bars (bf16 inputs/outputs with fp32 accumulation):
+"""Shared helpers of the tests: device transfer of the seeded 16-bit inputs and
+the parity bars (bf16 or f16 inputs/outputs with fp32 accumulation):
 max |dO| <= 2e-2, mean |dO| <= 2e-3, |dLSE| <= 1e-3 absolute, and for each
 gradient max |dg| / max |g_oracle| <= 5e-2.  A per-row relative bar
 ||dO_i|| / ||O_i|| <= 2e-2 is added because O rows of long causal rows are
 small enough that the absolute bar alone could miss a wrong row."""
 import numpy as np
 
-from synth import bf16_bits_to_f32
+from synth import bits_to_f32
 
 O_MAX = 2e-2
 O_MEAN = 2e-3
@@ -15,9 +15,10 @@ GRAD_REL = 5e-2
 O_ROW_REL = 2e-2
 
 
-def to_device(bits):
+def to_device(bits, fmt="bf16"):
     import torch
-    t = torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16)
+    dtype = torch.float16 if fmt == "f16" else torch.bfloat16
+    t = torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(dtype)
     return t.cuda()
 
 
@@ -25,8 +26,8 @@ def to_f64(t):
     return t.float().cpu().numpy().astype(np.float64)
 
 
-def f64(bits):
-    return bf16_bits_to_f32(bits).astype(np.float64)
+def f64(bits, fmt="bf16"):
+    return bits_to_f32(bits, fmt).astype(np.float64)
 
 
 def check_fwd(o, lse, o_ref, lse_ref, what=""):

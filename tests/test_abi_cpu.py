@@ -32,13 +32,19 @@ def test_library_exports_every_declared_symbol():
 def test_status_enum_matches_binding():
     from exact_attention_156_b200 import ATTN_STATUS
     text = open(HEADER).read()
-    enum = dict((int(v), k) for k, v in re.findall(r"(ATTN_\w+)\s*=\s*(\d+)", text))
+    block = text[:text.index("} attn_status;")]
+    block = block[block.rindex("typedef enum"):]
+    enum = dict((int(v), k) for k, v in re.findall(r"(ATTN_\w+)\s*=\s*(\d+)", block))
     assert enum == ATTN_STATUS
+    dtypes = re.search(r"typedef enum \{([^}]*)\} attn_dtype;", text).group(1)
+    from exact_attention_156_b200._binding import ATTN_DTYPE_BF16, ATTN_DTYPE_F16
+    assert dict(re.findall(r"(ATTN_DTYPE_\w+)\s*=\s*(\d+)", dtypes)) == {
+        "ATTN_DTYPE_BF16": str(ATTN_DTYPE_BF16), "ATTN_DTYPE_F16": str(ATTN_DTYPE_F16)}
 
 
 def test_status_strings():
     from exact_attention_156_b200 import status_string
-    for s in range(12):
+    for s in range(13):
         assert status_string(s) and status_string(s) != "unknown status"
     assert status_string(99) == "unknown status"
 
@@ -105,25 +111,34 @@ def test_binding_refuses_cpu_tensors():
         attn_fwd(q, q, q)
 
 
-def test_grouped_head_counts_are_validated():
+def test_extended_entry_points_validate_heads_and_dtype():
     from exact_attention_156_b200 import lib
+    DTYPE = 12
 
-    def fwd(H, Hk, D=128):
-        return lib.attn_fwd_gqa(0x1000, 0x2000, 0x3000, 0x4000, 0x5000, 1, 128, 128, H, Hk, D,
-                                0.125, 1, -1, -1, None)
+    def fwd(H, Hk, D=128, dtype=0):
+        return lib.attn_fwd_ex(0x1000, 0x2000, 0x3000, 0x4000, 0x5000, 1, 128, 128, H, Hk, D,
+                               dtype, 0.125, 1, -1, -1, None)
     assert fwd(8, 0) == SHAPE
     assert fwd(8, 16) == SHAPE
     assert fwd(8, 3) == SHAPE
     assert fwd(6, 4) == SHAPE
     assert fwd(8, 2, D=96) == HEADDIM
-    assert fwd(8, 2) in (ARCH, DEVICE)       # well-formed: stops at the device checks
-    assert fwd(8, 1) in (ARCH, DEVICE)
+    assert fwd(8, 2, dtype=2) == DTYPE
+    assert fwd(8, 2, dtype=-1) == DTYPE
+    for dtype in (0, 1):                     # well-formed: stops at the device checks
+        assert fwd(8, 2, dtype=dtype) in (ARCH, DEVICE)
+        assert fwd(8, 1, dtype=dtype) in (ARCH, DEVICE)
     p = [0x1000 * (i + 1) for i in range(9)]
     ws = lib.attn_bwd_workspace_size(1, 128, 8, 128)
-    assert lib.attn_bwd_gqa(*p, 1, 128, 128, 8, 3, 128, 0.1, 1, -1, -1, 0x100000, ws, None) == SHAPE
-    assert lib.attn_bwd_main_gqa(*p[:6], 1, 128, 128, 8, 0, 128, 0.1, 1, -1, -1, 0x100000, ws,
-                                 None) == SHAPE
-    assert lib.attn_bwd_gqa(*p, 1, 128, 128, 8, 2, 128, 0.1, 1, -1, -1, None, ws, None) == 10
+    assert lib.attn_bwd_ex(*p, 1, 128, 128, 8, 3, 128, 0, 0.1, 1, -1, -1, 0x100000, ws,
+                           None) == SHAPE
+    assert lib.attn_bwd_ex(*p, 1, 128, 128, 8, 2, 128, 5, 0.1, 1, -1, -1, 0x100000, ws,
+                           None) == DTYPE
+    assert lib.attn_bwd_main_ex(*p[:6], 1, 128, 128, 8, 0, 128, 1, 0.1, 1, -1, -1, 0x100000, ws,
+                                None) == SHAPE
+    assert lib.attn_bwd_ex(*p, 1, 128, 128, 8, 2, 128, 1, 0.1, 1, -1, -1, None, ws, None) == 10
+    assert lib.attn_bwd_preprocess_ex(*p[:3], 1, 128, 8, 128, 7, 0x100000, ws, None) == DTYPE
+    assert lib.attn_bwd_dq_finalize_ex(p[0], 1, 128, 8, 128, 9, 0.1, 0x100000, ws, None) == DTYPE
 
 
 def test_binding_checks_key_value_heads():
