@@ -10,6 +10,7 @@ from .attn_ref import (  # noqa: F401
     attention_backward_kv_head,
     attention_backward_rows,
     attention_backward_rows_dq,
+    attention_decode,
     attention_forward,
     attention_forward_rows,
     kv_head,

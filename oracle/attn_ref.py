@@ -298,6 +298,34 @@ def attention_backward_kv_head(q, k, v, do, b: int, g: int, scale: float,
     return dk, dv
 
 
+def attention_decode(q, k_cache, v_cache, cache_seqlens, scale: float, causal: int = 0):
+    """O and LSE for a few new query rows per sequence against a K/V cache.
+
+    FlashAttention-2 overview (lshu.cn), section 3.3: flash_attn_func has no
+    incremental (KV-cache) path and flash_attn_with_kvcache is the entry point
+    for it; the pages give no further semantics.  Reading: q (B, Sq, H, D) holds
+    the Sq newest query rows of each sequence, k_cache, v_cache (B, Smax, Hk, D)
+    hold that sequence's keys and values in their first cache_seqlens[b] rows
+    (the new keys already appended), and those rows are all the keys it
+    attends over; rows past the length are never read.  Causal is the same
+    bottom-right rule as everywhere (query i of Sq sees keys
+    j <= i + cache_seqlens[b] - Sq).  Returns o (B, Sq, H, D), lse (B, H, Sq).
+    """
+    q = _f64(q)
+    B, Sq, H, D = q.shape
+    o = np.zeros((B, Sq, H, D))
+    lse = np.zeros((B, H, Sq))
+    for b in range(B):
+        L = int(cache_seqlens[b])
+        if L < 1:
+            raise ValueError("every sequence needs at least one cached key")
+        ob, lb = attention_forward(q[b:b + 1], _f64(k_cache[b:b + 1, :L]),
+                                   _f64(v_cache[b:b + 1, :L]), scale, causal)
+        o[b] = ob[0]
+        lse[b] = lb[0]
+    return o, lse
+
+
 def online_softmax_forward(q, k, v, scale: float, tile: int, causal: int = 0,
                            win_left: int = -1, win_right: int = -1):
     """The pages' online-softmax recurrence, one key tile at a time.
