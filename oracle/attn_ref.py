@@ -317,8 +317,13 @@ def attention_decode(q, k_cache, v_cache, cache_seqlens, scale: float, causal: i
     lse = np.zeros((B, H, Sq))
     for b in range(B):
         L = int(cache_seqlens[b])
-        if L < 1:
-            raise ValueError("every sequence needs at least one cached key")
+        if L < 0:
+            raise ValueError("cache lengths are counts of rows")
+        if L == 0:
+            # no key to attend to: every row of the sequence is a row with no
+            # visible key, O = 0 and LSE = -inf as in attention_forward
+            lse[b] = -np.inf
+            continue
         ob, lb = attention_forward(q[b:b + 1], _f64(k_cache[b:b + 1, :L]),
                                    _f64(v_cache[b:b + 1, :L]), scale, causal)
         o[b] = ob[0]

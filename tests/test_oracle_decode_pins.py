@@ -76,7 +76,15 @@ def test_brute_force_rows():
                 assert abs(lse[b, h, i] - (m + np.log(z))) < 1e-13
 
 
-def test_empty_cache_is_refused():
-    q, k, v = _inputs(1, 1, 4, 1, 1, 4, 6)
+def test_empty_cache_gives_rows_with_no_visible_key():
+    """A zero-length cache leaves every row of that sequence without a visible
+    key: O = 0 and LSE = -inf (the rule for such rows everywhere), and the other
+    sequences are unaffected."""
+    q, k, v = _inputs(2, 2, 4, 1, 1, 4, 6)
+    o, lse = attention_decode(q, k, v, [0, 3], 0.5, 0)
+    assert np.all(o[0] == 0) and np.all(np.isneginf(lse[0]))
+    o1, lse1 = attention_decode(q[1:], k[1:], v[1:], [3], 0.5, 0)
+    np.testing.assert_array_equal(o[1], o1[0])
+    np.testing.assert_array_equal(lse[1], lse1[0])
     with pytest.raises(ValueError):
-        attention_decode(q, k, v, [0], 0.5, 0)
+        attention_decode(q, k, v, [-1, 3], 0.5, 0)
