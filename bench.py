@@ -40,7 +40,11 @@ WORKLOAD = dict(name="c5_b1h32s8192d128_fwdbwd", B=1, H=32, Hk=32, Sq=8192, Sk=8
 # grouped K/V heads (GQA, 4 query heads per K/V head) at the same sizes
 GQA_WORKLOAD = dict(name="gqa_b1h32hk8s8192d128_fwdbwd", B=1, H=32, Hk=8, Sq=8192, Sk=8192,
                     D=128, causal=1, win_left=-1, win_right=-1, input_scale=0.5, seed=1006)
-WORKLOADS = {"fwdbwd": WORKLOAD, "gqa": GQA_WORKLOAD}
+# KV-cache decode: one new query row per sequence over a full 8192-row cache
+DECODE_WORKLOAD = dict(name="decode_b8h32hk8l8192d128", B=8, Sq=1, H=32, Hk=8, Smax=8192,
+                       D=128, causal=0, input_scale=0.5, seed=1007)
+WORKLOADS = {"fwdbwd": WORKLOAD, "gqa": GQA_WORKLOAD, "decode": DECODE_WORKLOAD}
+DECODE_METRIC = "KV-cache decode: cached K/V bytes read per second"
 FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "hbm_gbs": 6650.0, "source": "fallback"}
 BWD_KERNEL_SOURCES = ["bwd_sm100.cuh", "ptx.cuh", "common.cuh"]
 FWD_KERNEL_SOURCES = ["fwd_sm100.cuh", "ptx.cuh", "common.cuh"]
@@ -444,6 +448,177 @@ def run_gpu(args):
     return 0
 
 
+def decode_bytes(w) -> float:
+    """Algorithmic HBM bytes of one decode call: every valid cached K and V
+    element once, plus the query rows read and the output rows written."""
+    kv = 2.0 * w["B"] * w["Smax"] * w["Hk"] * w["D"] * 2
+    qo = 2.0 * w["B"] * w["Sq"] * w["H"] * w["D"] * 2
+    return kv + qo
+
+
+DECODE_KERNEL_SOURCES = ["decode_sm100.cuh", "ptx.cuh", "common.cuh"]
+
+
+def decode_oracle_inputs(w, rank: int = 0):
+    from synth import bits_to_f32, make_inputs
+    bits = make_inputs(w["B"], w["Sq"], w["Smax"], w["H"], w["D"], w["seed"] + rank,
+                       w["input_scale"], Hk=w["Hk"])
+    return {n: bits_to_f32(bits[n]) for n in ("q", "k", "v")}
+
+
+def decode_oracle_step(inputs, w):
+    """One oracle pass over the whole decode workload (every sequence, every
+    head, full-length cache).  Returns its seconds."""
+    import numpy as np
+    import oracle
+    t0 = time.perf_counter()
+    oracle.attention_decode(inputs["q"], inputs["k"], inputs["v"],
+                            np.full(w["B"], w["Smax"]), 1.0 / math.sqrt(w["D"]), w["causal"])
+    return time.perf_counter() - t0
+
+
+def decode_cpu_baseline(w, budget_s: float = 10.0):
+    inputs = decode_oracle_inputs(w)
+    tot, n = 0.0, 0
+    while tot < budget_s and n < 64:
+        tot += decode_oracle_step(inputs, w)
+        n += 1
+    return {"value": n * decode_bytes(w) / tot / 1e9, "unit": "GB/s", "cores": blas_threads(),
+            "kind": "oracle",
+            "sample": f"{n} passes of the float64 numpy oracle over the whole {w['name']} "
+                      f"workload ({tot:.1f} s total)"}
+
+
+def decode_config(w):
+    return {"workload": f"{w['name']}: decode, B={w['B']} Sq={w['Sq']} H={w['H']} Hk={w['Hk']} "
+                        f"cache {w['Smax']} rows (all valid) D={w['D']}, inputs "
+                        f"N(0,1)*{w['input_scale']}",
+            "B": w["B"], "Sq": w["Sq"], "H": w["H"], "Hk": w["Hk"], "Smax": w["Smax"],
+            "D": w["D"],
+            "l2": f"no flush: the K/V cache ({decode_bytes(w) / 2**20:.0f} MiB) exceeds the "
+                  "126 MB L2"}
+
+
+def run_decode_reference(args):
+    rank, _, _ = dist_env()
+    if rank != 0:
+        return 0
+    w = DECODE_WORKLOAD
+    inputs = decode_oracle_inputs(w)
+    for _ in range(args.warmup):
+        decode_oracle_step(inputs, w)
+    tot = sum(decode_oracle_step(inputs, w) for _ in range(args.steps))
+    value = args.steps * decode_bytes(w) / tot / 1e9
+    print(json.dumps({
+        "impl": "reference", "metric": DECODE_METRIC, "value": value, "unit": "GB/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": tot / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": decode_config(w),
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": blas_threads(),
+                         "kind": "oracle",
+                         "sample": f"each step: the whole {w['name']} workload, float64 numpy"},
+        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0}}), flush=True)
+    return 0
+
+
+def run_decode(args):
+    """The KV-cache decode workload: the cache is resident on the device (it is
+    the state a decode step reads); one call = split kernel + combine kernel."""
+    import torch
+    rank, world, local = dist_env()
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    device = torch.device("cuda", local if world > 1 else torch.cuda.current_device())
+    torch.cuda.set_device(device)
+    from exact_attention_156_b200 import (attn_decode, attn_decode_workspace_size,
+                                          get_last_device_error)
+    from synth import make_inputs
+    w = DECODE_WORKLOAD
+    B, Sq, H, Hk, Smax, D = w["B"], w["Sq"], w["H"], w["Hk"], w["Smax"], w["D"]
+    bits = make_inputs(B, Sq, Smax, H, D, w["seed"] + rank, w["input_scale"], Hk=Hk,
+                       fmt=args.dtype)
+    tdtype = torch.float16 if args.dtype == "f16" else torch.bfloat16
+    as_t = lambda a: torch.from_numpy(a.view("int16")).view(tdtype)
+    q_host = as_t(bits["q"]).pin_memory()
+    q = q_host.to(device)
+    kc, vc = as_t(bits["k"]).to(device), as_t(bits["v"]).to(device)
+    seqlens = torch.full((B,), Smax, dtype=torch.int32, device=device)
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, Sq), dtype=torch.float32, device=device)
+    ws = torch.empty(attn_decode_workspace_size(B, Sq, Smax, H, Hk, D), dtype=torch.uint8,
+                     device=device)
+    stream = torch.cuda.current_stream(device)
+    step = lambda: attn_decode(q, kc, vc, seqlens, causal=bool(w["causal"]), out=o, lse=lse,
+                               workspace=ws, stream=stream)
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(device)
+    barrier(device)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler("GPU-" + str(torch.cuda.get_device_properties(device).uuid))
+    sampler.start()
+    start.record(stream)
+    for _ in range(args.steps):
+        step()
+    end.record(stream)
+    torch.cuda.synchronize(device)
+    barrier(device)
+    clocks = sampler.stop()
+    if get_last_device_error() != 0:
+        raise RuntimeError("device-side timeout during the timed region")
+    ms = reduce_max(start.elapsed_time(end), device) / args.steps
+    gbs = world * decode_bytes(w) / (ms * 1e-3) / 1e9
+    # end to end: the new query rows from pinned host memory, O and LSE back to the host
+    o_host = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+    l_host = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+    torch.cuda.synchronize(device)
+    barrier(device)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        q.copy_(q_host, non_blocking=True)
+        step()
+        o_host.copy_(o, non_blocking=True)
+        l_host.copy_(lse, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize(device)
+    barrier(device)
+    e2e_ms = reduce_max(e0.elapsed_time(e1), device) / args.steps
+    peaks = load_peaks()
+    peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    line = {
+        "metric": DECODE_METRIC, "value": gbs, "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": args.dtype, "data": "synthetic",
+        "config": decode_config(w),
+        "roofline": {"bound": "hbm",
+                     "kernel": "attn_decode_kernel<128> (timed with its combine launch)",
+                     "achieved": decode_bytes(w) / (ms * 1e-3) / 1e9, "peak": peak,
+                     "unit": "GB/s", "frac": decode_bytes(w) / (ms * 1e-3) / 1e9 / peak,
+                     "peak_source": f"{peaks.get('source')} hbm_gbs",
+                     "traffic": committed_traffic(traffic_key("attn_decode_kernel", w, args.dtype),
+                                                  sources_sha(DECODE_KERNEL_SOURCES))},
+        "e2e": {"value": world * decode_bytes(w) / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
+                "h2d_bytes_per_step": q_host.numel() * q_host.element_size(),
+                "d2h_bytes_per_step": o_host.numel() * o_host.element_size()
+                + l_host.numel() * l_host.element_size(), "ms_per_step": e2e_ms},
+        "gpu_launches": 2 * args.steps,
+        "clocks": clocks,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = decode_cpu_baseline(w)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -454,7 +629,8 @@ def main(argv=None):
                     help="element format of the 16-bit tensors (default bf16)")
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="fwdbwd",
                     help="fwdbwd: the headline fwd+bwd workload (default); gqa: the same sizes "
-                         "with 8 K/V heads for 32 query heads")
+                         "with 8 K/V heads for 32 query heads; decode: KV-cache decode "
+                         "(B8 H32 Hk8, 8192 cached rows, one new row)")
     ap.add_argument("--no-cpu-baseline", action="store_true",
                     help="skip the timed oracle sample (it adds ~15 s of CPU time)")
     ap.add_argument("--no-e2e", action="store_true",
@@ -462,6 +638,8 @@ def main(argv=None):
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.workload == "decode":
+        return run_decode_reference(args) if args.impl == "reference" else run_decode(args)
     if args.impl == "reference":
         return run_reference(args)
     return run_gpu(args)

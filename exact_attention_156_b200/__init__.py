@@ -4,6 +4,7 @@ recompute-based backward, behind the C ABI of include/attn.h.
     from exact_attention_156_b200 import attn_fwd, attn_bwd
     o, lse = attn_fwd(q, k, v, causal=True)              # q, k, v: bf16 (B, S, H, D) CUDA
     dq, dk, dv = attn_bwd(q, k, v, o, do, lse, causal=True)
+    o, lse = attn_decode(q_new, k_cache, v_cache, cache_seqlens, causal=True)  # KV-cache decode
 """
 from ._binding import (  # noqa: F401
     ATTN_STATUS,
@@ -12,6 +13,8 @@ from ._binding import (  # noqa: F401
     attn_bwd,
     attn_bwd_stages,
     attn_bwd_workspace_size,
+    attn_decode,
+    attn_decode_workspace_size,
     attn_fwd,
     device_timeout_selftest,
     get_last_device_error,

@@ -61,6 +61,10 @@ def _load() -> ctypes.CDLL:
     lib.attn_bwd_main_ex.restype = i
     lib.attn_bwd_dq_finalize_ex.argtypes = [vp, i, i, i, i, i, f, vp, sz, vp]
     lib.attn_bwd_dq_finalize_ex.restype = i
+    lib.attn_decode_workspace_size.argtypes = [i, i, i, i, i, i]
+    lib.attn_decode_workspace_size.restype = sz
+    lib.attn_decode.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, f, i, vp, sz, vp]
+    lib.attn_decode.restype = i
     lib.attn_bwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, i,
                                      i, vp]
     lib.attn_bwd_noalloc.restype = i
@@ -260,6 +264,43 @@ def attn_bwd_stages(q, k, v, out, dout, lse, dq, dk, dv, workspace,
     if between:
         between(3)
     return dq, dk, dv
+
+
+def attn_decode_workspace_size(B: int, Sq: int, Smax: int, H: int, Hk: int, D: int) -> int:
+    return int(lib.attn_decode_workspace_size(B, Sq, Smax, H, Hk, D))
+
+
+def attn_decode(q, k_cache, v_cache, cache_seqlens, softmax_scale: Optional[float] = None,
+                causal: bool = False, out=None, lse=None, workspace=None, stream=None):
+    """Attention of the Sq newest query rows q (B,Sq,H,D) of each sequence over
+    the first cache_seqlens[b] rows of k_cache, v_cache (B,Smax,Hk,D).
+
+    cache_seqlens is an int32 CUDA tensor (B,).  All 16-bit tensors share one
+    format (bf16 or float16).  Returns (o (B,Sq,H,D), lse fp32 (B,H,Sq)).
+    """
+    import torch
+    dt = _dtype_code(q)
+    for t, n in ((q, "q"), (k_cache, "k_cache"), (v_cache, "v_cache")):
+        _check(t, n, q.dtype, 4)
+    _check(cache_seqlens, "cache_seqlens", torch.int32, 1)
+    B, Sq, H, D = q.shape
+    Smax = k_cache.shape[1]
+    Hk = _kv_heads(q, k_cache, v_cache)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, H, Sq), dtype=torch.float32, device=q.device)
+    need = attn_decode_workspace_size(B, Sq, Smax, H, Hk, D)
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
+    st = lib.attn_decode(q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(),
+                         cache_seqlens.data_ptr(), out.data_ptr(), lse.data_ptr(), B, Sq, Smax, H,
+                         Hk, D, dt, _scale(softmax_scale, D), 1 if causal else 0,
+                         workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                         _stream_handle(stream, q.device))
+    if st != 0:
+        raise AttnError(st, "attn_decode")
+    return out, lse
 
 
 def get_last_device_error() -> int:

@@ -14,6 +14,7 @@
 
 #include "../../include/attn.h"
 #include "bwd_sm100.cuh"
+#include "decode_sm100.cuh"
 #include "fwd_sm100.cuh"
 
 using namespace attn156;
@@ -78,6 +79,7 @@ attn_status device_state(DeviceState** out) {
         constexpr int D = decltype(d)::value;
         using E = decltype(e);
         ok = ok && set_smem(fwd::attn_fwd_kernel<D, E>, fwd::Cfg<D>::kSmemBytes) == cudaSuccess &&
+             set_smem(dec::attn_decode_kernel<D, E>, dec::Cfg<D>::kSmemBytes) == cudaSuccess &&
              set_smem(bwd::attn_bwd_main_kernel<D, E>, bwd::Cfg<D>::kSmemBytes) == cudaSuccess &&
              regs_of(fwd::attn_fwd_kernel<D, E>) == fwd::kLaunchRegs &&
              regs_of(bwd::attn_bwd_main_kernel<D, E>) == bwd::kLaunchRegs;
@@ -314,6 +316,92 @@ attn_status run_backward(const DeviceState& st, const void* q, const void* k, co
     if (s == ATTN_OK) s = launch_bwd_dq<DD, E>(dq, B, Sq, H, scale, w, cs);
     return s;
   });
+}
+
+// Decode: the key range of each (batch, K/V head) is cut into splits of whole
+// 128-key tiles, one CTA each.  The split length minimises the estimated time
+// ceil(CTAs / SMs) x (tiles per split + 1) (the + 1: a CTA's start-up and
+// pipeline fill), so the last wave of CTAs is not left mostly empty.  Splits
+// have at least two tiles unless the cache has one; the workspace is sized for
+// the largest split count this allows.
+struct DecodePlan {
+  int nsplit, tiles_per_split;
+};
+DecodePlan decode_plan(int B, int Smax, int Hk, int num_sms) {
+  const int tiles = (Smax + dec::BN - 1) / dec::BN;
+  const long long pairs = (long long)B * Hk;
+  DecodePlan best{tiles, 1};
+  long long best_cost = -1;
+  for (int tps = tiles > 1 ? 2 : 1; tps <= tiles; ++tps) {
+    const int nsplit = (tiles + tps - 1) / tps;
+    const long long waves = (pairs * nsplit + num_sms - 1) / num_sms;
+    const long long cost = waves * (tps + 1);
+    if (best_cost < 0 || cost < best_cost) {
+      best_cost = cost;
+      best = {nsplit, tps};
+    }
+  }
+  return best;
+}
+int decode_max_splits(int Smax) {
+  const int tiles = (Smax + dec::BN - 1) / dec::BN;
+  return tiles > 1 ? (tiles + 1) / 2 : 1;
+}
+size_t decode_workspace_bytes(int B, int Sq, int Smax, int H, int Hk, int D) {
+  const size_t rows = size_t(B) * H * Sq * decode_max_splits(Smax);
+  return ((rows * D * 4 + 255) / 256) * 256 + rows * 4;
+}
+
+template <int D, class E>
+attn_status launch_decode(const DeviceState& st, const void* q, const void* kc, const void* vc,
+                          const int* seqlens, void* o, float* lse, int B, int Sq, int Smax,
+                          int H, int Hk, float scale, int causal, void* workspace,
+                          cudaStream_t stream) {
+  constexpr CUtensorMapDataType dt = tmap_type<E>();
+  const int group = H / Hk;
+  alignas(64) CUtensorMap mq, mk, mv;
+  {
+    // the K/V head's query heads at every new position: box (64 d, group heads, Sq rows)
+    const cuuint64_t dims[4] = {cuuint64_t(D), cuuint64_t(H), cuuint64_t(Sq), cuuint64_t(B)};
+    const cuuint64_t strides[3] = {cuuint64_t(D) * 2, cuuint64_t(H) * D * 2,
+                                   cuuint64_t(Sq) * H * D * 2};
+    const cuuint32_t box[4] = {64, cuuint32_t(group), cuuint32_t(Sq), 1};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    if (g_encode(&mq, dt, 4, const_cast<void*>(q), dims, strides, box, estr,
+                 CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                 CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return ATTN_ERR_LAUNCH;
+  }
+  if (make_map(&mk, kc, B, Smax, Hk, D, dt) != ATTN_OK ||
+      make_map(&mv, vc, B, Smax, Hk, D, dt) != ATTN_OK)
+    return ATTN_ERR_LAUNCH;
+  const DecodePlan plan = decode_plan(B, Smax, Hk, st.num_sms > 0 ? st.num_sms : 148);
+  // partial results are laid out for the largest split count (the workspace size)
+  const size_t rows = size_t(B) * H * Sq * decode_max_splits(Smax);
+  dec::Params p;
+  p.seqlens = seqlens;
+  p.opart = static_cast<float*>(workspace);
+  p.lsepart = p.opart + ((rows * D * 4 + 255) / 256) * 256 / 4;
+  p.B = B;
+  p.Sq = Sq;
+  p.Smax = Smax;
+  p.H = H;
+  p.Hk = Hk;
+  p.group = group;
+  p.nsplit = plan.nsplit;
+  p.tiles_per_split = plan.tiles_per_split;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.causal = causal ? 1 : 0;
+  p.err = st.err;
+  p.timeout_ns = kTimeoutNs;
+  dec::attn_decode_kernel<D, E><<<dim3(plan.nsplit, Hk, B), dec::kThreads,
+                                  dec::Cfg<D>::kSmemBytes, stream>>>(mq, mk, mv, p);
+  if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_LAUNCH;
+  const long long nrow = (long long)B * H * Sq;
+  dec::attn_decode_combine_kernel<D, E><<<unsigned((nrow + 7) / 8), 256, 0, stream>>>(
+      p.opart, p.lsepart, static_cast<uint16_t*>(o), lse, B, Sq, H, plan.nsplit);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_LAUNCH;
 }
 
 attn_status check_workspace(const void* workspace, size_t bytes, int B, int Sq, int H, int D) {
@@ -577,6 +665,40 @@ attn_status attn_bwd_noalloc(const void* q, const void* k, const void* v, const 
   return run_backward(*st, q, k, v, o, dout, lse, dq, dk, dv, B, Sq, Sk, H, H, D,
                       ATTN_DTYPE_BF16, scale, causal, win_left, win_right,
                       carve(scratch, B, Sq, H, D), static_cast<cudaStream_t>(stream));
+}
+
+size_t attn_decode_workspace_size(int B, int Sq, int Smax, int H, int Hk, int D) {
+  if (B < 1 || Sq < 1 || Smax < 1 || H < 1 || Hk < 1 || H % Hk || (D != 64 && D != 128))
+    return 0;
+  return decode_workspace_bytes(B, Sq, Smax, H, Hk, D);
+}
+
+attn_status attn_decode(const void* q, const void* k_cache, const void* v_cache,
+                        const int* cache_seqlens, void* o, float* lse, int B, int Sq, int Smax,
+                        int H, int Hk, int D, int dtype, float scale, int causal,
+                        void* workspace, size_t workspace_size, void* stream) {
+  if (!q || !k_cache || !v_cache || !cache_seqlens || !o || !lse) return ATTN_ERR_NULLPTR;
+  attn_status s = check_common(B, Sq, Smax, H, D, scale, -1, -1, Hk);
+  if (s != ATTN_OK) return s;
+  if ((H / Hk) * Sq > dec::BM) return ATTN_ERR_SHAPE;  // the group's rows fill one 128-row tile
+  if ((s = check_dtype(dtype)) != ATTN_OK) return s;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(o) ||
+      (reinterpret_cast<uintptr_t>(lse) & 3u) || (reinterpret_cast<uintptr_t>(cache_seqlens) & 3u))
+    return ATTN_ERR_ALIGN;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) ||
+      workspace_size < decode_workspace_bytes(B, Sq, Smax, H, Hk, D))
+    return ATTN_ERR_WORKSPACE;
+  DeviceState* st = nullptr;
+  s = device_state(&st);
+  if (s != ATTN_OK) return s;
+  if (!all_on_device({q, k_cache, v_cache, cache_seqlens, o, lse, workspace}))
+    return ATTN_ERR_DEVICE;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  return dispatch(D, dtype, [&](auto d, auto e) {
+    return launch_decode<decltype(d)::value, decltype(e)>(*st, q, k_cache, v_cache,
+                                                          cache_seqlens, o, lse, B, Sq, Smax, H,
+                                                          Hk, scale, causal, workspace, cs);
+  });
 }
 
 attn_status attn_get_last_device_error(void) {

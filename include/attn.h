@@ -226,6 +226,33 @@ ATTN_API attn_status attn_bwd_noalloc(const void* q, const void* k, const void* 
                                       void* dv, int B, int Sq, int Sk, int H, int D, float scale,
                                       int causal, int win_left, int win_right, void* stream);
 
+/*
+ * attn_decode - a few new query rows per sequence against a K/V cache (the
+ * pages name flash_attn_with_kvcache as the incremental-inference entry point,
+ * FlashAttention-2 overview, lshu.cn, section 3.3, and give no further
+ * semantics).  Sequence b attends over the first cache_seqlens[b] rows of its
+ * cache (the new keys already appended by the caller); rows past that are
+ * never read into the result, whatever they hold.  Causal uses the same
+ * bottom-right rule: new query i (of Sq) sees keys j <= i + cache_seqlens[b] - Sq.
+ * Grouped K/V heads and dtype as in the _ex entry points.
+ *
+ *   q             [B, Sq, H, D] (in)       k_cache, v_cache [B, Smax, Hk, D] (in)
+ *   cache_seqlens [B] int32, device (in; values clamped to [0, Smax]; a row that
+ *                 sees no key gets O = 0 and LSE = -inf)
+ *   o             [B, Sq, H, D] (out)      lse [B, H, Sq] float32 (out)
+ *   workspace     at least attn_decode_workspace_size(B, Sq, Smax, H, Hk, D) bytes,
+ *                 256-byte aligned (partial results of the key splits).
+ * Limits: (H / Hk) * Sq <= 128 (one K/V head's query rows form one tile).
+ * Errors: as attn_fwd_ex; ATTN_ERR_SHAPE also for (H / Hk) * Sq > 128;
+ * ATTN_ERR_WORKSPACE for a missing, misaligned or small workspace.
+ */
+ATTN_API size_t attn_decode_workspace_size(int B, int Sq, int Smax, int H, int Hk, int D);
+ATTN_API attn_status attn_decode(const void* q, const void* k_cache, const void* v_cache,
+                                 const int* cache_seqlens, void* o, float* lse, int B, int Sq,
+                                 int Smax, int H, int Hk, int D, int dtype, float scale,
+                                 int causal, void* workspace, size_t workspace_bytes,
+                                 void* stream);
+
 /* attn_status_string - static English text for a status code (never NULL). */
 ATTN_API const char* attn_status_string(attn_status s);
 

@@ -151,3 +151,24 @@ def test_binding_checks_key_value_heads():
     for k, v in ((t(1, 8, 3, 64), t(1, 8, 3, 64)), (t(1, 8, 2, 64), t(1, 8, 4, 64))):
         with pytest.raises(ValueError):
             _kv_heads(t(1, 8, 8, 64), k, v)
+
+
+def test_decode_validation():
+    from exact_attention_156_b200 import lib
+    ws = lib.attn_decode_workspace_size(2, 1, 1024, 8, 2, 128)
+    assert ws > 0
+    assert lib.attn_decode_workspace_size(2, 1, 1024, 8, 3, 128) == 0
+    assert lib.attn_decode_workspace_size(2, 1, 1024, 8, 2, 96) == 0
+
+    def dec(Sq=1, H=8, Hk=2, D=128, dtype=0, wsp=0x100000, wsz=ws, seq=0x9000):
+        return lib.attn_decode(0x1000, 0x2000, 0x3000, seq, 0x5000, 0x6000, 2, Sq, 1024, H, Hk,
+                               D, dtype, 0.1, 1, wsp, wsz, None)
+    assert dec(seq=None) == NULLPTR
+    assert dec(Hk=3) == SHAPE
+    assert dec(Sq=33, H=8, Hk=2) == SHAPE     # 4 heads x 33 rows > one 128-row tile
+    assert dec(D=80) == HEADDIM
+    assert dec(dtype=3) == 12
+    assert dec(seq=0x9002) == ALIGN
+    assert dec(wsp=None) == 10
+    assert dec(wsz=ws - 1) == 10
+    assert dec() in (ARCH, DEVICE)

@@ -1,0 +1,42 @@
+"""KV-cache decode (attn_decode): the CUDA path against the float64 oracle's
+attention_decode on the same seeded inputs, with the forward parity bars.
+Cache rows past each sequence's length are filled with NaN and huge values:
+they must not reach the result."""
+import numpy as np
+import pytest
+
+import oracle
+from helpers import check_fwd, f64, to_device, to_f64
+from synth import make_inputs
+
+pytestmark = pytest.mark.gpu
+
+CASES = [
+    # B, Sq, Smax, H, Hk, D, causal, lengths, fmt
+    (2, 1, 1000, 8, 2, 128, 0, (1000, 333), "bf16"),
+    (3, 4, 1024, 4, 4, 64, 1, (7, 513, 1024), "bf16"),
+    (1, 2, 4096, 16, 1, 128, 1, (4000,), "bf16"),          # multi-query, two new rows
+    (2, 1, 8192, 32, 8, 128, 0, (8192, 5000), "f16"),
+    (2, 3, 300, 4, 2, 128, 1, (2, 300), "bf16"),           # a row that sees no key (L < Sq)
+    (3, 1, 640, 8, 8, 64, 0, (0, 129, 640), "bf16"),       # an empty cache, one row past a tile
+]
+
+
+@pytest.mark.parametrize("case", CASES, ids=[str(c) for c in CASES])
+def test_decode_against_the_oracle(case):
+    import torch
+    from exact_attention_156_b200 import attn_decode, get_last_device_error
+    B, Sq, Smax, H, Hk, D, causal, lens, fmt = case
+    bits = make_inputs(B, Sq, Smax, H, D, 5000 + sum(case[:6]), 1.0, Hk=Hk, fmt=fmt)
+    q, k, v = (to_device(bits[n], fmt) for n in ("q", "k", "v"))
+    for b, L in enumerate(lens):          # stale, non-finite cache tail
+        k[b, L:] = float("inf")
+        v[b, L:] = float("nan")
+    seqlens = torch.tensor(lens, dtype=torch.int32, device="cuda")
+    scale = 1.0 / np.sqrt(D)
+    o, lse = attn_decode(q, k, v, seqlens, softmax_scale=scale, causal=bool(causal))
+    torch.cuda.synchronize()
+    assert get_last_device_error() == 0
+    o_ref, lse_ref = oracle.attention_decode(f64(bits["q"], fmt), f64(bits["k"], fmt),
+                                             f64(bits["v"], fmt), lens, scale, causal)
+    check_fwd(to_f64(o), lse.cpu().numpy().astype(np.float64), o_ref, lse_ref, str(case))
