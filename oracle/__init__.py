@@ -10,9 +10,11 @@ from .attn_ref import (  # noqa: F401
     attention_backward_kv_head,
     attention_backward_rows,
     attention_backward_rows_dq,
+    attention_backward_varlen,
     attention_decode,
     attention_forward,
     attention_forward_rows,
+    attention_forward_varlen,
     kv_head,
     online_softmax_forward,
     visible_mask,

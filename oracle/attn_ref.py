@@ -331,6 +331,77 @@ def attention_decode(q, k_cache, v_cache, cache_seqlens, scale: float, causal: i
     return o, lse
 
 
+def _cu_seqlens(cu, total: int, name: str):
+    """Sequence boundaries: cu[0] = 0, non-decreasing, cu[-1] = total."""
+    cu = np.asarray(cu, dtype=np.int64)
+    if cu.ndim != 1 or cu.size < 2 or cu[0] != 0 or cu[-1] != total or np.any(np.diff(cu) < 0):
+        raise ValueError(f"{name} must start at 0, never decrease and end at {total}")
+    return cu
+
+
+def attention_forward_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, scale: float,
+                             causal: int = 0, win_left: int = -1, win_right: int = -1):
+    """O and LSE for a batch of sequences of different lengths packed end to end.
+
+    The pages only name the upstream tests for variable-length and padded
+    batches (FlashAttention-2 overview, lshu.cn, section 3.2).  Reading:
+    q (total_q, H, D) and k, v (total_k, Hk, D) hold the sequences back to
+    back; sequence b is rows cu_seqlens_q[b] .. cu_seqlens_q[b+1]-1 of q and
+    cu_seqlens_k[b] .. cu_seqlens_k[b+1]-1 of k and v, and attends only within
+    itself, with the masks applied to its own lengths (bottom-right causal per
+    sequence).  A sequence with no keys gives its rows O = 0, LSE = -inf.
+    Returns o (total_q, H, D) and lse (H, total_q).
+    """
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    cq = _cu_seqlens(cu_seqlens_q, q.shape[0], "cu_seqlens_q")
+    ck = _cu_seqlens(cu_seqlens_k, k.shape[0], "cu_seqlens_k")
+    if cq.size != ck.size:
+        raise ValueError("cu_seqlens_q and cu_seqlens_k describe different batch sizes")
+    H = q.shape[1]
+    o = np.zeros_like(q)
+    lse = np.full((H, q.shape[0]), -np.inf)
+    for b in range(cq.size - 1):
+        q0, q1, k0, k1 = cq[b], cq[b + 1], ck[b], ck[b + 1]
+        if q1 == q0 or k1 == k0:
+            continue  # no rows, or rows that see no key (O = 0, LSE = -inf)
+        ob, lb = attention_forward(q[None, q0:q1], k[None, k0:k1], v[None, k0:k1], scale,
+                                   causal, win_left, win_right)
+        o[q0:q1] = ob[0]
+        lse[:, q0:q1] = lb[0]
+    return o, lse
+
+
+def attention_backward_varlen(q, k, v, do, cu_seqlens_q, cu_seqlens_k, scale: float,
+                              causal: int = 0, win_left: int = -1, win_right: int = -1):
+    """Gradient of L = sum(O * dO) for packed variable-length sequences (the
+    layout and reading of ``attention_forward_varlen``).  Each sequence's
+    gradient is that of its own attention; sequences never mix.  Returns a dict
+    with o, dq (total_q, H, D), dk, dv (total_k, Hk, D), lse, delta (H, total_q).
+    """
+    q, k, v, do = _f64(q), _f64(k), _f64(v), _f64(do)
+    cq = _cu_seqlens(cu_seqlens_q, q.shape[0], "cu_seqlens_q")
+    ck = _cu_seqlens(cu_seqlens_k, k.shape[0], "cu_seqlens_k")
+    if cq.size != ck.size:
+        raise ValueError("cu_seqlens_q and cu_seqlens_k describe different batch sizes")
+    H = q.shape[1]
+    out = {"o": np.zeros_like(q), "dq": np.zeros_like(q), "dk": np.zeros_like(k),
+           "dv": np.zeros_like(v), "lse": np.full((H, q.shape[0]), -np.inf),
+           "delta": np.zeros((H, q.shape[0]))}
+    for b in range(cq.size - 1):
+        q0, q1, k0, k1 = cq[b], cq[b + 1], ck[b], ck[b + 1]
+        if q1 == q0 or k1 == k0:
+            continue  # nothing visible: zero output and zero gradients
+        r = attention_backward(q[None, q0:q1], k[None, k0:k1], v[None, k0:k1], do[None, q0:q1],
+                               scale, causal, win_left, win_right)
+        out["o"][q0:q1] = r["o"][0]
+        out["dq"][q0:q1] = r["dq"][0]
+        out["dk"][k0:k1] = r["dk"][0]
+        out["dv"][k0:k1] = r["dv"][0]
+        out["lse"][:, q0:q1] = r["lse"][0]
+        out["delta"][:, q0:q1] = r["delta"][0]
+    return out
+
+
 def online_softmax_forward(q, k, v, scale: float, tile: int, causal: int = 0,
                            win_left: int = -1, win_right: int = -1):
     """The pages' online-softmax recurrence, one key tile at a time.
