@@ -5,6 +5,7 @@ recompute-based backward, behind the C ABI of include/attn.h.
     o, lse = attn_fwd(q, k, v, causal=True)              # q, k, v: bf16 (B, S, H, D) CUDA
     dq, dk, dv = attn_bwd(q, k, v, o, do, lse, causal=True)
     o, lse = attn_decode(q_new, k_cache, v_cache, cache_seqlens, causal=True)  # KV-cache decode
+    o, lse = attn_fwd_varlen(q, k, v, cu_q, cu_k, max_q, max_k, causal=True)   # packed batches
 """
 from ._binding import (  # noqa: F401
     ATTN_STATUS,
@@ -12,10 +13,13 @@ from ._binding import (  # noqa: F401
     AttnError,
     attn_bwd,
     attn_bwd_stages,
+    attn_bwd_varlen,
+    attn_bwd_varlen_workspace_size,
     attn_bwd_workspace_size,
     attn_decode,
     attn_decode_workspace_size,
     attn_fwd,
+    attn_fwd_varlen,
     device_timeout_selftest,
     get_last_device_error,
     lib,

@@ -19,7 +19,7 @@ ATTN_STATUS = {
     0: "ATTN_OK", 1: "ATTN_ERR_NULLPTR", 2: "ATTN_ERR_SHAPE", 3: "ATTN_ERR_HEADDIM",
     4: "ATTN_ERR_ALIGN", 5: "ATTN_ERR_WINDOW", 6: "ATTN_ERR_ARCH", 7: "ATTN_ERR_DEVICE",
     8: "ATTN_ERR_LAUNCH", 9: "ATTN_ERR_TIMEOUT", 10: "ATTN_ERR_WORKSPACE",
-    11: "ATTN_ERR_SCRATCH", 12: "ATTN_ERR_DTYPE",
+    11: "ATTN_ERR_SCRATCH", 12: "ATTN_ERR_DTYPE", 13: "ATTN_ERR_SEQLENS",
 }
 ATTN_DTYPE_BF16, ATTN_DTYPE_F16 = 0, 1
 
@@ -65,6 +65,14 @@ def _load() -> ctypes.CDLL:
     lib.attn_decode_workspace_size.restype = sz
     lib.attn_decode.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, f, i, vp, sz, vp]
     lib.attn_decode.restype = i
+    lib.attn_fwd_varlen.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, i, i, f,
+                                    i, i, i, vp]
+    lib.attn_fwd_varlen.restype = i
+    lib.attn_bwd_varlen_workspace_size.argtypes = [i, i, i, i]
+    lib.attn_bwd_varlen_workspace_size.restype = sz
+    lib.attn_bwd_varlen.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i,
+                                    i, i, i, f, i, i, i, vp, sz, vp]
+    lib.attn_bwd_varlen.restype = i
     lib.attn_bwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, i,
                                      i, vp]
     lib.attn_bwd_noalloc.restype = i
@@ -303,8 +311,95 @@ def attn_decode(q, k_cache, v_cache, cache_seqlens, softmax_scale: Optional[floa
     return out, lse
 
 
+def _check_cu(cu, name, B_plus_1=None):
+    import torch
+    _check(cu, name, torch.int32, 1)
+    if cu.numel() < 2 or (B_plus_1 is not None and cu.numel() != B_plus_1):
+        raise ValueError(f"{name} must hold batch + 1 >= 2 boundaries, got {cu.numel()}")
+
+
+def attn_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int, max_seqlen_k: int,
+                    softmax_scale: Optional[float] = None, causal: bool = False,
+                    window_size: Optional[Tuple[int, int]] = None, out=None, lse=None,
+                    stream=None):
+    """Exact attention of a batch of sequences of different lengths packed end
+    to end: q (total_q, H, D), k, v (total_k, Hk, D); sequence b is rows
+    cu_seqlens_q[b]:cu_seqlens_q[b+1] of q and cu_seqlens_k[b]:cu_seqlens_k[b+1]
+    of k and v (int32 CUDA tensors of batch + 1 boundaries).  max_seqlen_q/_k
+    bound the sequence lengths (host ints, as the caller knows them).  Returns
+    (o (total_q, H, D), lse fp32 (H, total_q)).
+    """
+    import torch
+    dt = _dtype_code(q)
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _check(t, n, q.dtype, 3)
+    _check_cu(cu_seqlens_q, "cu_seqlens_q")
+    _check_cu(cu_seqlens_k, "cu_seqlens_k", cu_seqlens_q.numel())
+    total_q, H, D = q.shape
+    total_k, Hk = k.shape[0], k.shape[1]
+    if v.shape[1] != Hk or Hk < 1 or H % Hk != 0:
+        raise ValueError(f"k and v must have the same number of heads, dividing q's {H}")
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((H, total_q), dtype=torch.float32, device=q.device)
+    _check(out, "out", q.dtype, 3)
+    _check(lse, "lse", torch.float32, 2)
+    c, wl, wr = _window(causal, window_size)
+    st = lib.attn_fwd_varlen(q.data_ptr(), k.data_ptr(), v.data_ptr(), cu_seqlens_q.data_ptr(),
+                             cu_seqlens_k.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                             cu_seqlens_q.numel() - 1, total_q, total_k, int(max_seqlen_q),
+                             int(max_seqlen_k), H, Hk, D, dt, _scale(softmax_scale, D), c, wl,
+                             wr, _stream_handle(stream, q.device))
+    if st != 0:
+        raise AttnError(st, "attn_fwd_varlen")
+    return out, lse
+
+
+def attn_bwd_varlen_workspace_size(B: int, total_q: int, H: int, D: int) -> int:
+    return int(lib.attn_bwd_varlen_workspace_size(B, total_q, H, D))
+
+
+def attn_bwd_varlen(q, k, v, out, dout, lse, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int,
+                    max_seqlen_k: int, softmax_scale: Optional[float] = None,
+                    causal: bool = False, window_size: Optional[Tuple[int, int]] = None,
+                    dq=None, dk=None, dv=None, workspace=None, stream=None):
+    """dQ, dK, dV of ``attn_fwd_varlen`` (same packed layout) given its O and
+    LSE and dO.  Returns (dq, dk, dv)."""
+    import torch
+    dt = _dtype_code(q)
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (out, "out"), (dout, "dout")):
+        _check(t, n, q.dtype, 3)
+    _check(lse, "lse", torch.float32, 2)
+    _check_cu(cu_seqlens_q, "cu_seqlens_q")
+    _check_cu(cu_seqlens_k, "cu_seqlens_k", cu_seqlens_q.numel())
+    total_q, H, D = q.shape
+    total_k, Hk = k.shape[0], k.shape[1]
+    if v.shape[1] != Hk or Hk < 1 or H % Hk != 0:
+        raise ValueError(f"k and v must have the same number of heads, dividing q's {H}")
+    B = cu_seqlens_q.numel() - 1
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    if workspace is None:
+        workspace = torch.empty(attn_bwd_varlen_workspace_size(B, total_q, H, D),
+                                dtype=torch.uint8, device=q.device)
+    c, wl, wr = _window(causal, window_size)
+    st = lib.attn_bwd_varlen(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                             dout.data_ptr(), lse.data_ptr(), cu_seqlens_q.data_ptr(),
+                             cu_seqlens_k.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
+                             B, total_q, total_k, int(max_seqlen_q), int(max_seqlen_k), H, Hk, D,
+                             dt, _scale(softmax_scale, D), c, wl, wr, workspace.data_ptr(),
+                             workspace.numel() * workspace.element_size(),
+                             _stream_handle(stream, q.device))
+    if st != 0:
+        raise AttnError(st, "attn_bwd_varlen")
+    return dq, dk, dv
+
+
 def get_last_device_error() -> int:
-    """Synchronises the device; returns the status a timed-out wait recorded (0 if none)."""
+    """Synchronises the device; returns the status a kernel recorded (a timed-out
+    wait, malformed packed-sequence boundaries), 0 if none."""
     return int(lib.attn_get_last_device_error())
 
 

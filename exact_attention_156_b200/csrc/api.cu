@@ -78,11 +78,19 @@ attn_status device_state(DeviceState** out) {
       auto prepare = [&](auto d, auto e) {
         constexpr int D = decltype(d)::value;
         using E = decltype(e);
-        ok = ok && set_smem(fwd::attn_fwd_kernel<D, E>, fwd::Cfg<D>::kSmemBytes) == cudaSuccess &&
-             set_smem(dec::attn_decode_kernel<D, E>, dec::Cfg<D>::kSmemBytes) == cudaSuccess &&
-             set_smem(bwd::attn_bwd_main_kernel<D, E>, bwd::Cfg<D>::kSmemBytes) == cudaSuccess &&
-             regs_of(fwd::attn_fwd_kernel<D, E>) == fwd::kLaunchRegs &&
-             regs_of(bwd::attn_bwd_main_kernel<D, E>) == bwd::kLaunchRegs;
+        auto both = [&](auto v) {
+          constexpr bool kV = decltype(v)::value;
+          ok = ok &&
+               set_smem(fwd::attn_fwd_kernel<D, E, kV>, fwd::Cfg<D>::kSmemBytes) == cudaSuccess &&
+               set_smem(bwd::attn_bwd_main_kernel<D, E, kV>, bwd::Cfg<D>::kSmemBytes) ==
+                   cudaSuccess &&
+               regs_of(fwd::attn_fwd_kernel<D, E, kV>) == fwd::kLaunchRegs &&
+               regs_of(bwd::attn_bwd_main_kernel<D, E, kV>) == bwd::kLaunchRegs;
+        };
+        both(std::false_type{});  // (B, S, H, D) batches
+        both(std::true_type{});   // packed variable-length batches
+        ok = ok &&
+             set_smem(dec::attn_decode_kernel<D, E>, dec::Cfg<D>::kSmemBytes) == cudaSuccess;
       };
       prepare(std::integral_constant<int, 64>{}, ElemBF16{});
       prepare(std::integral_constant<int, 128>{}, ElemBF16{});
@@ -201,11 +209,15 @@ attn_status launch_fwd(const DeviceState& st, const void* q, const void* k, cons
   p.causal = causal ? 1 : 0;
   p.win_left = win_left;
   p.win_right = win_right;
+  p.cu_q = nullptr;
+  p.cu_k = nullptr;
+  p.total_q = 0;
+  p.total_k = 0;
   p.num_mblocks = (Sq + fwd::NQ * fwd::BM - 1) / (fwd::NQ * fwd::BM);
   p.err = st.err;
   p.timeout_ns = kTimeoutNs;
   dim3 grid(p.num_mblocks, H, B);
-  fwd::attn_fwd_kernel<D, E><<<grid, fwd::kThreads, fwd::Cfg<D>::kSmemBytes, stream>>>(mq, mk, mv,
+  fwd::attn_fwd_kernel<D, E, false><<<grid, fwd::kThreads, fwd::Cfg<D>::kSmemBytes, stream>>>(mq, mk, mv,
                                                                                        p);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_LAUNCH;
 }
@@ -261,6 +273,11 @@ attn_status launch_bwd_main(const DeviceState& st, const void* q, const void* k,
   p.Sq = Sq;
   p.Sk = Sk;
   p.Sq_pad = w.Sq_pad;
+  p.cu_q = nullptr;
+  p.cu_k = nullptr;
+  p.total_q = 0;
+  p.total_k = 0;
+  p.R = 0;
   p.Hk = Hk;
   p.scale = scale;
   p.scale_log2 = scale * 1.4426950408889634f;
@@ -270,7 +287,7 @@ attn_status launch_bwd_main(const DeviceState& st, const void* q, const void* k,
   p.err = st.err;
   p.timeout_ns = kTimeoutNs;
   dim3 grid((Sk + bwd::BN - 1) / bwd::BN, Hk, B);
-  bwd::attn_bwd_main_kernel<D, E>
+  bwd::attn_bwd_main_kernel<D, E, false>
       <<<grid, bwd::kThreads, bwd::Cfg<D>::kSmemBytes, stream>>>(mq, mk, mv, mdo, mdq, p);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_LAUNCH;
 }
@@ -316,6 +333,143 @@ attn_status run_backward(const DeviceState& st, const void* q, const void* k, co
     if (s == ATTN_OK) s = launch_bwd_dq<DD, E>(dq, B, Sq, H, scale, w, cs);
     return s;
   });
+}
+
+// ---------------------------------------------------------------------------
+// Packed variable-length batches
+// ---------------------------------------------------------------------------
+struct Varlen {
+  const int* cu_q;  // [B + 1] device
+  const int* cu_k;
+  int total_q, total_k;
+  int max_q, max_k;  // largest sequence lengths (the grid covers these)
+};
+
+// Rows per query head of the varlen row values and dQ accumulator: every
+// sequence's block starts on a multiple of 4 rows and has 128 spare rows
+// (the kernels' rv_start), so total_q + 132 B rows rounded up to 4 suffice.
+long long varlen_rows(int B, int total_q) {
+  return ((long long)total_q + 132ll * B + 3) & ~3ll;
+}
+
+size_t varlen_workspace_bytes(int B, int total_q, int H, int D) {
+  const size_t rows = size_t(H) * size_t(varlen_rows(B, total_q));
+  return rows * D * 4 + rows * 4 * 2;
+}
+
+attn_status check_varlen(int B, int total_q, int total_k, int max_q, int max_k, int H, int Hk,
+                         int D, float scale, int win_left, int win_right) {
+  if (B < 1 || B > 65535 || total_q < 1 || total_k < 1 || H < 1 || H > 65535)
+    return ATTN_ERR_SHAPE;
+  if (max_q < 1 || max_k < 1 || max_q > total_q || max_k > total_k) return ATTN_ERR_SHAPE;
+  if (Hk < 1 || Hk > H || H % Hk != 0) return ATTN_ERR_SHAPE;
+  if (D != 64 && D != 128) return ATTN_ERR_HEADDIM;
+  if ((long long)total_q * H * D >= (1ll << 31) || (long long)total_k * Hk * D >= (1ll << 31) ||
+      varlen_rows(B, total_q) * H * D >= (1ll << 31))
+    return ATTN_ERR_SHAPE;
+  if (!(scale > 0.f) || !isfinite(scale)) return ATTN_ERR_SHAPE;
+  if (win_left < -1 || win_right < -1) return ATTN_ERR_WINDOW;
+  return ATTN_OK;
+}
+
+bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+
+template <int D, class E>
+attn_status launch_fwd_varlen(const DeviceState& st, const void* q, const void* k, const void* v,
+                              void* o, float* lse, const Varlen& vl, int B, int H, int Hk,
+                              float scale, int causal, int win_left, int win_right,
+                              cudaStream_t stream) {
+  constexpr CUtensorMapDataType dt = tmap_type<E>();
+  alignas(64) CUtensorMap mq, mk, mv;
+  if (make_map(&mq, q, 1, vl.total_q, H, D, dt) != ATTN_OK ||
+      make_map(&mk, k, 1, vl.total_k, Hk, D, dt) != ATTN_OK ||
+      make_map(&mv, v, 1, vl.total_k, Hk, D, dt) != ATTN_OK)
+    return ATTN_ERR_LAUNCH;
+  fwd::Params p;
+  p.o = static_cast<uint16_t*>(o);
+  p.lse = lse;
+  p.B = B;
+  p.H = H;
+  p.Hk = Hk;
+  p.Sq = vl.max_q;
+  p.Sk = vl.max_k;
+  p.cu_q = vl.cu_q;
+  p.cu_k = vl.cu_k;
+  p.total_q = vl.total_q;
+  p.total_k = vl.total_k;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.causal = causal ? 1 : 0;
+  p.win_left = win_left;
+  p.win_right = win_right;
+  p.num_mblocks = (vl.max_q + fwd::NQ * fwd::BM - 1) / (fwd::NQ * fwd::BM);
+  p.err = st.err;
+  p.timeout_ns = kTimeoutNs;
+  dim3 grid(p.num_mblocks, H, B);
+  fwd::attn_fwd_kernel<D, E, true><<<grid, fwd::kThreads, fwd::Cfg<D>::kSmemBytes, stream>>>(mq, mk, mv,
+                                                                                       p);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_LAUNCH;
+}
+
+template <int D, class E>
+attn_status run_backward_varlen(const DeviceState& st, const void* q, const void* k,
+                                const void* v, const void* o, const void* dout, const float* lse,
+                                void* dq, void* dk, void* dv, const Varlen& vl, int B, int H,
+                                int Hk, float scale, int causal, int win_left, int win_right,
+                                void* workspace, cudaStream_t stream) {
+  constexpr CUtensorMapDataType dt = tmap_type<E>();
+  const long long R = varlen_rows(B, vl.total_q);
+  const size_t rows = size_t(H) * size_t(R);
+  float* dq_acc = static_cast<float*>(workspace);
+  float* nlse2 = dq_acc + rows * D;
+  float* ndelta = nlse2 + rows;
+  {
+    const unsigned blocks = unsigned((rows + 7) / 8);
+    bwd::attn_bwd_pre_varlen_kernel<D, E><<<blocks, 256, 0, stream>>>(
+        static_cast<const uint16_t*>(o), static_cast<const uint16_t*>(dout), lse, nlse2, ndelta,
+        dq_acc, vl.cu_q, vl.cu_k, B, H, vl.total_q, vl.total_k, vl.max_q, vl.max_k, int(R),
+        st.err);
+    if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_LAUNCH;
+  }
+  alignas(64) CUtensorMap mq, mk, mv, mdo, mdq;
+  if (make_map(&mq, q, 1, vl.total_q, H, D, dt) != ATTN_OK ||
+      make_map(&mk, k, 1, vl.total_k, Hk, D, dt) != ATTN_OK ||
+      make_map(&mv, v, 1, vl.total_k, Hk, D, dt) != ATTN_OK ||
+      make_map(&mdo, dout, 1, vl.total_q, H, D, dt) != ATTN_OK ||
+      make_dq_map(&mdq, dq_acc, (long long)rows, D) != ATTN_OK)
+    return ATTN_ERR_LAUNCH;
+  bwd::Params p;
+  p.dk = static_cast<uint16_t*>(dk);
+  p.dv = static_cast<uint16_t*>(dv);
+  p.nlse2 = nlse2;
+  p.ndelta = ndelta;
+  p.dq_acc = dq_acc;
+  p.B = B;
+  p.H = H;
+  p.Sq = vl.max_q;
+  p.Sk = vl.max_k;
+  p.Sq_pad = 0;
+  p.cu_q = vl.cu_q;
+  p.cu_k = vl.cu_k;
+  p.total_q = vl.total_q;
+  p.total_k = vl.total_k;
+  p.R = int(R);
+  p.Hk = Hk;
+  p.scale = scale;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.causal = causal ? 1 : 0;
+  p.win_left = win_left;
+  p.win_right = win_right;
+  p.err = st.err;
+  p.timeout_ns = kTimeoutNs;
+  dim3 grid((vl.max_k + bwd::BN - 1) / bwd::BN, Hk, B);
+  bwd::attn_bwd_main_kernel<D, E, true>
+      <<<grid, bwd::kThreads, bwd::Cfg<D>::kSmemBytes, stream>>>(mq, mk, mv, mdo, mdq, p);
+  if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_LAUNCH;
+  const long long total = (long long)vl.total_q * H * (D / 8);
+  bwd::attn_bwd_dq_varlen_kernel<D, E><<<unsigned((total + 255) / 256), 256, 0, stream>>>(
+      dq_acc, static_cast<uint16_t*>(dq), vl.cu_q, vl.cu_k, B, H, vl.total_q, vl.total_k,
+      vl.max_q, vl.max_k, int(R), scale);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_LAUNCH;
 }
 
 // Decode: the key range of each (batch, K/V head) is cut into splits of whole
@@ -482,6 +636,9 @@ const char* attn_status_string(attn_status s) {
       return "backward scratch for this problem exceeds the 64 MiB built into attn_bwd_noalloc "
              "(call attn_bwd with a workspace instead)";
     case ATTN_ERR_DTYPE: return "dtype must be ATTN_DTYPE_BF16 (0) or ATTN_DTYPE_F16 (1)";
+    case ATTN_ERR_SEQLENS:
+      return "cu_seqlens found malformed on the device (not 0 <= cu[b] <= cu[b+1] <= total, or "
+             "a sequence longer than its max_seqlen); the malformed sequences were skipped";
   }
   return "unknown status";
 }
@@ -549,6 +706,72 @@ attn_status attn_bwd(const void* q, const void* k, const void* v, const void* o,
                      size_t workspace_size, void* stream) {
   return attn_bwd_ex(q, k, v, o, dout, lse, dq, dk, dv, B, Sq, Sk, H, H, D, ATTN_DTYPE_BF16,
                      scale, causal, win_left, win_right, workspace, workspace_size, stream);
+}
+
+attn_status attn_fwd_varlen(const void* q, const void* k, const void* v,
+                            const int* cu_seqlens_q, const int* cu_seqlens_k, void* o, float* lse,
+                            int B, int total_q, int total_k, int max_seqlen_q, int max_seqlen_k,
+                            int H, int Hk, int D, int dtype, float scale, int causal,
+                            int win_left, int win_right, void* stream) {
+  if (!q || !k || !v || !cu_seqlens_q || !cu_seqlens_k || !o || !lse) return ATTN_ERR_NULLPTR;
+  attn_status s = check_varlen(B, total_q, total_k, max_seqlen_q, max_seqlen_k, H, Hk, D, scale,
+                               win_left, win_right);
+  if (s != ATTN_OK) return s;
+  if ((s = check_dtype(dtype)) != ATTN_OK) return s;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned4(lse) ||
+      !aligned4(cu_seqlens_q) || !aligned4(cu_seqlens_k))
+    return ATTN_ERR_ALIGN;
+  DeviceState* st = nullptr;
+  s = device_state(&st);
+  if (s != ATTN_OK) return s;
+  if (!all_on_device({q, k, v, o, lse, cu_seqlens_q, cu_seqlens_k})) return ATTN_ERR_DEVICE;
+  const Varlen vl{cu_seqlens_q, cu_seqlens_k, total_q, total_k, max_seqlen_q, max_seqlen_k};
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  return dispatch(D, dtype, [&](auto d, auto e) {
+    return launch_fwd_varlen<decltype(d)::value, decltype(e)>(*st, q, k, v, o, lse, vl, B, H, Hk,
+                                                              scale, causal, win_left, win_right,
+                                                              cs);
+  });
+}
+
+size_t attn_bwd_varlen_workspace_size(int B, int total_q, int H, int D) {
+  if (B < 1 || total_q < 1 || H < 1 || (D != 64 && D != 128)) return 0;
+  return varlen_workspace_bytes(B, total_q, H, D);
+}
+
+attn_status attn_bwd_varlen(const void* q, const void* k, const void* v, const void* o,
+                            const void* dout, const float* lse, const int* cu_seqlens_q,
+                            const int* cu_seqlens_k, void* dq, void* dk, void* dv, int B,
+                            int total_q, int total_k, int max_seqlen_q, int max_seqlen_k, int H,
+                            int Hk, int D, int dtype, float scale, int causal, int win_left,
+                            int win_right, void* workspace, size_t workspace_size,
+                            void* stream) {
+  if (!q || !k || !v || !o || !dout || !lse || !cu_seqlens_q || !cu_seqlens_k || !dq || !dk ||
+      !dv)
+    return ATTN_ERR_NULLPTR;
+  attn_status s = check_varlen(B, total_q, total_k, max_seqlen_q, max_seqlen_k, H, Hk, D, scale,
+                               win_left, win_right);
+  if (s != ATTN_OK) return s;
+  if ((s = check_dtype(dtype)) != ATTN_OK) return s;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) ||
+      !aligned16(dq) || !aligned16(dk) || !aligned16(dv) || !aligned4(lse) ||
+      !aligned4(cu_seqlens_q) || !aligned4(cu_seqlens_k))
+    return ATTN_ERR_ALIGN;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) ||
+      workspace_size < varlen_workspace_bytes(B, total_q, H, D))
+    return ATTN_ERR_WORKSPACE;
+  DeviceState* st = nullptr;
+  s = device_state(&st);
+  if (s != ATTN_OK) return s;
+  if (!all_on_device({q, k, v, o, dout, lse, cu_seqlens_q, cu_seqlens_k, dq, dk, dv, workspace}))
+    return ATTN_ERR_DEVICE;
+  const Varlen vl{cu_seqlens_q, cu_seqlens_k, total_q, total_k, max_seqlen_q, max_seqlen_k};
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  return dispatch(D, dtype, [&](auto d, auto e) {
+    return run_backward_varlen<decltype(d)::value, decltype(e)>(
+        *st, q, k, v, o, dout, lse, dq, dk, dv, vl, B, H, Hk, scale, causal, win_left, win_right,
+        workspace, cs);
+  });
 }
 
 attn_status attn_bwd_preprocess_ex(const void* o, const void* dout, const float* lse, int B,
@@ -711,7 +934,9 @@ attn_status attn_get_last_device_error(void) {
   if (word == 0) return ATTN_OK;
   const uint32_t zero = 0;
   cudaMemcpyToSymbol(g_attn_err, &zero, sizeof(zero));
-  return (word & 0xFFu) == kErrTimeout ? ATTN_ERR_TIMEOUT : ATTN_ERR_LAUNCH;
+  if ((word & 0xFFu) == kErrTimeout) return ATTN_ERR_TIMEOUT;
+  if ((word & 0xFFu) == kErrSeqlens) return ATTN_ERR_SEQLENS;
+  return ATTN_ERR_LAUNCH;
 }
 
 attn_status attn_device_timeout_selftest(int limit_us, void* stream) {

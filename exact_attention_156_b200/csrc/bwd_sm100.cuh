@@ -109,7 +109,15 @@ struct Params {
   const float* nlse2;   // [B*H][Sq_pad] -LSE * log2(e); -inf for padding rows
   const float* ndelta;  // [B*H][Sq_pad] -Delta
   float* dq_acc;       // [B*H][Sq_pad][D]
-  int B, H, Sq, Sk, Sq_pad;
+  int B, H, Sq, Sk, Sq_pad;  // packed sequences: Sq, Sk are the largest lengths
+  // Packed variable-length sequences (null for the (B, S, H, D) layout): sequence
+  // b is rows cu_q[b] .. cu_q[b+1]-1 of Q/dO and cu_k[b] .. cu_k[b+1]-1 of K/V.
+  // The row values and the dQ accumulator then hold, per query head, R rows
+  // (varlen_rows): query i of sequence b is row rv_start(cu_q, b) + i, each
+  // sequence starting on a 16-byte boundary and followed by >= 128 padding rows.
+  const int* cu_q;
+  const int* cu_k;
+  int total_q, total_k, R;
   int Hk;  // key/value heads: the CTA's K/V head is shared by H / Hk query heads
   float scale;
   float scale_log2;
@@ -203,6 +211,121 @@ __global__ void __launch_bounds__(256) attn_bwd_dq_kernel(const float* __restric
 }
 
 // ---------------------------------------------------------------------------
+// Packed variable-length batches: the preprocess and the dQ finalize.
+// ---------------------------------------------------------------------------
+// First row of sequence b in the per-head row-value / dQ-accumulator layout
+// of packed batches: cu[b] + 132 b rounded up to a multiple of 4 (16 bytes of
+// fp32, the alignment of the bulk copies that read the row values).  Sequence
+// b's block then has at least Lq_b + 128 rows before sequence b + 1 starts, so
+// a ragged query tile never reaches another sequence's rows.
+constexpr int kRvGap = BM + 4;
+__device__ __forceinline__ long long rv_start(const int* cu, int b) {
+  return ((long long)cu[b] + (long long)kRvGap * b + 3) & ~3ll;
+}
+
+// Largest b in [0, B) with key(b) <= x for a key non-decreasing in b (true
+// for valid boundaries); callers re-check the sequence, so malformed
+// boundaries cannot steer an access.
+template <class KeyFn>
+__device__ __forceinline__ int find_seq(int B, long long x, KeyFn key) {
+  int lo = 0, hi = B - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) / 2;
+    if (key(mid) <= x)
+      lo = mid;
+    else
+      hi = mid - 1;
+  }
+  return lo;
+}
+
+// One warp per row of the [H][R] row-value layout: Delta and -LSE*log2(e) of
+// query rows, neutral values (P = 0) for the padding rows, dQ accumulator zeroed.
+template <int D, class E>
+__global__ void __launch_bounds__(256) attn_bwd_pre_varlen_kernel(
+    const uint16_t* __restrict__ o, const uint16_t* __restrict__ dout,
+    const float* __restrict__ lse, float* __restrict__ nlse2, float* __restrict__ ndelta,
+    float* __restrict__ dq_acc, const int* __restrict__ cu_q, const int* __restrict__ cu_k, int B,
+    int H, int total_q, int total_k, int max_q, int max_k, int R, uint32_t* err) {
+  const long long gw = (long long)blockIdx.x * 8 + threadIdx.x / 32;
+  const int lane = threadIdx.x % 32;
+  if (gw >= (long long)H * R) return;
+  const int h = int(gw / R);
+  const long long y = gw % R;
+  const int b = find_seq(B, y, [&](int c) { return rv_start(cu_q, c); });
+  const SeqSpan sp = seq_span(cu_q, cu_k, b, total_q, total_k, max_q, max_k);
+  if (!sp.ok && lane == 0 && h == 0) atomicCAS(err, 0u, kErrSeqlens);
+  const long long i = y - rv_start(cu_q, b);  // query index in the sequence
+  const bool real = sp.ok && i >= 0 && i < sp.Lq;
+  float dot = 0.f;
+  if (real) {
+    const size_t base = ((size_t(sp.q0) + size_t(i)) * H + h) * D;
+    constexpr int kPer = D / 32;
+    uint32_t ow[kPer / 2], dw[kPer / 2];
+    if constexpr (kPer == 4) {
+      const uint2 ov = *reinterpret_cast<const uint2*>(o + base + lane * 4);
+      const uint2 dv = *reinterpret_cast<const uint2*>(dout + base + lane * 4);
+      ow[0] = ov.x; ow[1] = ov.y;
+      dw[0] = dv.x; dw[1] = dv.y;
+    } else {
+      ow[0] = *reinterpret_cast<const uint32_t*>(o + base + lane * 2);
+      dw[0] = *reinterpret_cast<const uint32_t*>(dout + base + lane * 2);
+    }
+#pragma unroll
+    for (int t = 0; t < kPer / 2; ++t) {
+      float a0, a1, c0, c1;
+      E::unpack2(ow[t], a0, a1);
+      E::unpack2(dw[t], c0, c1);
+      dot = fmaf(a0, c0, dot);
+      dot = fmaf(a1, c1, dot);
+    }
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, off);
+  if (lane == 0) {
+    float nl2 = -INFINITY;
+    if (real) {
+      const float l = lse[size_t(h) * total_q + size_t(sp.q0) + size_t(i)];
+      if (l != -INFINITY) nl2 = -l * 1.4426950408889634f;
+    }
+    nlse2[gw] = nl2;
+    ndelta[gw] = -dot;
+  }
+  float4* acc = reinterpret_cast<float4*>(dq_acc + size_t(gw) * D);
+  for (int c = lane; c < D / 4; c += 32) acc[c] = make_float4(0.f, 0.f, 0.f, 0.f);
+}
+
+// dq[x, h, :] = 16-bit(scale * acc[h][rv_start(b) + i]) for packed row x =
+// cu_q[b] + i; 8 elements per thread.
+template <int D, class E>
+__global__ void __launch_bounds__(256) attn_bwd_dq_varlen_kernel(
+    const float* __restrict__ dq_acc, uint16_t* __restrict__ dq, const int* __restrict__ cu_q,
+    const int* __restrict__ cu_k, int B, int H, int total_q, int total_k, int max_q, int max_k,
+    int R, float scale) {
+  const long long t = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  constexpr int kVec = D / 8;
+  if (t >= (long long)total_q * H * kVec) return;
+  const int v = int(t % kVec);
+  const long long r = t / kVec;  // (x, h) in packed (row, head) order
+  const int h = int(r % H);
+  const long long x = r / H;
+  const int b = find_seq(B, x, [&](int c) { return (long long)cu_q[c]; });
+  const SeqSpan sp = seq_span(cu_q, cu_k, b, total_q, total_k, max_q, max_k);
+  // rows of malformed sequences are left untouched
+  if (!sp.ok || x < sp.q0 || x >= (long long)sp.q0 + sp.Lq) return;
+  const float4* src = reinterpret_cast<const float4*>(
+      dq_acc + (size_t(h) * R + size_t(rv_start(cu_q, b) + (x - sp.q0))) * D + v * 8);
+  const float4 a = src[0];
+  const float4 c = src[1];
+  uint4 w;
+  w.x = E::pack2(a.x * scale, a.y * scale);
+  w.y = E::pack2(a.z * scale, a.w * scale);
+  w.z = E::pack2(c.x * scale, c.y * scale);
+  w.w = E::pack2(c.z * scale, c.w * scale);
+  *reinterpret_cast<uint4*>(dq + (size_t(x) * H + h) * D + v * 8) = w;
+}
+
+// ---------------------------------------------------------------------------
 // 2. main backward kernel
 // ---------------------------------------------------------------------------
 // Query-tile range [qlo, qhi) that can see keys [n0, n1]; empty if qhi <= qlo.
@@ -219,7 +342,7 @@ __device__ __forceinline__ void qtile_range(const MaskGeom& g, int n0, int n1, i
 }
 
 // E: element format of Q, K, V, dO, P, dS and the gradients (ElemBF16 or ElemF16).
-template <int D, class E>
+template <int D, class E, bool kVarlen>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ,
                          const __grid_constant__ CUtensorMap tmK,
@@ -244,9 +367,24 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int hk = blockIdx.y;  // key/value head
   const int b = blockIdx.z;
   const int group = p.H / p.Hk;  // query heads sharing this K/V head
-  const MaskGeom g = MaskGeom::make(p.Sq, p.Sk, p.causal, p.win_left, p.win_right);
+  // This sequence's lengths, first rows, TMA batch coordinate and row-value base.
+  int Lq = p.Sq, Lk = p.Sk, q_row0 = 0, k_row0 = 0, bc = b;
+  if constexpr (kVarlen) {
+    const SeqSpan sp = seq_span(p.cu_q, p.cu_k, b, p.total_q, p.total_k, p.Sq, p.Sk);
+    if (!sp.ok && threadIdx.x == 0) atomicCAS(p.err, 0u, kErrSeqlens);
+    Lq = sp.Lq;  // 0 for a malformed sequence: nothing is read or written
+    Lk = sp.Lk;
+    q_row0 = sp.q0;
+    k_row0 = sp.k0;
+    bc = 0;
+  }
+  // first row of query head h's row values / dQ accumulator rows
+  auto rv_base = [&](int h) -> long long {
+    return kVarlen ? (long long)h * p.R + rv_start(p.cu_q, b) : ((long long)b * p.H + h) * p.Sq_pad;
+  };
+  const MaskGeom g = MaskGeom::make(Lq, Lk, p.causal, p.win_left, p.win_right);
   const int n0 = kt * BN;
-  const int n1 = min(n0 + BN - 1, p.Sk - 1);
+  const int n1 = min(n0 + BN - 1, Lk - 1);
   int qlo, qhi;
   qtile_range(g, n0, n1, qlo, qhi);
   const int nq_head = qhi - qlo;  // query tiles per query head
@@ -328,8 +466,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tDP = tmem + lane_off + C::kColDP;
     const uint64_t sl2 = f2_pack(p.scale_log2, p.scale_log2);
     const int qmin_k = g.qmin(kk_idx);
-    const int qmax_k = min(g.qmax(kk_idx), p.Sq - 1);
-    const bool key_ok = kk_idx < p.Sk;
+    const int qmax_k = min(g.qmax(kk_idx), Lq - 1);
+    const bool key_ok = kk_idx < Lk;
     // rows of the dS^T buffer: 128 bytes per 64 columns, 16-byte chunks swizzled by row % 8
     const uint32_t ds_row = ds_addr + uint32_t(r) * 128;
     const uint32_t sw = uint32_t(r & 7);
@@ -346,7 +484,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       {
         uint32_t rr[BM];
         tmem_ld128(tS, rr);
-        const bool full = key_ok && n0 + BN - 1 <= p.Sk - 1 && i0 + BM - 1 <= p.Sq - 1 &&
+        const bool full = key_ok && n0 + BN - 1 <= Lk - 1 && i0 + BM - 1 <= Lq - 1 &&
                           i0 >= g.qmin(n0 + BN - 1) && i0 + BM - 1 <= g.qmax(n0);
         if (full) {
           // every entry visible: a quarter of the exponentials on the FMA pipe
@@ -434,7 +572,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (ok && nq > 0) ok = bw.wait_warp(bar(C::kBarDSEmpty), (nq - 1) & 1, 30);
     if (ok) {
       tc_fence_after();
-      const size_t orow = ((size_t(b) * p.Sk + size_t(kk_idx)) * p.Hk + hk) * D;
+      const size_t orow =
+          ((kVarlen ? size_t(k_row0) + kk_idx : size_t(b) * p.Sk + size_t(kk_idx)) * p.Hk + hk) * D;
 #pragma unroll 1
       for (int which = 0; which < 2; ++which) {
         const uint32_t col = which == 0 ? C::kColDK : C::kColDV;
@@ -491,7 +630,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // tensor memory is free again: the MMA warp may start dP of the next tile
       tc_fence_before();
       mbar_arrive(bar(C::kBarDQEmpty));
-      const int row0 = (b * p.H + item_head(t)) * p.Sq_pad + item_row0(t);
+      const int row0 = int(rv_base(item_head(t)) + item_row0(t));
 #pragma unroll
       for (int c = 0; c < C::kDQChunks; ++c, ++n) {
         const uint32_t buf = sbase + C::kDQOff + uint32_t(n & 1) * C::kDQBufBytes;
@@ -525,8 +664,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_prefetch_desc(&tmV);
       mbar_arrive_expect_tx(bar(C::kBarKV), 2 * C::kTileBytes);
       for (int x = 0; x < C::kBoxes; ++x) {
-        tma_load_4d(k_addr + x * C::kBoxBytes, &tmK, bar(C::kBarKV), x * 64, hk, n0, b);
-        tma_load_4d(v_addr + x * C::kBoxBytes, &tmV, bar(C::kBarKV), x * 64, hk, n0, b);
+        tma_load_4d(k_addr + x * C::kBoxBytes, &tmK, bar(C::kBarKV), x * 64, hk, k_row0 + n0, bc);
+        tma_load_4d(v_addr + x * C::kBoxBytes, &tmV, bar(C::kBarKV), x * 64, hk, k_row0 + n0, bc);
       }
       for (int t = 0; t < nq; ++t) {
         const int s = t % kQStages;
@@ -537,8 +676,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t fb = bar(C::kBarQFull + s);
         mbar_arrive_expect_tx(fb, C::kTileBytes + 2 * BM * 4);
         for (int x = 0; x < C::kBoxes; ++x)
-          tma_load_4d(q_addr(s) + x * C::kBoxBytes, &tmQ, fb, x * 64, h, i0, b);
-        const size_t roff = size_t(b * p.H + h) * p.Sq_pad + i0;
+          tma_load_4d(q_addr(s) + x * C::kBoxBytes, &tmQ, fb, x * 64, h, q_row0 + i0, bc);
+        const size_t roff = size_t(rv_base(h) + i0);
         bulk_load(sbase + C::kLseOff + s * BM * 4, p.nlse2 + roff, BM * 4, fb);
         bulk_load(sbase + C::kDeltaOff + s * BM * 4, p.ndelta + roff, BM * 4, fb);
         if (s == 0) ++q_loads0; else ++q_loads1;
@@ -554,7 +693,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive_expect_tx(bar(C::kBarDOFull), C::kTileBytes);
         for (int x = 0; x < C::kBoxes; ++x)
           tma_load_4d(do_addr + x * C::kBoxBytes, &tmDO, bar(C::kBarDOFull), x * 64, item_head(t),
-                      i0, b);
+                      q_row0 + i0, bc);
         do_loads++;
       }
     }

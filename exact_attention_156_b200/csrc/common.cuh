@@ -1,4 +1,4 @@
-// common.cuh - mask geometry shared by the forward and backward kernels.
+// common.cuh - mask geometry and packed-sequence spans shared by the kernels.
 #pragma once
 
 #include <stdint.h>
@@ -46,5 +46,31 @@ struct MaskGeom {
   __host__ __device__ int qmin(int j) const { return j - delta - right; }
   __host__ __device__ int qmax(int j) const { return j - delta + left; }
 };
+
+// Device error word code for malformed packed-sequence boundaries.
+constexpr uint32_t kErrSeqlens = 13u;
+
+// One sequence of a packed variable-length batch: its first query and key
+// rows and its lengths.  `ok` is false (and the lengths 0, so that nothing is
+// read or written) unless 0 <= cu_q[b] <= cu_q[b+1] <= total_q with length at
+// most max_q, and the same for the keys.
+struct SeqSpan {
+  int q0, k0, Lq, Lk;
+  bool ok;
+};
+__device__ __forceinline__ SeqSpan seq_span(const int* cu_q, const int* cu_k, int b, int total_q,
+                                            int total_k, int max_q, int max_k) {
+  const int a0 = cu_q[b], a1 = cu_q[b + 1], c0 = cu_k[b], c1 = cu_k[b + 1];
+  SeqSpan s{0, 0, 0, 0, false};
+  if (a0 < 0 || a1 < a0 || a1 > total_q || a1 - a0 > max_q || c0 < 0 || c1 < c0 ||
+      c1 > total_k || c1 - c0 > max_k)
+    return s;
+  s.q0 = a0;
+  s.k0 = c0;
+  s.Lq = a1 - a0;
+  s.Lk = c1 - c0;
+  s.ok = true;
+  return s;
+}
 
 }  // namespace attn156

@@ -81,7 +81,13 @@ struct Cfg {
 struct Params {
   uint16_t* o;  // 16-bit elements (bf16 or f16, as the kernel's element format)
   float* lse;
-  int B, H, Sq, Sk;
+  int B, H, Sq, Sk;  // packed sequences: Sq, Sk are the largest lengths
+  // Packed variable-length sequences (null for the (B, S, H, D) layout):
+  // sequence b is rows cu_q[b] .. cu_q[b+1]-1 of Q/O and cu_k[b] .. cu_k[b+1]-1
+  // of K/V, of total_q / total_k rows; LSE is then (H, total_q).
+  const int* cu_q;
+  const int* cu_k;
+  int total_q, total_k;
   int Hk;            // key/value heads (H a multiple of Hk; query head h reads h / (H / Hk))
   float scale_log2;  // scale * log2(e)
   int causal, win_left, win_right;
@@ -104,7 +110,7 @@ __device__ __forceinline__ void tile_range(const MaskGeom& g, int r0, int r1, in
 }
 
 // E: element format of Q, K, V, P and O (ElemBF16 or ElemF16).
-template <int D, class E>
+template <int D, class E, bool kVarlen>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const Params p) {
@@ -129,7 +135,18 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int h = blockIdx.y;
   const int hk = h / (p.H / p.Hk);  // the key/value head this query head reads
   const int b = blockIdx.z;
-  const MaskGeom g = MaskGeom::make(p.Sq, p.Sk, p.causal, p.win_left, p.win_right);
+  // This sequence's lengths, first rows and TMA batch coordinate.
+  int Lq = p.Sq, Lk = p.Sk, q_row0 = 0, k_row0 = 0, bc = b;
+  if constexpr (kVarlen) {
+    const SeqSpan sp = seq_span(p.cu_q, p.cu_k, b, p.total_q, p.total_k, p.Sq, p.Sk);
+    if (!sp.ok && threadIdx.x == 0) atomicCAS(p.err, 0u, kErrSeqlens);
+    Lq = sp.Lq;  // 0 for a malformed sequence: nothing is read or written
+    Lk = sp.Lk;
+    q_row0 = sp.q0;
+    k_row0 = sp.k0;
+    bc = 0;
+  }
+  const MaskGeom g = MaskGeom::make(Lq, Lk, p.causal, p.win_left, p.win_right);
 
   int r0[NQ], jlo[NQ], jhi[NQ];
   bool valid[NQ];
@@ -137,8 +154,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
   for (int k = 0; k < NQ; ++k) {
     r0[k] = (mb * NQ + k) * BM;
-    valid[k] = r0[k] < p.Sq;
-    const int r1 = min(r0[k] + BM - 1, p.Sq - 1);
+    valid[k] = r0[k] < Lq;
+    const int r1 = min(r0[k] + BM - 1, Lq - 1);
     tile_range(g, r0[k], r1, jlo[k], jhi[k]);
     if (jhi[k] > jlo[k]) {
       ju_lo = min(ju_lo, jlo[k]);
@@ -223,7 +240,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tO = tmem + lane_off + C::col_o(k);
     const int lo_i = g.lo(i);
     const int hi_i = g.hi(i);
-    const int r1 = min(r0[k] + BM - 1, p.Sq - 1);
+    const int r1 = min(r0[k] + BM - 1, Lq - 1);
     const int tile_lo_max = g.lo(r1);  // largest row lower bound in this tile
     const int tile_hi_min = g.hi(r0[k]);
     const float sl2 = p.scale_log2;
@@ -334,8 +351,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     // Epilogue: O = O / l (input format), LSE = (m + log2 l) ln 2.
     if (valid[k] && ok) {
-      const bool row_ok = i < p.Sq;
-      const size_t orow = ((size_t(b) * p.Sq + size_t(i)) * p.H + h) * D;
+      const bool row_ok = i < Lq;
+      const size_t orow =
+          ((kVarlen ? size_t(q_row0) + i : size_t(b) * p.Sq + size_t(i)) * p.H + h) * D;
       if (n_k > 0) {
         ok = bw.wait_warp(bar(C::kBarO + k), (n_k - 1) & 1, 14 + k);
       }
@@ -364,7 +382,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (row_ok) {
           const float lse = l_run > 0.f ? (m_run + __log2f(l_run)) * 0.69314718055994530942f : -INFINITY;
-          p.lse[(size_t(b) * p.H + h) * p.Sq + i] = lse;
+          const size_t lrow = kVarlen ? size_t(h) * p.total_q + q_row0 + i
+                                     : (size_t(b) * p.H + h) * p.Sq + i;
+          p.lse[lrow] = lse;
         }
       }
     }
@@ -385,7 +405,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int k = 0; k < NQ; ++k) {
         if (!(valid[k] && jhi[k] > jlo[k])) continue;
         for (int x = 0; x < C::kBoxes; ++x)
-          tma_load_4d(q_addr(k) + x * C::kBoxBytes, &tmQ, bar(C::kBarQ), x * 64, h, r0[k], b);
+          tma_load_4d(q_addr(k) + x * C::kBoxBytes, &tmQ, bar(C::kBarQ), x * 64, h,
+                      q_row0 + r0[k], bc);
       }
       const int nloads = 2 * (ju_hi - ju_lo);
       for (int L = 0; L < nloads; ++L) {
@@ -396,8 +417,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const void* map = (L & 1) ? static_cast<const void*>(&tmV) : static_cast<const void*>(&tmK);
         mbar_arrive_expect_tx(bar(C::kBarFull + s), C::kTileBytes);
         for (int x = 0; x < C::kBoxes; ++x)
-          tma_load_4d(kv_addr(s) + x * C::kBoxBytes, map, bar(C::kBarFull + s), x * 64, hk, j * BN,
-                      b);
+          tma_load_4d(kv_addr(s) + x * C::kBoxBytes, map, bar(C::kBarFull + s), x * 64, hk,
+                      k_row0 + j * BN, bc);
         load_count[s]++;
       }
     }

@@ -73,7 +73,8 @@ typedef enum {
     ATTN_ERR_TIMEOUT = 9,   /* a device-side bounded wait ran out                 */
     ATTN_ERR_WORKSPACE = 10, /* workspace NULL, misaligned or smaller than needed */
     ATTN_ERR_SCRATCH = 11,   /* problem too large for attn_bwd_noalloc's scratch  */
-    ATTN_ERR_DTYPE = 12      /* element format not one of attn_dtype              */
+    ATTN_ERR_DTYPE = 12,     /* element format not one of attn_dtype              */
+    ATTN_ERR_SEQLENS = 13    /* (device) malformed cu_seqlens of a packed batch   */
 } attn_status;
 
 /* Element format of the 16-bit tensors (Q, K, V, O, dO, dQ, dK, dV): the RTX
@@ -253,13 +254,56 @@ ATTN_API attn_status attn_decode(const void* q, const void* k_cache, const void*
                                  int causal, void* workspace, size_t workspace_bytes,
                                  void* stream);
 
+/*
+ * attn_fwd_varlen / attn_bwd_varlen - a batch of B sequences of different
+ * lengths packed end to end (the pages name the upstream variable-length and
+ * padded-batch tests, FlashAttention-2 overview, lshu.cn, section 3.2, and say
+ * nothing more).  Sequence b is rows cu_seqlens_q[b] .. cu_seqlens_q[b+1]-1 of
+ * q, o, dout and dq and rows cu_seqlens_k[b] .. cu_seqlens_k[b+1]-1 of k, v, dk
+ * and dv; it attends only within itself, with the causal / window rules of
+ * attn_fwd applied to its own lengths (bottom-right alignment per sequence).
+ * A sequence with no keys gives its rows O = 0, LSE = -inf; one with no query
+ * rows gives its keys dK = dV = 0.  Grouped K/V heads and dtype as in the _ex
+ * entry points.
+ *
+ *   q, o, dout, dq  [total_q, H, D]        k, v, dk, dv [total_k, Hk, D]
+ *   lse             [H, total_q] float32 (out of attn_fwd_varlen, in of bwd)
+ *   cu_seqlens_q/k  [B + 1] int32, device: cu[0] = 0, non-decreasing,
+ *                   cu[B] = total; no sequence longer than max_seqlen_q / _k
+ *                   (the grid is sized from the two maxima).
+ *   workspace       (bwd) at least attn_bwd_varlen_workspace_size(B, total_q,
+ *                   H, D) bytes, 256-byte aligned, contents ignored.
+ * The boundaries live on the device, so they are checked there: a malformed
+ * sequence is skipped (nothing of it read or written) and the next
+ * attn_get_last_device_error returns ATTN_ERR_SEQLENS.
+ * Errors: as attn_fwd_ex / attn_bwd_ex; ATTN_ERR_SHAPE also if total_q or
+ * total_k < 1, or a max_seqlen is < 1 or above its total; ATTN_ERR_ALIGN if lse
+ * or a cu_seqlens pointer is not 4-byte aligned.
+ */
+ATTN_API attn_status attn_fwd_varlen(const void* q, const void* k, const void* v,
+                                     const int* cu_seqlens_q, const int* cu_seqlens_k, void* o,
+                                     float* lse, int B, int total_q, int total_k,
+                                     int max_seqlen_q, int max_seqlen_k, int H, int Hk, int D,
+                                     int dtype, float scale, int causal, int win_left,
+                                     int win_right, void* stream);
+ATTN_API size_t attn_bwd_varlen_workspace_size(int B, int total_q, int H, int D);
+ATTN_API attn_status attn_bwd_varlen(const void* q, const void* k, const void* v, const void* o,
+                                     const void* dout, const float* lse,
+                                     const int* cu_seqlens_q, const int* cu_seqlens_k, void* dq,
+                                     void* dk, void* dv, int B, int total_q, int total_k,
+                                     int max_seqlen_q, int max_seqlen_k, int H, int Hk, int D,
+                                     int dtype, float scale, int causal, int win_left,
+                                     int win_right, void* workspace, size_t workspace_size,
+                                     void* stream);
+
 /* attn_status_string - static English text for a status code (never NULL). */
 ATTN_API const char* attn_status_string(attn_status s);
 
 /*
  * attn_get_last_device_error - synchronises the current device, then returns
  * ATTN_ERR_TIMEOUT if a kernel of this library recorded a timed-out wait since
- * the last call (and clears the record), ATTN_ERR_LAUNCH if the device reports
+ * the last call, ATTN_ERR_SEQLENS if one found malformed packed-sequence
+ * boundaries (and clears the record), ATTN_ERR_LAUNCH if the device reports
  * an error, ATTN_OK otherwise.
  */
 ATTN_API attn_status attn_get_last_device_error(void);

@@ -44,7 +44,7 @@ def test_status_enum_matches_binding():
 
 def test_status_strings():
     from exact_attention_156_b200 import status_string
-    for s in range(13):
+    for s in range(14):
         assert status_string(s) and status_string(s) != "unknown status"
     assert status_string(99) == "unknown status"
 
@@ -172,3 +172,42 @@ def test_decode_validation():
     assert dec(wsp=None) == 10
     assert dec(wsz=ws - 1) == 10
     assert dec() in (ARCH, DEVICE)
+
+
+def test_varlen_validation_and_workspace_size():
+    from exact_attention_156_b200 import lib
+    # rows per head: total_q + 132 B rounded up to 4; fp32 dQ row + two row values each
+    assert lib.attn_bwd_varlen_workspace_size(3, 1000, 2, 64) == 2 * 1396 * (64 * 4 + 8)
+    assert lib.attn_bwd_varlen_workspace_size(1, 1, 1, 128) == 136 * (128 * 4 + 8)
+    assert lib.attn_bwd_varlen_workspace_size(0, 1000, 2, 64) == 0
+    assert lib.attn_bwd_varlen_workspace_size(2, 1000, 2, 96) == 0
+
+    def fwd(cu_q=0x9000, cu_k=0xA000, B=2, tq=300, tk=400, mq=200, mk=250, H=4, Hk=2, D=128,
+            dtype=0, q=0x1000, lse=0x6000, wl=-1):
+        return lib.attn_fwd_varlen(q, 0x2000, 0x3000, cu_q, cu_k, 0x4000, lse, B, tq, tk, mq, mk,
+                                   H, Hk, D, dtype, 0.1, 1, wl, -1, None)
+    assert fwd(cu_q=None) == NULLPTR
+    assert fwd(B=0) == SHAPE
+    assert fwd(tq=0) == SHAPE
+    assert fwd(mq=0) == SHAPE
+    assert fwd(mq=301) == SHAPE          # a sequence cannot be longer than the batch
+    assert fwd(mk=401) == SHAPE
+    assert fwd(Hk=3) == SHAPE
+    assert fwd(D=80) == HEADDIM
+    assert fwd(wl=-3) == WINDOW
+    assert fwd(dtype=2) == 12
+    assert fwd(q=0x1008) == ALIGN
+    assert fwd(cu_k=0xA002) == ALIGN
+    assert fwd(lse=0x6001) == ALIGN
+    assert fwd() in (ARCH, DEVICE)
+    ws = lib.attn_bwd_varlen_workspace_size(2, 300, 4, 128)
+
+    def bwd(wsp=0x100000, wsz=ws, cu_q=0x9000):
+        return lib.attn_bwd_varlen(0x1000, 0x2000, 0x3000, 0x4000, 0x5000, 0x6000, cu_q, 0xA000,
+                                   0x7000, 0x8000, 0xB000, 2, 300, 400, 200, 250, 4, 2, 128, 0,
+                                   0.1, 1, -1, -1, wsp, wsz, None)
+    assert bwd(cu_q=None) == NULLPTR
+    assert bwd(wsp=None) == 10
+    assert bwd(wsp=0x100080) == 10       # not 256-byte aligned
+    assert bwd(wsz=ws - 1) == 10
+    assert bwd() in (ARCH, DEVICE)
