@@ -43,7 +43,11 @@ GQA_WORKLOAD = dict(name="gqa_b1h32hk8s8192d128_fwdbwd", B=1, H=32, Hk=8, Sq=819
 # KV-cache decode: one new query row per sequence over a full 8192-row cache
 DECODE_WORKLOAD = dict(name="decode_b8h32hk8l8192d128", B=8, Sq=1, H=32, Hk=8, Smax=8192,
                        D=128, causal=0, input_scale=0.5, seed=1007)
-WORKLOADS = {"fwdbwd": WORKLOAD, "gqa": GQA_WORKLOAD, "decode": DECODE_WORKLOAD}
+# packed variable-length batch: 32768 tokens in sequences of 128..4096 tokens
+VARLEN_WORKLOAD = dict(name="varlen_t32768h32d128_fwdbwd", total=32768, len_lo=128,
+                       len_hi=4096, H=32, Hk=32, D=128, causal=1, input_scale=0.5, seed=1008)
+WORKLOADS = {"fwdbwd": WORKLOAD, "gqa": GQA_WORKLOAD, "decode": DECODE_WORKLOAD,
+             "varlen": VARLEN_WORKLOAD}
 DECODE_METRIC = "KV-cache decode: cached K/V bytes read per second"
 FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "hbm_gbs": 6650.0, "source": "fallback"}
 BWD_KERNEL_SOURCES = ["bwd_sm100.cuh", "ptx.cuh", "common.cuh"]
@@ -619,6 +623,224 @@ def run_decode(args):
     return 0
 
 
+def varlen_lengths(w):
+    from synth import packed_lengths
+    return packed_lengths(w["total"], w["len_lo"], w["len_hi"], w["seed"])
+
+
+def varlen_fwd_flops(w, lengths) -> float:
+    """4*D per (query, key) pair of each sequence, halved for causal (the
+    headline's convention, per sequence)."""
+    f = sum(4.0 * w["H"] * L * L * w["D"] for L in lengths)
+    return f / 2 if w["causal"] else f
+
+
+def varlen_config(w, lengths):
+    return {"workload": f"{w['name']}: fwd+bwd of a packed batch, {len(lengths)} sequences of "
+                        f"{min(lengths)}..{max(lengths)} tokens ({w['total']} in all, lengths "
+                        f"log-uniform in [{w['len_lo']}, {w['len_hi']}]), H={w['H']} "
+                        f"D={w['D']} causal, inputs N(0,1)*{w['input_scale']}",
+            "total_tokens": w["total"], "sequences": len(lengths), "H": w["H"], "D": w["D"],
+            "causal": bool(w["causal"]),
+            "l2": "no flush: inputs (Q,K,V,dO 256 MiB) and outputs exceed the 126 MB L2"}
+
+
+def varlen_oracle_step(inputs, w, lengths, idx: int):
+    """Oracle fwd+bwd of one head of one sequence of the batch (seeded pick).
+    Returns (seconds, flops by the metric's convention)."""
+    import numpy as np
+    import oracle
+    rng = np.random.default_rng(20_000 + idx)
+    b = int(rng.integers(0, len(lengths)))
+    h = int(rng.integers(0, w["H"]))
+    c0 = sum(lengths[:b])
+    L = lengths[b]
+    cu = [0, L]
+    sl = lambda x: x[c0:c0 + L, h:h + 1]
+    t0 = time.perf_counter()
+    oracle.attention_backward_varlen(sl(inputs["q"]), sl(inputs["k"]), sl(inputs["v"]),
+                                     sl(inputs["do"]), cu, cu, 1.0 / math.sqrt(w["D"]),
+                                     w["causal"])
+    dt = time.perf_counter() - t0
+    return dt, 3.5 * 4.0 * L * L * w["D"] / (2 if w["causal"] else 1)
+
+
+def varlen_oracle_inputs(w, rank: int = 0):
+    from synth import bits_to_f32, make_inputs
+    T = w["total"]
+    bits = make_inputs(1, T, T, w["H"], w["D"], w["seed"] + rank, w["input_scale"],
+                       with_dout=True, Hk=w["Hk"])
+    return {n: bits_to_f32(bits[n])[0] for n in ("q", "k", "v", "do")}
+
+
+def run_varlen_reference(args):
+    rank, _, _ = dist_env()
+    if rank != 0:
+        return 0
+    w = VARLEN_WORKLOAD
+    lengths = varlen_lengths(w)
+    inputs = varlen_oracle_inputs(w)
+    for i in range(args.warmup):
+        varlen_oracle_step(inputs, w, lengths, 1000 + i)
+    tot_s = tot_f = 0.0
+    for i in range(args.steps):
+        dt, fl = varlen_oracle_step(inputs, w, lengths, i)
+        tot_s += dt
+        tot_f += fl
+    value = tot_f / tot_s / 1e12
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": tot_s / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": varlen_config(w, lengths),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+                         "sample": f"each step: fwd+bwd of one seeded (sequence, head) of "
+                                   f"{w['name']}, float64 numpy"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0}}), flush=True)
+    return 0
+
+
+def run_varlen(args):
+    """fwd + bwd of a packed variable-length batch (one step = both calls)."""
+    import numpy as np
+    import torch
+    rank, world, local = dist_env()
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    device = torch.device("cuda", local if world > 1 else torch.cuda.current_device())
+    torch.cuda.set_device(device)
+    from exact_attention_156_b200 import (attn_bwd_varlen, attn_bwd_varlen_workspace_size,
+                                          attn_fwd_varlen, get_last_device_error)
+    from synth import make_inputs
+    w = VARLEN_WORKLOAD
+    lengths = varlen_lengths(w)
+    T, H, D = w["total"], w["H"], w["D"]
+    bits = make_inputs(1, T, T, H, D, w["seed"] + rank, w["input_scale"], with_dout=True,
+                       Hk=w["Hk"], fmt=args.dtype)
+    tdtype = torch.float16 if args.dtype == "f16" else torch.bfloat16
+    host = {n: torch.from_numpy(bits[n][0].view("int16")).view(tdtype).pin_memory()
+            for n in ("q", "k", "v", "do")}
+    cu_host = torch.from_numpy(np.concatenate([[0], np.cumsum(lengths)]).astype(np.int32))
+    host["cu"] = cu_host.pin_memory()
+    dev = {n: t.to(device) for n, t in host.items()}
+    q, k, v, do, cu = dev["q"], dev["k"], dev["v"], dev["do"], dev["cu"]
+    Lmax = max(lengths)
+    o = torch.empty_like(q)
+    lse = torch.empty((H, T), dtype=torch.float32, device=device)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws = torch.empty(attn_bwd_varlen_workspace_size(len(lengths), T, H, D), dtype=torch.uint8,
+                     device=device)
+    stream = torch.cuda.current_stream(device)
+    causal = bool(w["causal"])
+
+    def step(evs=None):
+        if evs is not None:
+            evs[0].record(stream)
+        attn_fwd_varlen(q, k, v, cu, cu, Lmax, Lmax, causal=causal, out=o, lse=lse,
+                        stream=stream)
+        if evs is not None:
+            evs[1].record(stream)
+        attn_bwd_varlen(q, k, v, o, do, lse, cu, cu, Lmax, Lmax, causal=causal, dq=dq, dk=dk,
+                        dv=dv, workspace=ws, stream=stream)
+        if evs is not None:
+            evs[2].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(device)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler("GPU-" + str(torch.cuda.get_device_properties(device).uuid))
+    barrier(device)
+    torch.cuda.synchronize(device)
+    sampler.start()
+    start.record(stream)
+    for i in range(args.steps):
+        step(evs[i])
+    end.record(stream)
+    torch.cuda.synchronize(device)
+    barrier(device)
+    clocks = sampler.stop()
+    if get_last_device_error() != 0:
+        raise RuntimeError("device-side error during the timed region")
+    fwd_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+    bwd_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+    ms = reduce_max(start.elapsed_time(end), device) / args.steps
+    ff = varlen_fwd_flops(w, lengths)
+    value = world * 3.5 * ff / (ms * 1e-3) / 1e12
+    out_host = {n: torch.empty(t.shape, dtype=t.dtype).pin_memory()
+                for n, t in (("o", o), ("lse", lse), ("dq", dq), ("dk", dk), ("dv", dv))}
+    e2e = None
+    if not args.no_e2e:
+        def e2e_step():
+            for n in ("q", "k", "v", "do", "cu"):
+                dev[n].copy_(host[n], non_blocking=True)
+            step()
+            for n, t in (("o", o), ("lse", lse), ("dq", dq), ("dk", dk), ("dv", dv)):
+                out_host[n].copy_(t, non_blocking=True)
+        e2e_step()
+        torch.cuda.synchronize(device)
+        barrier(device)
+        n_e2e = max(3, min(args.steps, 10))
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(n_e2e):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize(device)
+        barrier(device)
+        e2e_ms = reduce_max(e0.elapsed_time(e1), device) / n_e2e
+        e2e = {"value": world * 3.5 * ff / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
+               "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in host.values()),
+               "d2h_bytes_per_step": sum(t.numel() * t.element_size()
+                                         for t in out_host.values()),
+               "ms_per_step": e2e_ms, "steps": n_e2e}
+    peaks = load_peaks()
+    peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    bwd_tf = 2.5 * ff / (bwd_ms * 1e-3) / 1e12
+    fwd_tf = ff / (fwd_ms * 1e-3) / 1e12
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": args.dtype, "data": "synthetic",
+        "config": varlen_config(w, lengths),
+        "roofline": {"bound": "tensor",
+                     "kernel": "attn_bwd_varlen (preprocess + main + dQ finalize launches)",
+                     "achieved": bwd_tf, "peak": peak, "unit": "TFLOP/s", "frac": bwd_tf / peak,
+                     "peak_source": f"{peaks.get('source')} bf16_tflops (burst)",
+                     "traffic": None},
+        "kernels": {"fwd_varlen": {"ms": fwd_ms, "tflops": fwd_tf, "frac": fwd_tf / peak},
+                    "bwd_varlen": {"ms": bwd_ms, "tflops": bwd_tf, "frac": bwd_tf / peak}},
+        "e2e": e2e,
+        "gpu_launches": 4 * args.steps,
+        "clocks": clocks,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        inputs = varlen_oracle_inputs(w)
+        tot_s = tot_f = 0.0
+        n = 0
+        while tot_s < 10.0 and n < 64:
+            dt, fl = varlen_oracle_step(inputs, w, lengths, n)
+            tot_s += dt
+            tot_f += fl
+            n += 1
+        line["cpu_baseline"] = {"value": tot_f / tot_s / 1e12, "unit": UNIT,
+                                "cores": blas_threads(), "kind": "oracle",
+                                "sample": f"{n} seeded (sequence, head) pairs of {w['name']}, "
+                                          f"fwd+bwd in float64 numpy, {tot_s:.1f} s"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -630,7 +852,8 @@ def main(argv=None):
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="fwdbwd",
                     help="fwdbwd: the headline fwd+bwd workload (default); gqa: the same sizes "
                          "with 8 K/V heads for 32 query heads; decode: KV-cache decode "
-                         "(B8 H32 Hk8, 8192 cached rows, one new row)")
+                         "(B8 H32 Hk8, 8192 cached rows, one new row); varlen: a packed batch "
+                         "of 32768 tokens in sequences of 128..4096")
     ap.add_argument("--no-cpu-baseline", action="store_true",
                     help="skip the timed oracle sample (it adds ~15 s of CPU time)")
     ap.add_argument("--no-e2e", action="store_true",
@@ -640,6 +863,8 @@ def main(argv=None):
         ap.error("--warmup must be >= 3")
     if args.workload == "decode":
         return run_decode_reference(args) if args.impl == "reference" else run_decode(args)
+    if args.workload == "varlen":
+        return run_varlen_reference(args) if args.impl == "reference" else run_varlen(args)
     if args.impl == "reference":
         return run_reference(args)
     return run_gpu(args)

@@ -91,6 +91,9 @@ attn_status device_state(DeviceState** out) {
         both(std::true_type{});   // packed variable-length batches
         ok = ok &&
              set_smem(dec::attn_decode_kernel<D, E>, dec::Cfg<D>::kSmemBytes) == cudaSuccess;
+        if constexpr (D == 128)
+          ok = ok && set_smem(dec::t16::attn_decode_t16_kernel<E>, dec::t16::Cfg::kSmemBytes) ==
+                         cudaSuccess;
       };
       prepare(std::integral_constant<int, 64>{}, ElemBF16{});
       prepare(std::integral_constant<int, 128>{}, ElemBF16{});
@@ -474,8 +477,9 @@ attn_status run_backward_varlen(const DeviceState& st, const void* q, const void
 
 // Decode: the key range of each (batch, K/V head) is cut into splits of whole
 // 128-key tiles, one CTA each.  The split length minimises the estimated time
-// ceil(CTAs / SMs) x (tiles per split + 1) (the + 1: a CTA's start-up and
-// pipeline fill), so the last wave of CTAs is not left mostly empty.  Splits
+// ceil(CTAs / SMs) x (tiles per split + 3) (the + 3: a CTA's start-up and
+// pipeline fill, measured at about three tiles' time), so the last wave of
+// CTAs is not left mostly empty.  Splits
 // have at least two tiles unless the cache has one; the workspace is sized for
 // the largest split count this allows.
 struct DecodePlan {
@@ -489,7 +493,7 @@ DecodePlan decode_plan(int B, int Smax, int Hk, int num_sms) {
   for (int tps = tiles > 1 ? 2 : 1; tps <= tiles; ++tps) {
     const int nsplit = (tiles + tps - 1) / tps;
     const long long waves = (pairs * nsplit + num_sms - 1) / num_sms;
-    const long long cost = waves * (tps + 1);
+    const long long cost = waves * (tps + 3);
     if (best_cost < 0 || cost < best_cost) {
       best_cost = cost;
       best = {nsplit, tps};
@@ -549,8 +553,18 @@ attn_status launch_decode(const DeviceState& st, const void* q, const void* kc, 
   p.causal = causal ? 1 : 0;
   p.err = st.err;
   p.timeout_ns = kTimeoutNs;
-  dec::attn_decode_kernel<D, E><<<dim3(plan.nsplit, Hk, B), dec::kThreads,
-                                  dec::Cfg<D>::kSmemBytes, stream>>>(mq, mk, mv, p);
+  // at most 16 query rows per K/V head (one new token, up to 16 query heads
+  // each): keys on the tensor-memory lanes; otherwise query rows on the lanes
+  bool transposed = false;
+  if constexpr (D == 128) transposed = group * Sq <= dec::t16::kRows;
+  if (transposed) {
+    if constexpr (D == 128)
+      dec::t16::attn_decode_t16_kernel<E><<<dim3(plan.nsplit, Hk, B), dec::t16::kThreads,
+                                            dec::t16::Cfg::kSmemBytes, stream>>>(mq, mk, mv, p);
+  } else {
+    dec::attn_decode_kernel<D, E><<<dim3(plan.nsplit, Hk, B), dec::kThreads,
+                                    dec::Cfg<D>::kSmemBytes, stream>>>(mq, mk, mv, p);
+  }
   if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_LAUNCH;
   const long long nrow = (long long)B * H * Sq;
   dec::attn_decode_combine_kernel<D, E><<<unsigned((nrow + 7) / 8), 256, 0, stream>>>(

@@ -363,7 +363,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     return;
   }
 
-  const int kt = blockIdx.x;  // key tile; low indices see the most query tiles when causal
+  // Grid: (key tile, K/V head, batch).  The key tiles of one head run side by
+  // side, so they share that head's Q and dO tiles in L2; low key tiles (the
+  // most query tiles when causal) start first.
+  const int kt = blockIdx.x;
   const int hk = blockIdx.y;  // key/value head
   const int b = blockIdx.z;
   const int group = p.H / p.Hk;  // query heads sharing this K/V head
@@ -384,6 +387,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   };
   const MaskGeom g = MaskGeom::make(Lq, Lk, p.causal, p.win_left, p.win_right);
   const int n0 = kt * BN;
+  // No key of this sequence falls in this CTA (shorter sequences of a packed
+  // batch): nothing to compute or write.
+  if (n0 >= Lk) return;
   const int n1 = min(n0 + BN - 1, Lk - 1);
   int qlo, qhi;
   qtile_range(g, n0, n1, qlo, qhi);

@@ -131,6 +131,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     return;
   }
 
+  // Grid: (query-tile pair, head, batch).  The pairs of one head run side by
+  // side, so they share that head's K/V tiles in L2; causal launches each
+  // head's pairs with the most keys first.
   const int mb = p.causal ? (p.num_mblocks - 1 - int(blockIdx.x)) : int(blockIdx.x);
   const int h = blockIdx.y;
   const int hk = h / (p.H / p.Hk);  // the key/value head this query head reads
@@ -163,6 +166,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
   const bool any_work = ju_hi > ju_lo;
+  // No query row of this sequence falls in this CTA (shorter sequences of a
+  // packed batch): nothing to compute or write.
+  if (!valid[0] && !valid[1]) return;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::kNumBars; ++i) {

@@ -312,6 +312,82 @@ __device__ __forceinline__ void mma_chain_mnmn8(uint32_t d_tmem, uint64_t a_desc
       : "memory");
 }
 
+// 8 chained K-steps, A K-major (16 KB boxes), B K-major in boxes of 16 rows
+// (2 KB: a small N = 16 operand) (SS form).
+__device__ __forceinline__ void mma_chain_kk8_b16(uint32_t d_tmem, uint64_t a_desc,
+                                                  uint64_t b_desc, uint32_t idesc,
+                                                  uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .b32 alo, ahi, blo, bhi, al, bl;\n\t.reg .b64 ad, bd;\n\t.reg .pred pa, pt;\n\t"
+      "mov.b64 {alo, ahi}, %1;\n\tmov.b64 {blo, bhi}, %2;\n\t"
+      "setp.ne.b32 pa, %4, 0;\n\tsetp.eq.b32 pt, 0, 0;\n\t"
+      "add.u32 al, alo, 0;\n\tadd.u32 bl, blo, 0;\n\t"
+      "mov.b64 ad, {al, ahi};\n\tmov.b64 bd, {bl, bhi};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], ad, bd, %3, pa;\n\t"
+      "add.u32 al, alo, 2;\n\tadd.u32 bl, blo, 2;\n\t"
+      "mov.b64 ad, {al, ahi};\n\tmov.b64 bd, {bl, bhi};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], ad, bd, %3, pt;\n\t"
+      "add.u32 al, alo, 4;\n\tadd.u32 bl, blo, 4;\n\t"
+      "mov.b64 ad, {al, ahi};\n\tmov.b64 bd, {bl, bhi};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], ad, bd, %3, pt;\n\t"
+      "add.u32 al, alo, 6;\n\tadd.u32 bl, blo, 6;\n\t"
+      "mov.b64 ad, {al, ahi};\n\tmov.b64 bd, {bl, bhi};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], ad, bd, %3, pt;\n\t"
+      "add.u32 al, alo, 1024;\n\tadd.u32 bl, blo, 128;\n\t"
+      "mov.b64 ad, {al, ahi};\n\tmov.b64 bd, {bl, bhi};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], ad, bd, %3, pt;\n\t"
+      "add.u32 al, alo, 1026;\n\tadd.u32 bl, blo, 130;\n\t"
+      "mov.b64 ad, {al, ahi};\n\tmov.b64 bd, {bl, bhi};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], ad, bd, %3, pt;\n\t"
+      "add.u32 al, alo, 1028;\n\tadd.u32 bl, blo, 132;\n\t"
+      "mov.b64 ad, {al, ahi};\n\tmov.b64 bd, {bl, bhi};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], ad, bd, %3, pt;\n\t"
+      "add.u32 al, alo, 1030;\n\tadd.u32 bl, blo, 134;\n\t"
+      "mov.b64 ad, {al, ahi};\n\tmov.b64 bd, {bl, bhi};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], ad, bd, %3, pt;\n\t"
+      "}"
+      :: "r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// 8 chained K-steps, A MN-major, B K-major in boxes of 16 rows (2 KB: a small
+// N = 16 operand, the next 64-element K block 2 KB further on) (SS form).
+__device__ __forceinline__ void mma_chain_mnk8_b16(uint32_t d_tmem, uint64_t a_desc,
+                                                   uint64_t b_desc, uint32_t idesc,
+                                                   uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .b32 alo, ahi, blo, bhi, al, bl;\n\t.reg .b64 ad, bd;\n\t.reg .pred pa, pt;\n\t"
+      "mov.b64 {alo, ahi}, %1;\n\tmov.b64 {blo, bhi}, %2;\n\t"
+      "setp.ne.b32 pa, %4, 0;\n\tsetp.eq.b32 pt, 0, 0;\n\t"
+      "add.u32 al, alo, 0;\n\tadd.u32 bl, blo, 0;\n\t"
+      "mov.b64 ad, {al, ahi};\n\tmov.b64 bd, {bl, bhi};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], ad, bd, %3, pa;\n\t"
+      "add.u32 al, alo, 128;\n\tadd.u32 bl, blo, 2;\n\t"
+      "mov.b64 ad, {al, ahi};\n\tmov.b64 bd, {bl, bhi};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], ad, bd, %3, pt;\n\t"
+      "add.u32 al, alo, 256;\n\tadd.u32 bl, blo, 4;\n\t"
+      "mov.b64 ad, {al, ahi};\n\tmov.b64 bd, {bl, bhi};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], ad, bd, %3, pt;\n\t"
+      "add.u32 al, alo, 384;\n\tadd.u32 bl, blo, 6;\n\t"
+      "mov.b64 ad, {al, ahi};\n\tmov.b64 bd, {bl, bhi};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], ad, bd, %3, pt;\n\t"
+      "add.u32 al, alo, 512;\n\tadd.u32 bl, blo, 128;\n\t"
+      "mov.b64 ad, {al, ahi};\n\tmov.b64 bd, {bl, bhi};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], ad, bd, %3, pt;\n\t"
+      "add.u32 al, alo, 640;\n\tadd.u32 bl, blo, 130;\n\t"
+      "mov.b64 ad, {al, ahi};\n\tmov.b64 bd, {bl, bhi};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], ad, bd, %3, pt;\n\t"
+      "add.u32 al, alo, 768;\n\tadd.u32 bl, blo, 132;\n\t"
+      "mov.b64 ad, {al, ahi};\n\tmov.b64 bd, {bl, bhi};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], ad, bd, %3, pt;\n\t"
+      "add.u32 al, alo, 896;\n\tadd.u32 bl, blo, 134;\n\t"
+      "mov.b64 ad, {al, ahi};\n\tmov.b64 bd, {bl, bhi};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], ad, bd, %3, pt;\n\t"
+      "}"
+      :: "r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // 8 chained K-steps, A from tensor memory (8 columns per step), B MN-major (TS form).
 __device__ __forceinline__ void mma_chain_ts_mn8(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
                                    uint32_t idesc, uint32_t accumulate) {

@@ -15,5 +15,6 @@ from .inputs import (  # noqa: F401
     f32_to_bf16_bits,
     f32_to_f16_bits,
     make_inputs,
+    packed_lengths,
     sample_rows,
 )

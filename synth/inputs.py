@@ -148,6 +148,21 @@ def make_inputs(B: int, Sq: int, Sk: int, H: int, D: int, seed: int,
     return out
 
 
+def packed_lengths(total: int, lo: int, hi: int, seed: int) -> Tuple[int, ...]:
+    """Sequence lengths of a packed batch of exactly ``total`` tokens: lengths
+    drawn log-uniformly in [lo, hi] (numpy PCG64(seed)) until the total is
+    reached, the last one cut to fit.  The mix of many short and a few long
+    sequences is that of a packed fine-tuning batch."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    out, used = [], 0
+    while used < total:
+        n = int(round(math.exp(rng.uniform(math.log(lo), math.log(hi)))))
+        n = min(max(n, 1), total - used)
+        out.append(n)
+        used += n
+    return tuple(out)
+
+
 def make_config_inputs(cfg: AttnConfig, with_dout: Optional[bool] = None):
     wd = cfg.backward if with_dout is None else with_dout
     return make_inputs(cfg.B, cfg.Sq, cfg.Sk, cfg.H, cfg.D, cfg.seed, cfg.input_scale, wd)

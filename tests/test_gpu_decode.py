@@ -1,5 +1,7 @@
 """KV-cache decode (attn_decode): the CUDA path against the float64 oracle's
 attention_decode on the same seeded inputs, with the forward parity bars.
+Cases with head_dim 128 and at most 16 query rows per K/V head run the
+keys-on-lanes kernel, the others the rows-on-lanes kernel.
 Cache rows past each sequence's length are filled with NaN and huge values:
 they must not reach the result."""
 import numpy as np
@@ -19,6 +21,9 @@ CASES = [
     (2, 1, 8192, 32, 8, 128, 0, (8192, 5000), "f16"),
     (2, 3, 300, 4, 2, 128, 1, (2, 300), "bf16"),           # a row that sees no key (L < Sq)
     (3, 1, 640, 8, 8, 64, 0, (0, 129, 640), "bf16"),       # an empty cache, one row past a tile
+    (2, 1, 2048, 16, 1, 128, 0, (2048, 1500), "bf16"),     # 16 query heads on one K/V head
+    (3, 1, 777, 4, 4, 128, 1, (777, 1, 129), "f16"),       # one row per K/V head, a one-key cache
+    (1, 8, 1024, 2, 1, 128, 1, (1000,), "bf16"),           # 8 new positions x 2 heads, causal
 ]
 
 
