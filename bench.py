@@ -600,11 +600,12 @@ def run_decode(args):
         "scaling": "weak", "vs_baseline": None, "dtype": args.dtype, "data": "synthetic",
         "config": decode_config(w),
         "roofline": {"bound": "hbm",
-                     "kernel": "attn_decode_kernel<128> (timed with its combine launch)",
+                     "kernel": "attn_decode_t16_kernel (timed with its combine launch)",
                      "achieved": decode_bytes(w) / (ms * 1e-3) / 1e9, "peak": peak,
                      "unit": "GB/s", "frac": decode_bytes(w) / (ms * 1e-3) / 1e9 / peak,
                      "peak_source": f"{peaks.get('source')} hbm_gbs",
-                     "traffic": committed_traffic(traffic_key("attn_decode_kernel", w, args.dtype),
+                     "traffic": committed_traffic(traffic_key("attn_decode_t16_kernel", w,
+                                                              args.dtype),
                                                   sources_sha(DECODE_KERNEL_SOURCES))},
         "e2e": {"value": world * decode_bytes(w) / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
                 "h2d_bytes_per_step": q_host.numel() * q_host.element_size(),

@@ -566,10 +566,24 @@ attn_status launch_decode(const DeviceState& st, const void* q, const void* kc, 
                                     dec::Cfg<D>::kSmemBytes, stream>>>(mq, mk, mv, p);
   }
   if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_LAUNCH;
+  // The combine is a programmatic dependent of the split kernel: its launch
+  // overlaps the split kernel's tail, and it waits for that grid's results.
   const long long nrow = (long long)B * H * Sq;
-  dec::attn_decode_combine_kernel<D, E><<<unsigned((nrow + 7) / 8), 256, 0, stream>>>(
-      p.opart, p.lsepart, static_cast<uint16_t*>(o), lse, B, Sq, H, plan.nsplit);
-  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_LAUNCH;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(unsigned((nrow + 7) / 8));
+  cfg.blockDim = dim3(256);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e =
+      cudaLaunchKernelEx(&cfg, dec::attn_decode_combine_kernel<D, E>,
+                         static_cast<const float*>(p.opart), static_cast<const float*>(p.lsepart),
+                         static_cast<uint16_t*>(o), lse, B, Sq, H, plan.nsplit);
+  return (e == cudaSuccess && cudaGetLastError() == cudaSuccess) ? ATTN_OK : ATTN_ERR_LAUNCH;
 }
 
 attn_status check_workspace(const void* workspace, size_t bytes, int B, int Sq, int H, int D) {

@@ -115,6 +115,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (threadIdx.x == 0) atomicCAS(p.err, 0u, 8u);
     return;
   }
+  // the combine grid may be scheduled now; it waits for this grid to finish
+  griddep_launch_dependents();
 
   const int split = blockIdx.x;
   const int g = blockIdx.y;  // K/V head
@@ -471,6 +473,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (threadIdx.x == 0) atomicCAS(p.err, 0u, 8u);
     return;
   }
+  // the combine grid may be scheduled now; it waits for this grid to finish
+  griddep_launch_dependents();
 
   const int split = blockIdx.x;
   const int g = blockIdx.y;  // K/V head
@@ -776,6 +780,9 @@ template <int D, class E>
 __global__ void __launch_bounds__(256) attn_decode_combine_kernel(
     const float* __restrict__ opart, const float* __restrict__ lsepart,
     uint16_t* __restrict__ o, float* __restrict__ lse, int B, int Sq, int H, int nsplit) {
+  // launched as a programmatic dependent of the split kernel: wait for it to
+  // complete before reading its partial results
+  griddep_wait();
   const long long row = (long long)blockIdx.x * 8 + threadIdx.x / 32;  // (b, h, i)
   const int lane = threadIdx.x % 32;
   if (row >= (long long)B * H * Sq) return;

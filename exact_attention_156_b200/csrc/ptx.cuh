@@ -565,6 +565,16 @@ __device__ __forceinline__ void regs_realloc() {
 }
 
 // Named barrier over `count` threads (ids 1..15; id 0 is __syncthreads).
+// Programmatic dependent launch: a grid launched after this one with the
+// programmatic-serialization attribute may start once every CTA of this grid
+// has signalled (or exited); it must call griddep_wait() before it reads what
+// this grid writes (the wait returns once this grid has completed and its
+// memory operations are visible).
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 __device__ __forceinline__ void named_bar_sync(int id, int count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
