@@ -46,8 +46,12 @@ DECODE_WORKLOAD = dict(name="decode_b8h32hk8l8192d128", B=8, Sq=1, H=32, Hk=8, S
 # packed variable-length batch: 32768 tokens in sequences of 128..4096 tokens
 VARLEN_WORKLOAD = dict(name="varlen_t32768h32d128_fwdbwd", total=32768, len_lo=128,
                        len_hi=4096, H=32, Hk=32, D=128, causal=1, input_scale=0.5, seed=1008)
+# head_dim 256 (forward only): B1 H16 S8192 causal
+D256_WORKLOAD = dict(name="fwd_b1h16s8192d256_causal", B=1, H=16, Hk=16, Sq=8192, Sk=8192,
+                     D=256, causal=1, win_left=-1, win_right=-1, input_scale=0.5, seed=1009)
 WORKLOADS = {"fwdbwd": WORKLOAD, "gqa": GQA_WORKLOAD, "decode": DECODE_WORKLOAD,
-             "varlen": VARLEN_WORKLOAD}
+             "varlen": VARLEN_WORKLOAD, "d256": D256_WORKLOAD}
+D256_FWD_METRIC = "attention fwd TFLOPS, head_dim 256, bf16 vs B200 dense BF16 peak"
 DECODE_METRIC = "KV-cache decode: cached K/V bytes read per second"
 FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "hbm_gbs": 6650.0, "source": "fallback"}
 BWD_KERNEL_SOURCES = ["bwd_sm100.cuh", "ptx.cuh", "common.cuh"]
@@ -842,6 +846,163 @@ def run_varlen(args):
     return 0
 
 
+def run_fwd_only(args):
+    """Forward-only workload (head_dim 256, which has no backward here)."""
+    import torch
+    rank, world, local = dist_env()
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    device = torch.device("cuda", local if world > 1 else torch.cuda.current_device())
+    torch.cuda.set_device(device)
+    from exact_attention_156_b200 import attn_fwd, get_last_device_error
+    from synth import make_inputs
+    w = D256_WORKLOAD
+    B, H, Sq, Sk, D = w["B"], w["H"], w["Sq"], w["Sk"], w["D"]
+    bits = make_inputs(B, Sq, Sk, H, D, w["seed"] + rank, w["input_scale"], Hk=w["Hk"],
+                       fmt=args.dtype)
+    tdtype = torch.float16 if args.dtype == "f16" else torch.bfloat16
+    host = {n: torch.from_numpy(bits[n].view("int16")).view(tdtype).pin_memory()
+            for n in ("q", "k", "v")}
+    dev = {n: t.to(device) for n, t in host.items()}
+    q, k, v = dev["q"], dev["k"], dev["v"]
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, Sq), dtype=torch.float32, device=device)
+    stream = torch.cuda.current_stream(device)
+    causal = bool(w["causal"])
+    step = lambda: attn_fwd(q, k, v, causal=causal, out=o, lse=lse, stream=stream)
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(device)
+    barrier(device)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler("GPU-" + str(torch.cuda.get_device_properties(device).uuid))
+    sampler.start()
+    start.record(stream)
+    for _ in range(args.steps):
+        step()
+    end.record(stream)
+    torch.cuda.synchronize(device)
+    barrier(device)
+    clocks = sampler.stop()
+    if get_last_device_error() != 0:
+        raise RuntimeError("device-side error during the timed region")
+    ms = reduce_max(start.elapsed_time(end), device) / args.steps
+    ff = fwd_flops(w)
+    tf = ff / (ms * 1e-3) / 1e12
+    e2e = None
+    if not args.no_e2e:
+        o_host = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+        l_host = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+        n_e2e = max(3, min(args.steps, 10))
+        torch.cuda.synchronize(device)
+        barrier(device)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(n_e2e):
+            for n in ("q", "k", "v"):
+                dev[n].copy_(host[n], non_blocking=True)
+            step()
+            o_host.copy_(o, non_blocking=True)
+            l_host.copy_(lse, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize(device)
+        barrier(device)
+        e2e_ms = reduce_max(e0.elapsed_time(e1), device) / n_e2e
+        e2e = {"value": world * ff / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
+               "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in host.values()),
+               "d2h_bytes_per_step": o_host.numel() * o_host.element_size()
+               + l_host.numel() * l_host.element_size(), "ms_per_step": e2e_ms, "steps": n_e2e}
+    peaks = load_peaks()
+    peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    line = {
+        "metric": D256_FWD_METRIC, "value": world * tf, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": args.dtype, "data": "synthetic",
+        "config": {"workload": f"{w['name']}: forward, B={B} H={H} Sq=Sk={Sq} D={D} causal, "
+                               f"inputs N(0,1)*{w['input_scale']}", "B": B, "H": H, "Sq": Sq,
+                   "Sk": Sk, "D": D, "causal": causal,
+                   "l2": "no flush: inputs (Q,K,V 384 MiB) exceed the 126 MB L2"},
+        "roofline": {"bound": "tensor", "kernel": "attn_fwd_d256_kernel", "achieved": tf,
+                     "peak": peak, "unit": "TFLOP/s", "frac": tf / peak,
+                     "peak_source": f"{peaks.get('source')} bf16_tflops (burst)",
+                     "traffic": None},
+        "e2e": e2e,
+        "gpu_launches": args.steps,
+        "clocks": clocks,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = fwd_oracle_baseline(w)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+def fwd_oracle_sample(inputs, w, sample_idx: int):
+    """Oracle forward of ORACLE_ROWS_PER_SAMPLE seeded query rows of one head.
+    Returns (seconds, flops: 4*D per visible pair)."""
+    import numpy as np
+    import oracle
+    rng = np.random.default_rng(30_000 + sample_idx)
+    h = int(rng.integers(0, w["H"]))
+    rows = np.sort(rng.choice(w["Sq"], size=ORACLE_ROWS_PER_SAMPLE, replace=False))
+    trip = np.stack([np.zeros_like(rows), np.full_like(rows, h), rows], axis=1)
+    pairs = sum(visible_keys(int(i), w) for i in rows)
+    t0 = time.perf_counter()
+    oracle.attention_forward_rows(inputs["q"], inputs["k"], inputs["v"], trip,
+                                  1.0 / math.sqrt(w["D"]), w["causal"], w["win_left"],
+                                  w["win_right"])
+    return time.perf_counter() - t0, 4.0 * w["D"] * pairs
+
+
+def fwd_oracle_baseline(w, budget_s: float = 10.0):
+    inputs = oracle_sample_inputs(w)
+    tot_s = tot_f = 0.0
+    n = 0
+    while tot_s < budget_s and n < 64:
+        dt, fl = fwd_oracle_sample(inputs, w, n)
+        tot_s += dt
+        tot_f += fl
+        n += 1
+    return {"value": tot_f / tot_s / 1e12, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+            "sample": f"{n} samples x {ORACLE_ROWS_PER_SAMPLE} seeded query rows of one head of "
+                      f"{w['name']}, forward in float64 numpy, {tot_s:.1f} s"}
+
+
+def run_fwd_only_reference(args):
+    rank, _, _ = dist_env()
+    if rank != 0:
+        return 0
+    w = D256_WORKLOAD
+    inputs = oracle_sample_inputs(w)
+    for i in range(args.warmup):
+        fwd_oracle_sample(inputs, w, 1000 + i)
+    tot_s = tot_f = 0.0
+    for i in range(args.steps):
+        dt, fl = fwd_oracle_sample(inputs, w, i)
+        tot_s += dt
+        tot_f += fl
+    value = tot_f / tot_s / 1e12
+    print(json.dumps({
+        "impl": "reference", "metric": D256_FWD_METRIC, "value": value, "unit": UNIT,
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": tot_s / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": f"{w['name']}: forward, B={w['B']} H={w['H']} "
+                               f"Sq=Sk={w['Sq']} D={w['D']} causal"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+                         "sample": f"each step: {ORACLE_ROWS_PER_SAMPLE} seeded query rows of one "
+                                   f"head of {w['name']}, forward in float64 numpy"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0}}), flush=True)
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -854,7 +1015,8 @@ def main(argv=None):
                     help="fwdbwd: the headline fwd+bwd workload (default); gqa: the same sizes "
                          "with 8 K/V heads for 32 query heads; decode: KV-cache decode "
                          "(B8 H32 Hk8, 8192 cached rows, one new row); varlen: a packed batch "
-                         "of 32768 tokens in sequences of 128..4096")
+                         "of 32768 tokens in sequences of 128..4096; d256: head_dim 256 forward, "
+                         "B1 H16 S8192 causal")
     ap.add_argument("--no-cpu-baseline", action="store_true",
                     help="skip the timed oracle sample (it adds ~15 s of CPU time)")
     ap.add_argument("--no-e2e", action="store_true",
@@ -866,6 +1028,8 @@ def main(argv=None):
         return run_decode_reference(args) if args.impl == "reference" else run_decode(args)
     if args.workload == "varlen":
         return run_varlen_reference(args) if args.impl == "reference" else run_varlen(args)
+    if args.workload == "d256":
+        return run_fwd_only_reference(args) if args.impl == "reference" else run_fwd_only(args)
     if args.impl == "reference":
         return run_reference(args)
     return run_gpu(args)

@@ -15,6 +15,7 @@
 #include "../../include/attn.h"
 #include "bwd_sm100.cuh"
 #include "decode_sm100.cuh"
+#include "fwd256_sm100.cuh"
 #include "fwd_sm100.cuh"
 
 using namespace attn156;
@@ -90,7 +91,8 @@ attn_status device_state(DeviceState** out) {
         both(std::false_type{});  // (B, S, H, D) batches
         both(std::true_type{});   // packed variable-length batches
         ok = ok &&
-             set_smem(dec::attn_decode_kernel<D, E>, dec::Cfg<D>::kSmemBytes) == cudaSuccess;
+             set_smem(dec::attn_decode_kernel<D, E>, dec::Cfg<D>::kSmemBytes) == cudaSuccess &&
+             set_smem(fwd256::attn_fwd_d256_kernel<E>, fwd256::Cfg::kSmemBytes) == cudaSuccess;
         if constexpr (D == 128)
           ok = ok && set_smem(dec::t16::attn_decode_t16_kernel<E>, dec::t16::Cfg::kSmemBytes) ==
                          cudaSuccess;
@@ -134,12 +136,12 @@ bool on_current_device(const void* p) {
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 attn_status check_common(int B, int Sq, int Sk, int H, int D, float scale, int win_left,
-                         int win_right, int Hk = -1) {
+                         int win_right, int Hk = -1, bool allow_d256 = false) {
   if (Hk < 0) Hk = H;
   if (B < 1 || Sq < 1 || Sk < 1 || H < 1) return ATTN_ERR_SHAPE;
   if (B > 65535 || H > 65535) return ATTN_ERR_SHAPE;
   if (Hk < 1 || Hk > H || H % Hk != 0) return ATTN_ERR_SHAPE;
-  if (D != 64 && D != 128) return ATTN_ERR_HEADDIM;
+  if (D != 64 && D != 128 && !(allow_d256 && D == 256)) return ATTN_ERR_HEADDIM;
   if ((long long)B * Sq * H * D >= (1ll << 31) || (long long)B * Sk * Hk * D >= (1ll << 31))
     return ATTN_ERR_SHAPE;
   if (!(scale > 0.f) || !isfinite(scale)) return ATTN_ERR_SHAPE;
@@ -154,14 +156,14 @@ constexpr CUtensorMapDataType tmap_type() {
                                           : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
 }
 
-// 4-D map over a (B, S, H, D) tensor of 16-bit elements, box = 64 x 1 x 128 x 1,
-// 128-byte swizzle.
+// 4-D map over a (B, S, H, D) tensor of 16-bit elements, box = 64 x 1 x rows x 1
+// (rows = 128 unless given), 128-byte swizzle.
 attn_status make_map(CUtensorMap* map, const void* base, int B, int S, int H, int D,
-                     CUtensorMapDataType dtype) {
+                     CUtensorMapDataType dtype, int box_rows = 128) {
   const cuuint64_t dims[4] = {cuuint64_t(D), cuuint64_t(H), cuuint64_t(S), cuuint64_t(B)};
   const cuuint64_t strides[3] = {cuuint64_t(D) * 2, cuuint64_t(H) * D * 2,
                                  cuuint64_t(S) * H * D * 2};
-  const cuuint32_t box[4] = {64, 1, 128, 1};
+  const cuuint32_t box[4] = {64, 1, cuuint32_t(box_rows), 1};
   const cuuint32_t estr[4] = {1, 1, 1, 1};
   const CUresult r =
       g_encode(map, dtype, 4, const_cast<void*>(base), dims, strides,
@@ -222,6 +224,37 @@ attn_status launch_fwd(const DeviceState& st, const void* q, const void* k, cons
   dim3 grid(p.num_mblocks, H, B);
   fwd::attn_fwd_kernel<D, E, false><<<grid, fwd::kThreads, fwd::Cfg<D>::kSmemBytes, stream>>>(mq, mk, mv,
                                                                                        p);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_LAUNCH;
+}
+
+// head_dim 256 forward: one 128-row query tile per CTA, 64-key K/V tiles.
+template <class E>
+attn_status launch_fwd_d256(const DeviceState& st, const void* q, const void* k, const void* v,
+                            void* o, float* lse, int B, int Sq, int Sk, int H, int Hk, float scale,
+                            int causal, int win_left, int win_right, cudaStream_t stream) {
+  constexpr CUtensorMapDataType dt = tmap_type<E>();
+  alignas(64) CUtensorMap mq, mk, mv;
+  if (make_map(&mq, q, B, Sq, H, 256, dt, fwd256::BM) != ATTN_OK ||
+      make_map(&mk, k, B, Sk, Hk, 256, dt, fwd256::BN) != ATTN_OK ||
+      make_map(&mv, v, B, Sk, Hk, 256, dt, fwd256::BN) != ATTN_OK)
+    return ATTN_ERR_LAUNCH;
+  fwd256::Params p;
+  p.o = static_cast<uint16_t*>(o);
+  p.lse = lse;
+  p.B = B;
+  p.H = H;
+  p.Sq = Sq;
+  p.Sk = Sk;
+  p.Hk = Hk;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.causal = causal ? 1 : 0;
+  p.win_left = win_left;
+  p.win_right = win_right;
+  p.num_mblocks = (Sq + fwd256::BM - 1) / fwd256::BM;
+  p.err = st.err;
+  p.timeout_ns = kTimeoutNs;
+  fwd256::attn_fwd_d256_kernel<E><<<dim3(p.num_mblocks, H, B), fwd256::kThreads,
+                                    fwd256::Cfg::kSmemBytes, stream>>>(mq, mk, mv, p);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_LAUNCH;
 }
 
@@ -675,7 +708,7 @@ attn_status attn_fwd_ex(const void* q, const void* k, const void* v, void* o, fl
                         int Sq, int Sk, int H, int Hk, int D, int dtype, float scale, int causal,
                         int win_left, int win_right, void* stream) {
   if (!q || !k || !v || !o || !lse) return ATTN_ERR_NULLPTR;
-  attn_status s = check_common(B, Sq, Sk, H, D, scale, win_left, win_right, Hk);
+  attn_status s = check_common(B, Sq, Sk, H, D, scale, win_left, win_right, Hk, true);
   if (s != ATTN_OK) return s;
   if ((s = check_dtype(dtype)) != ATTN_OK) return s;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) ||
@@ -686,6 +719,13 @@ attn_status attn_fwd_ex(const void* q, const void* k, const void* v, void* o, fl
   if (s != ATTN_OK) return s;
   if (!all_on_device({q, k, v, o, lse})) return ATTN_ERR_DEVICE;
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  if (D == 256) {
+    return dtype == ATTN_DTYPE_F16
+               ? launch_fwd_d256<ElemF16>(*st, q, k, v, o, lse, B, Sq, Sk, H, Hk, scale, causal,
+                                          win_left, win_right, cs)
+               : launch_fwd_d256<ElemBF16>(*st, q, k, v, o, lse, B, Sq, Sk, H, Hk, scale, causal,
+                                           win_left, win_right, cs);
+  }
   return dispatch(D, dtype, [&](auto d, auto e) {
     return launch_fwd<decltype(d)::value, decltype(e)>(*st, q, k, v, o, lse, B, Sq, Sk, H, Hk,
                                                        scale, causal, win_left, win_right, cs);

@@ -37,7 +37,9 @@
  *     bottom-right corner when Sq != Sk.
  *   - scale must be finite and > 0 (callers wanting the default pass
  *     1/sqrt(head_dim)).
- *   - head_dim D must be 64 or 128.  B, H, Sq, Sk must be >= 1 and every
+ *   - head_dim D must be 64 or 128; the forward entry points attn_fwd and
+ *     attn_fwd_ex also take 256 (the backward, the varlen and the decode entry
+ *     points do not).  B, H, Sq, Sk must be >= 1 and every
  *     tensor must hold fewer than 2^31 elements.
  *   - The device must be compute capability 10.0 (B200, sm_100a).
  *   - Device-side waits are bounded (about one second); a wait that runs out
@@ -64,7 +66,7 @@ typedef enum {
     ATTN_OK = 0,
     ATTN_ERR_NULLPTR = 1,   /* a required pointer is NULL                         */
     ATTN_ERR_SHAPE = 2,     /* B, H, Sq or Sk < 1, a size overflows, or bad scale */
-    ATTN_ERR_HEADDIM = 3,   /* head_dim not in {64, 128}                          */
+    ATTN_ERR_HEADDIM = 3,   /* head_dim not in {64, 128} (forward: {64, 128, 256}) */
     ATTN_ERR_ALIGN = 4,     /* a tensor pointer is not 16-byte aligned            */
     ATTN_ERR_WINDOW = 5,    /* win_left or win_right < -1                         */
     ATTN_ERR_ARCH = 6,      /* current device is not compute capability 10.0      */

@@ -63,7 +63,8 @@ def test_fwd_validation_order_and_codes():
     assert _fwd(lib, H=70000) == SHAPE
     assert _fwd(lib, Sq=1 << 20, H=32, D=128) == SHAPE       # 2^32 elements
     assert _fwd(lib, D=96) == HEADDIM
-    assert _fwd(lib, D=256) == HEADDIM
+    assert _fwd(lib, D=512) == HEADDIM
+    assert _fwd(lib, D=256) in (ARCH, DEVICE)   # head_dim 256: forward only
     assert _fwd(lib, scale=0.0) == SHAPE
     assert _fwd(lib, scale=float("nan")) == SHAPE
     assert _fwd(lib, scale=float("inf")) == SHAPE
@@ -88,6 +89,7 @@ def test_bwd_validation_and_workspace_size():
     assert bwd(ptrs=[None] + p[1:]) == NULLPTR
     assert bwd(B=0) == SHAPE
     assert bwd(D=32) == HEADDIM
+    assert bwd(D=256) == HEADDIM            # head_dim 256 has a forward only
     assert bwd(wl=-3) == WINDOW
     assert bwd(ptrs=p[:6] + [0x7004] + p[7:]) == ALIGN
     assert bwd(wsp=None) == 10
