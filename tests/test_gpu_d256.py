@@ -61,3 +61,30 @@ def test_d256_sampled_rows_long_causal():
     o_d = to_f64(o)[trip[:, 0], trip[:, 2], trip[:, 1]]
     l_d = lse.cpu().numpy().astype(np.float64)[trip[:, 0], trip[:, 1], trip[:, 2]]
     check_fwd(o_d, l_d, o_ref, lse_ref, "d256 sampled rows")
+
+
+def test_d256_bench_workload_sampled_rows():
+    """The benchmark's head_dim 256 workload itself (B1 H16 Sq=Sk=8192 causal,
+    its seed and scale), 1024 seeded (head, row) samples plus the first and last
+    rows of every head, against the oracle row by row."""
+    import torch
+    import bench
+    from exact_attention_156_b200 import attn_fwd, get_last_device_error
+    w = bench.D256_WORKLOAD
+    B, S, H, D = w["B"], w["Sq"], w["H"], w["D"]
+    bits = make_inputs(B, S, S, H, D, w["seed"], w["input_scale"], Hk=w["Hk"])
+    q, k, v = (to_device(bits[n]) for n in ("q", "k", "v"))
+    scale = 1.0 / np.sqrt(D)
+    o, lse = attn_fwd(q, k, v, softmax_scale=scale, causal=True)
+    torch.cuda.synchronize()
+    assert get_last_device_error() == 0
+    rng = np.random.default_rng(9)
+    trip = np.stack([np.zeros(1024, dtype=np.int64), rng.integers(0, H, 1024),
+                     rng.integers(0, S, 1024)], axis=1)
+    edges = np.array([[0, h, r] for h in range(H) for r in (0, S - 1)], dtype=np.int64)
+    trip = np.unique(np.concatenate([trip, edges]), axis=0)
+    o_ref, lse_ref = oracle.attention_forward_rows(f64(bits["q"]), f64(bits["k"]), f64(bits["v"]),
+                                                   trip, scale, 1)
+    o_d = to_f64(o)[trip[:, 0], trip[:, 2], trip[:, 1]]
+    l_d = lse.cpu().numpy().astype(np.float64)[trip[:, 0], trip[:, 1], trip[:, 2]]
+    check_fwd(o_d, l_d, o_ref, lse_ref, "d256 bench workload rows")

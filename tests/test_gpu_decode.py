@@ -45,3 +45,27 @@ def test_decode_against_the_oracle(case):
     o_ref, lse_ref = oracle.attention_decode(f64(bits["q"], fmt), f64(bits["k"], fmt),
                                              f64(bits["v"], fmt), lens, scale, causal)
     check_fwd(to_f64(o), lse.cpu().numpy().astype(np.float64), o_ref, lse_ref, str(case))
+
+
+def test_decode_bench_workload_in_full():
+    """The benchmark's decode workload itself (B8, one new row, H32 Hk8, 8192
+    cached rows, D128, inputs N(0,1)*0.5, the seed bench.py uses), every output
+    row against the oracle, through the same call the benchmark times."""
+    import torch
+    import bench
+    from exact_attention_156_b200 import (attn_decode, attn_decode_workspace_size,
+                                          get_last_device_error)
+    w = bench.DECODE_WORKLOAD
+    B, Sq, H, Hk, S, D = w["B"], w["Sq"], w["H"], w["Hk"], w["Smax"], w["D"]
+    bits = make_inputs(B, Sq, S, H, D, w["seed"], w["input_scale"], Hk=Hk)
+    q, k, v = (to_device(bits[n]) for n in ("q", "k", "v"))
+    seqlens = torch.full((B,), S, dtype=torch.int32, device="cuda")
+    ws = torch.empty(attn_decode_workspace_size(B, Sq, S, H, Hk, D), dtype=torch.uint8,
+                     device="cuda")
+    o, lse = attn_decode(q, k, v, seqlens, causal=bool(w["causal"]), workspace=ws)
+    torch.cuda.synchronize()
+    assert get_last_device_error() == 0
+    o_ref, lse_ref = oracle.attention_decode(f64(bits["q"]), f64(bits["k"]), f64(bits["v"]),
+                                             [S] * B, 1.0 / np.sqrt(D), w["causal"])
+    check_fwd(to_f64(o), lse.cpu().numpy().astype(np.float64), o_ref, lse_ref,
+              "decode bench workload")

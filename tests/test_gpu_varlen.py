@@ -121,3 +121,44 @@ def test_malformed_boundaries_are_reported_and_skipped():
         check_grad(to_f64(got[:100]), ref[name][:100], f"{name} of the valid sequence",
                    floor=1e-3 * top)
         assert torch.all(got[100:] == sentinel), f"{name} rows of malformed sequences written"
+
+
+def test_varlen_bench_workload_sampled_sequences():
+    """The benchmark's packed batch itself (32768 tokens, 31 sequences of
+    138..3872, H32 D128 causal, its seed and scale), run whole through the calls
+    the benchmark times; the longest, the shortest and a middle sequence are
+    checked against the oracle on four heads each (sequences and heads are
+    independent, so their rows, keys and gradients are exact references)."""
+    import torch
+    import bench
+    from exact_attention_156_b200 import attn_bwd_varlen, attn_fwd_varlen, get_last_device_error
+    w = bench.VARLEN_WORKLOAD
+    lengths = bench.varlen_lengths(w)
+    T, H, D = w["total"], w["H"], w["D"]
+    bits = make_inputs(1, T, T, H, D, w["seed"], w["input_scale"], with_dout=True, Hk=w["Hk"])
+    x = {n: bits[n][0] for n in ("q", "k", "v", "do")}
+    q, k, v, do = (_to_dev(x[n], "bf16") for n in ("q", "k", "v", "do"))
+    cu = np.concatenate([[0], np.cumsum(lengths)]).astype(np.int32)
+    cu_d = torch.from_numpy(cu).cuda()
+    Lmax = max(lengths)
+    o, lse = attn_fwd_varlen(q, k, v, cu_d, cu_d, Lmax, Lmax, causal=True)
+    dq, dk, dv = attn_bwd_varlen(q, k, v, o, do, lse, cu_d, cu_d, Lmax, Lmax, causal=True)
+    torch.cuda.synchronize()
+    assert get_last_device_error() == 0
+    order = np.argsort(lengths)
+    picks = sorted({int(order[-1]), int(order[0]), int(order[len(order) // 2])})
+    heads = [0, 9, 21, 31]
+    o_h, lse_h = to_f64(o), lse.cpu().numpy().astype(np.float64)
+    g_h = {n: to_f64(t) for n, t in (("dq", dq), ("dk", dk), ("dv", dv))}
+    for bi in picks:
+        a, z = int(cu[bi]), int(cu[bi + 1])
+        for h in heads:
+            sl = lambda arr: f64(arr[a:z, h:h + 1])
+            ref = oracle.attention_backward_varlen(sl(x["q"]), sl(x["k"]), sl(x["v"]),
+                                                   sl(x["do"]), [0, z - a], [0, z - a],
+                                                   1.0 / np.sqrt(D), 1)
+            what = f"sequence {bi} (length {z - a}) head {h}"
+            check_fwd(o_h[a:z, h:h + 1], lse_h[h:h + 1, a:z].T, ref["o"], ref["lse"].T, what)
+            top = max(np.abs(ref[n]).max() for n in ("dq", "dk", "dv"))
+            for n in ("dq", "dk", "dv"):
+                check_grad(g_h[n][a:z, h:h + 1], ref[n], f"{n} {what}", floor=1e-3 * top)
