@@ -21,10 +21,9 @@
 //    running max is only raised when it grows by more than 2^8, so O is
 //    rescaled rarely (O and l share the stale max, O/l is unchanged);
 //  * warp 4: one thread issues the tcgen05 products; warp 5: one thread loads
-//    Q once (four 128 x 64 boxes) and then the K tiles into a ring of 3 slots
-//    of 32 KB (four 64 x 64 boxes each), warp 6 the V tiles into a ring of 2:
-//    a K slot is refilled as soon as S has read it, so K is fetched three
-//    tiles ahead (one ring of K and V would free K slots only behind P V);
+//    Q once (four 128 x 64 boxes) and then the K tiles into a ring of 2 slots
+//    of 32 KB (four 64 x 64 boxes each), warp 6 the V tiles into a ring of 3
+//    (a K slot is refilled as soon as S has read it; a V slot after P V);
 //  * epilogue: O / l in the input format and LSE = (m + log2 l) ln 2, after a
 //    barrier committed once behind the last P V (with S double-buffered the
 //    per-tile O barrier can be two phases behind when the softmax gets there).
@@ -57,8 +56,8 @@ struct Cfg {
   static constexpr int kBoxes = D / 64;           // 4 boxes across head_dim
   static constexpr int kQBytes = kBoxes * kQBox;  // 64 KB
   static constexpr int kTileBytes = kBoxes * kKVBox;  // 32 KB
-  static constexpr int kKSlots = 3;
-  static constexpr int kVSlots = 2;
+  static constexpr int kKSlots = 2;
+  static constexpr int kVSlots = 3;
   static constexpr int kQOff = 0;
   static constexpr int kKOff = kQBytes;
   static constexpr int kVOff = kKOff + kKSlots * kTileBytes;
