@@ -213,3 +213,44 @@ def test_varlen_validation_and_workspace_size():
     assert bwd(wsp=0x100080) == 10       # not 256-byte aligned
     assert bwd(wsz=ws - 1) == 10
     assert bwd() in (ARCH, DEVICE)
+
+
+def test_binding_refuses_cpu_tensors_on_every_entry_point():
+    """No entry point has a CPU path: CPU tensors are refused in the binding,
+    before the library is called."""
+    import torch
+    from exact_attention_156_b200 import (attn_bwd, attn_bwd_varlen, attn_decode,
+                                          attn_fwd_varlen)
+    q4 = torch.zeros(1, 128, 2, 64, dtype=torch.bfloat16)
+    q3 = torch.zeros(128, 2, 64, dtype=torch.bfloat16)
+    lse2 = torch.zeros(2, 128, dtype=torch.float32)
+    lse3 = torch.zeros(1, 2, 128, dtype=torch.float32)
+    cu = torch.tensor([0, 128], dtype=torch.int32)
+    seq = torch.tensor([128], dtype=torch.int32)
+    with pytest.raises(ValueError, match="CUDA"):
+        attn_bwd(q4, q4, q4, q4, q4, lse3)
+    with pytest.raises(ValueError, match="CUDA"):
+        attn_fwd_varlen(q3, q3, q3, cu, cu, 128, 128)
+    with pytest.raises(ValueError, match="CUDA"):
+        attn_bwd_varlen(q3, q3, q3, q3, q3, lse2, cu, cu, 128, 128)
+    with pytest.raises(ValueError, match="CUDA"):
+        attn_decode(torch.zeros(1, 1, 2, 64, dtype=torch.bfloat16), q4, q4, seq)
+
+
+def test_binding_rejects_mixed_or_unsupported_formats():
+    import torch
+    from exact_attention_156_b200 import attn_fwd
+    q = torch.zeros(1, 128, 2, 64, dtype=torch.float32)
+    with pytest.raises(TypeError, match="bfloat16 or torch.float16"):
+        attn_fwd(q, q, q)
+
+
+def test_binding_checks_varlen_boundaries_on_the_host():
+    """cu_seqlens must be a CUDA int32 vector; the binding refuses anything
+    else before the library (whose device-side checks handle the values)."""
+    import torch
+    from exact_attention_156_b200._binding import _check_cu
+    with pytest.raises(ValueError, match="CUDA"):
+        _check_cu(torch.zeros(3, dtype=torch.int32), "cu_seqlens_q")
+    with pytest.raises(TypeError):
+        _check_cu([0, 1, 2], "cu_seqlens_q")
