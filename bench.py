@@ -49,8 +49,17 @@ VARLEN_WORKLOAD = dict(name="varlen_t32768h32d128_fwdbwd", total=32768, len_lo=1
 # head_dim 256 (forward only): B1 H16 S8192 causal
 D256_WORKLOAD = dict(name="fwd_b1h16s8192d256_causal", B=1, H=16, Hk=16, Sq=8192, Sk=8192,
                      D=256, causal=1, win_left=-1, win_right=-1, input_scale=0.5, seed=1009)
+# forward alone on the attention configurations (name, B, H, S, causal, window, counted
+# GFLOP: 4*B*H*S*S*D, halved for causal; the window row counts visible pairs only)
+FWD_SWEEP = [
+    ("c2_b2h16s2048d128_causal", 2, 16, 2048, 1, (-1, -1), 34.36),
+    ("c3_b1h32s8192d128_causal", 1, 32, 8192, 1, (-1, -1), 549.76),
+    ("c3_b1h32s8192d128", 1, 32, 8192, 0, (-1, -1), 1099.51),
+    ("c4_b1h32s32768d128_causal", 1, 32, 32768, 1, (-1, -1), 8796.09),
+    ("c4_b1h32s32768d128_window4096", 1, 32, 32768, 1, (4096, 0), 2062.09),
+]
 WORKLOADS = {"fwdbwd": WORKLOAD, "gqa": GQA_WORKLOAD, "decode": DECODE_WORKLOAD,
-             "varlen": VARLEN_WORKLOAD, "d256": D256_WORKLOAD}
+             "varlen": VARLEN_WORKLOAD, "d256": D256_WORKLOAD, "fwdsweep": None}
 D256_FWD_METRIC = "attention fwd TFLOPS, head_dim 256, bf16 vs B200 dense BF16 peak"
 DECODE_METRIC = "KV-cache decode: cached K/V bytes read per second"
 FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "hbm_gbs": 6650.0, "source": "fallback"}
@@ -1003,6 +1012,65 @@ def run_fwd_only_reference(args):
     return 0
 
 
+def run_fwd_sweep(args):
+    """Forward alone on each attention configuration (one GPU; seeded inputs
+    N(0,1)*0.5 drawn on the device; K launches after W warm-ups per config).
+    One JSON line; `value` is the C3 causal forward."""
+    import torch
+    from exact_attention_156_b200 import attn_fwd, get_last_device_error
+    rank, world, _ = dist_env()
+    if world > 1:
+        raise SystemExit("--workload fwdsweep runs on one GPU")
+    peaks = load_peaks()
+    peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    gen = torch.Generator(device="cuda")
+    rows = []
+    for name, B, H, S, causal, win, gflop in FWD_SWEEP:
+        gen.manual_seed(1000 + len(rows))
+        q, k, v = ((torch.randn(B, S, H, 128, device="cuda", generator=gen) * 0.5).bfloat16()
+                   for _ in range(3))
+        o = torch.empty_like(q)
+        lse = torch.empty((B, H, S), dtype=torch.float32, device="cuda")
+        step = lambda: attn_fwd(q, k, v, causal=bool(causal), window_size=win, out=o, lse=lse)
+        for _ in range(args.warmup):
+            step()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        sampler = ClockSampler("GPU-" + str(torch.cuda.get_device_properties(0).uuid))
+        sampler.start()
+        e0.record()
+        for _ in range(args.steps):
+            step()
+        e1.record()
+        torch.cuda.synchronize()
+        clocks = sampler.stop()
+        if get_last_device_error() != 0:
+            raise RuntimeError(f"device-side error in {name}")
+        ms = e0.elapsed_time(e1) / args.steps
+        tf = gflop / ms
+        rows.append({"workload": name, "ms": ms, "tflops": tf, "frac": tf / peak,
+                     "l2": "inputs exceed L2" if 3 * q.numel() * 2 > 126e6 else
+                     "inputs fit in L2", "clocks": clocks})
+        del q, k, v, o, lse
+    head = rows[1]
+    print(json.dumps({
+        "metric": "attention forward TFLOP/s per configuration", "value": head["tflops"],
+        "unit": UNIT, "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": head["ms"], "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": "forward alone on C2, C3 (causal, non-causal), C4 (causal, "
+                               "window (4096, 0)); value = C3 causal"},
+        "roofline": {"bound": "tensor", "kernel": "attn_fwd_kernel<128>",
+                     "achieved": head["tflops"], "peak": peak, "unit": UNIT,
+                     "frac": head["tflops"] / peak,
+                     "peak_source": f"{peaks.get('source')} bf16_tflops (burst)",
+                     "traffic": committed_traffic("attn_fwd_kernel",
+                                                  sources_sha(FWD_KERNEL_SOURCES))},
+        "configs": rows, "gpu_launches": len(FWD_SWEEP) * (args.steps + args.warmup)}),
+        flush=True)
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -1016,7 +1084,7 @@ def main(argv=None):
                          "with 8 K/V heads for 32 query heads; decode: KV-cache decode "
                          "(B8 H32 Hk8, 8192 cached rows, one new row); varlen: a packed batch "
                          "of 32768 tokens in sequences of 128..4096; d256: head_dim 256 forward, "
-                         "B1 H16 S8192 causal")
+                         "B1 H16 S8192 causal; fwdsweep: the forward alone on C2-C4")
     ap.add_argument("--no-cpu-baseline", action="store_true",
                     help="skip the timed oracle sample (it adds ~15 s of CPU time)")
     ap.add_argument("--no-e2e", action="store_true",
@@ -1030,6 +1098,12 @@ def main(argv=None):
         return run_varlen_reference(args) if args.impl == "reference" else run_varlen(args)
     if args.workload == "d256":
         return run_fwd_only_reference(args) if args.impl == "reference" else run_fwd_only(args)
+    if args.workload == "fwdsweep":
+        if args.impl == "reference":
+            print(json.dumps({"impl": "reference", "unavailable": "the forward sweep has no "
+                              "oracle arm; the fwdbwd workload carries it"}))
+            return 0
+        return run_fwd_sweep(args)
     if args.impl == "reference":
         return run_reference(args)
     return run_gpu(args)
