@@ -13,7 +13,7 @@ the row maximum subtracted first (section 2.1, third anti-pattern, on
 stability), then the weighted sum of V.  Everything runs in float64 on the
 given (already bf16-rounded) inputs; no tiling, fusion or reordering.
 
-Readings of points the pages leave open (each listed in the design doc):
+Readings of points the pages leave open:
   * scale multiplies the scores: S = scale * Q K^T.  ``softmax_scale=None``
     in the pages' ``flash_attn_func`` call (section 3.3 snippet) means
     1/sqrt(head_dim); callers here always pass it explicitly.
