@@ -20,6 +20,7 @@ from ._binding import (  # noqa: F401
     attn_decode_workspace_size,
     attn_fwd,
     attn_fwd_varlen,
+    decode_split_plan,
     device_timeout_selftest,
     get_last_device_error,
     lib,

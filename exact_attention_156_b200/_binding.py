@@ -73,6 +73,8 @@ def _load() -> ctypes.CDLL:
     lib.attn_bwd_varlen.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i,
                                     i, i, i, f, i, i, i, vp, sz, vp]
     lib.attn_bwd_varlen.restype = i
+    lib.attn_decode_split_plan.argtypes = [i, i, i, i, ctypes.POINTER(i), ctypes.POINTER(i)]
+    lib.attn_decode_split_plan.restype = i
     lib.attn_bwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, i,
                                      i, vp]
     lib.attn_bwd_noalloc.restype = i
@@ -276,6 +278,16 @@ def attn_bwd_stages(q, k, v, out, dout, lse, dq, dk, dv, workspace,
 
 def attn_decode_workspace_size(B: int, Sq: int, Smax: int, H: int, Hk: int, D: int) -> int:
     return int(lib.attn_decode_workspace_size(B, Sq, Smax, H, Hk, D))
+
+
+def decode_split_plan(B: int, Smax: int, Hk: int, num_sms: int):
+    """(splits, tiles per split) attn_decode uses for this shape on a GPU with
+    num_sms SMs (host logic; no device needed)."""
+    ns, tps = ctypes.c_int(), ctypes.c_int()
+    st = lib.attn_decode_split_plan(B, Smax, Hk, num_sms, ctypes.byref(ns), ctypes.byref(tps))
+    if st != 0:
+        raise AttnError(st, "attn_decode_split_plan")
+    return ns.value, tps.value
 
 
 def attn_decode(q, k_cache, v_cache, cache_seqlens, softmax_scale: Optional[float] = None,

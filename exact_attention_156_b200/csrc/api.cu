@@ -992,6 +992,16 @@ attn_status attn_decode(const void* q, const void* k_cache, const void* v_cache,
   });
 }
 
+attn_status attn_decode_split_plan(int B, int Smax, int Hk, int num_sms, int* nsplit,
+                                   int* tiles_per_split) {
+  if (!nsplit || !tiles_per_split) return ATTN_ERR_NULLPTR;
+  if (B < 1 || Smax < 1 || Hk < 1 || num_sms < 1) return ATTN_ERR_SHAPE;
+  const DecodePlan plan = decode_plan(B, Smax, Hk, num_sms);
+  *nsplit = plan.nsplit;
+  *tiles_per_split = plan.tiles_per_split;
+  return ATTN_OK;
+}
+
 attn_status attn_get_last_device_error(void) {
   DeviceState* st = nullptr;
   attn_status s = device_state(&st);

@@ -298,6 +298,18 @@ ATTN_API attn_status attn_bwd_varlen(const void* q, const void* k, const void* v
                                      int win_right, void* workspace, size_t workspace_size,
                                      void* stream);
 
+/*
+ * attn_decode_split_plan - the key-split plan attn_decode uses (host logic
+ * only, no device call): the cache's 128-key tiles are cut into *nsplit splits
+ * of *tiles_per_split tiles, one CTA per (split, K/V head, sequence), chosen to
+ * minimise ceil(CTAs / num_sms) x (tiles_per_split + 3) with at least two tiles
+ * per split when the cache has more than one tile.  attn_decode passes the
+ * current device's SM count.  Errors: ATTN_ERR_NULLPTR, ATTN_ERR_SHAPE (an
+ * argument < 1).
+ */
+ATTN_API attn_status attn_decode_split_plan(int B, int Smax, int Hk, int num_sms, int* nsplit,
+                                            int* tiles_per_split);
+
 /* attn_status_string - static English text for a status code (never NULL). */
 ATTN_API const char* attn_status_string(attn_status s);
 

@@ -254,3 +254,38 @@ def test_binding_checks_varlen_boundaries_on_the_host():
         _check_cu(torch.zeros(3, dtype=torch.int32), "cu_seqlens_q")
     with pytest.raises(TypeError):
         _check_cu([0, 1, 2], "cu_seqlens_q")
+
+
+def _plan(lib, B, Smax, Hk, sms):
+    ns, tps = ctypes.c_int(), ctypes.c_int()
+    st = lib.attn_decode_split_plan(B, Smax, Hk, sms, ctypes.byref(ns), ctypes.byref(tps))
+    return st, ns.value, tps.value
+
+
+def test_decode_split_plan():
+    """The decode planner (host logic): splits cover the cache, have at least
+    two tiles unless the cache has one, never exceed the split count the
+    workspace is sized for, and minimise the stated cost; brute force over every
+    split length for a range of shapes and SM counts."""
+    import math
+    lib = ctypes.CDLL(LIB)
+    assert _plan(lib, 8, 8192, 8, 148) == (OK, 2, 32)        # the bench workload: 128 CTAs
+    from exact_attention_156_b200 import decode_split_plan
+    assert decode_split_plan(8, 8192, 8, 148) == (2, 32)
+    assert _plan(lib, 0, 8192, 8, 148)[0] == SHAPE
+    assert _plan(lib, 1, 8192, 8, 0)[0] == SHAPE
+    assert lib.attn_decode_split_plan(1, 1, 1, 1, None, None) == NULLPTR
+    for B in (1, 2, 3, 8, 16, 64):
+        for Smax in (1, 127, 128, 129, 1000, 4096, 8192, 32768):
+            for Hk in (1, 2, 8):
+                for sms in (1, 132, 148):
+                    st, ns, tps = _plan(lib, B, Smax, Hk, sms)
+                    assert st == OK
+                    tiles = math.ceil(Smax / 128)
+                    assert ns * tps >= tiles and (ns - 1) * tps < tiles
+                    assert tps >= (2 if tiles > 1 else 1)
+                    max_splits = (tiles + 1) // 2 if tiles > 1 else 1
+                    assert 1 <= ns <= max_splits
+                    cost = lambda t: math.ceil(B * Hk * math.ceil(tiles / t) / sms) * (t + 3)
+                    best = min(cost(t) for t in range(2 if tiles > 1 else 1, tiles + 1))
+                    assert cost(tps) == best, (B, Smax, Hk, sms, ns, tps)
