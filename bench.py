@@ -58,6 +58,18 @@ FWD_SWEEP = [
     ("c4_b1h32s32768d128_causal", 1, 32, 32768, 1, (-1, -1), 8796.09),
     ("c4_b1h32s32768d128_window4096", 1, 32, 32768, 1, (4096, 0), 2062.09),
 ]
+# the forward alone on the causal 7B-decoder-like layer (B1 H32 Sq=Sk=8192 D128,
+# inputs N(0,1)*0.5), timed by itself inside the default run
+C3_CAUSAL = dict(name="c3_b1h32s8192d128_causal_fwd", B=1, H=32, Hk=32, Sq=8192, Sk=8192,
+                 D=128, causal=1, win_left=-1, win_right=-1, input_scale=0.5, seed=1003)
+C3_LAUNCHES = 200
+# the two small configurations the oracle finishes in full (forward)
+ORACLE_FULL = [
+    dict(name="c1_b1h2s128d64", B=1, H=2, Hk=2, Sq=128, Sk=128, D=64, causal=0, win_left=-1,
+         win_right=-1, input_scale=1.0, seed=1001),
+    dict(name="c2_b2h16s2048d128_causal", B=2, H=16, Hk=16, Sq=2048, Sk=2048, D=128, causal=1,
+         win_left=-1, win_right=-1, input_scale=1.0, seed=1002),
+]
 WORKLOADS = {"fwdbwd": WORKLOAD, "gqa": GQA_WORKLOAD, "decode": DECODE_WORKLOAD,
              "varlen": VARLEN_WORKLOAD, "d256": D256_WORKLOAD, "fwdsweep": None}
 D256_FWD_METRIC = "attention fwd TFLOPS, head_dim 256, bf16 vs B200 dense BF16 peak"
@@ -275,6 +287,63 @@ def cpu_baseline(w, budget_s: float = 15.0):
                       f"{tot_s:.1f} s total; flops counted as 14*D per visible pair"}
 
 
+def oracle_full_forward():
+    """The oracle's forward over the two small configurations in full (every
+    row of every head), each timed once; TFLOP/s by the metric's convention."""
+    import oracle
+    from synth import bits_to_f32, make_inputs
+    out = []
+    for w in ORACLE_FULL:
+        bits = make_inputs(w["B"], w["Sq"], w["Sk"], w["H"], w["D"], w["seed"], w["input_scale"])
+        x = {n: bits_to_f32(bits[n]) for n in ("q", "k", "v")}
+        t0 = time.perf_counter()
+        oracle.attention_forward(x["q"], x["k"], x["v"], 1.0 / math.sqrt(w["D"]), w["causal"])
+        dt = time.perf_counter() - t0
+        out.append({"workload": w["name"], "seconds": dt,
+                    "tflops": fwd_flops(w) / dt / 1e12, "cores": blas_threads(),
+                    "sample": "whole configuration, forward, float64 numpy"})
+    return out
+
+
+def time_c3_causal_forward(device, stream, launches: int = C3_LAUNCHES, warmup: int = 5):
+    """The causal forward of B1 H32 Sq=Sk=8192 D128 (inputs N(0,1)*0.5, 192 MiB,
+    larger than L2) launched back to back, with its own clock samples."""
+    import torch
+    from exact_attention_156_b200 import attn_fwd, get_last_device_error
+    from synth import make_inputs
+    w = C3_CAUSAL
+    bits = make_inputs(w["B"], w["Sq"], w["Sk"], w["H"], w["D"], w["seed"], w["input_scale"])
+    q, k, v = (torch.from_numpy(bits[n].view("int16")).view(torch.bfloat16).to(device)
+               for n in ("q", "k", "v"))
+    o = torch.empty_like(q)
+    lse = torch.empty((w["B"], w["H"], w["Sq"]), dtype=torch.float32, device=device)
+    step = lambda: attn_fwd(q, k, v, causal=True, out=o, lse=lse, stream=stream)
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize(device)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler("GPU-" + str(torch.cuda.get_device_properties(device).uuid))
+    sampler.start()
+    e0.record(stream)
+    for _ in range(launches):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(device)
+    clocks = sampler.stop()
+    if get_last_device_error() != 0:
+        raise RuntimeError("device-side error in the C3 causal forward")
+    ms = e0.elapsed_time(e1) / launches
+    peaks = load_peaks()
+    peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    tf = fwd_flops(w) / (ms * 1e-3) / 1e12
+    del q, k, v, o, lse
+    return {"workload": f"{w['name']}: forward alone, B=1 H=32 Sq=Sk=8192 D=128 causal bf16, "
+                        f"inputs N(0,1)*0.5 (192 MiB, no L2 flush)",
+            "kernel": "attn_fwd_kernel<128>", "launches": launches, "warmup": warmup,
+            "ms": ms, "tflops": tf, "peak": peak, "frac": tf / peak,
+            "peak_source": f"{peaks.get('source')} bf16_tflops (burst)", "clocks": clocks}
+
+
 def run_reference(args):
     rank, world, _ = dist_env()
     if rank != 0:
@@ -423,6 +492,13 @@ def run_gpu(args):
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
                "steps": e2e_steps}
 
+    c3 = None
+    if args.workload == "fwdbwd" and args.dtype == "bf16" and not args.no_c3:
+        barrier(device)
+        c3 = time_c3_causal_forward(device, stream)
+        launches += c3["launches"] + c3["warmup"]
+        barrier(device)
+
     peaks = load_peaks()
     peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
     bwd_main_tflops = bwd_flops(w) / (per_kernel[2] * 1e-3) / 1e12
@@ -455,8 +531,12 @@ def run_gpu(args):
         "gpu_launches": launches,
         "clocks": clocks,
     }
+    if c3 is not None:
+        line["fwd_c3_causal"] = c3
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w)
+        if args.workload == "fwdbwd":
+            line["cpu_baseline"]["full_configs"] = oracle_full_forward()
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -1087,6 +1167,8 @@ def main(argv=None):
                          "B1 H16 S8192 causal; fwdsweep: the forward alone on C2-C4")
     ap.add_argument("--no-cpu-baseline", action="store_true",
                     help="skip the timed oracle sample (it adds ~15 s of CPU time)")
+    ap.add_argument("--no-c3", action="store_true",
+                    help="skip the standalone C3 causal forward leg of the default workload")
     ap.add_argument("--no-e2e", action="store_true",
                     help="skip the host-buffer end-to-end leg (fewer launches under a profiler)")
     args = ap.parse_args(argv)

@@ -25,6 +25,7 @@
 #include <stdint.h>
 
 #include "ptx.cuh"
+#include "ptx_pair.cuh"
 
 using namespace attn156;
 

@@ -222,6 +222,10 @@ ATTN_API attn_status attn_bwd_dq_finalize_ex(void* dq, int B, int Sq, int H, int
  *    call's contents (each call re-initialises what it needs).  Calls whose
  *    execution overlaps on the GPU (concurrent streams) race on it and give
  *    wrong results: serialise them.
+ *  - The looked-up address is kept for the life of the process.  The library
+ *    does not survive cudaDeviceReset: a reset destroys the context that holds
+ *    the array (and the library's device error word), so a process that
+ *    resets a device must not call this library on that device afterwards.
  */
 #define ATTN_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)
 ATTN_API attn_status attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* o,

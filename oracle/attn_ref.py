@@ -58,18 +58,20 @@ def _f64(x):
 
 
 def visible_mask(Sq: int, Sk: int, causal: int, win_left: int = -1,
-                 win_right: int = -1) -> np.ndarray:
-    """Boolean (Sq, Sk) matrix: True where key j is visible to query i.
+                 win_right: int = -1, rows=None) -> np.ndarray:
+    """Boolean (Sq, Sk) matrix: True where key j is visible to query i (only
+    the given query rows, in that order, when ``rows`` is given).
 
     Causal mask: FlashAttention-2 overview (lshu.cn), section 4.2 problem 4
     (upper-triangular mask, each token sees only earlier tokens); window:
     flash-attn install guide (yfxerp.com), section 1 (``window_size``).
     Alignment and inclusive bounds are this oracle's stated reading.
     """
-    i = np.arange(Sq, dtype=np.int64)[:, None]
+    i = (np.arange(Sq, dtype=np.int64) if rows is None
+         else np.asarray(rows, dtype=np.int64))[:, None]
     j = np.arange(Sk, dtype=np.int64)[None, :]
     delta = Sk - Sq
-    vis = np.ones((Sq, Sk), dtype=bool)
+    vis = np.ones((i.shape[0], Sk), dtype=bool)
     if causal:
         vis &= j <= i + delta
     if win_left >= 0:
@@ -100,7 +102,7 @@ def _softmax_rows(S: np.ndarray):
 def _scores(qh, kh, scale, rows, Sq, Sk, causal, wl, wr):
     """scale * Q K^T for the given query rows of one head, masked with -inf."""
     S = scale * (qh @ kh.T)
-    vis = visible_mask(Sq, Sk, causal, wl, wr)[rows]
+    vis = visible_mask(Sq, Sk, causal, wl, wr, rows=rows)
     return np.where(vis, S, -np.inf)
 
 
