@@ -71,12 +71,25 @@ ORACLE_FULL = [
          win_left=-1, win_right=-1, input_scale=1.0, seed=1002),
 ]
 WORKLOADS = {"fwdbwd": WORKLOAD, "gqa": GQA_WORKLOAD, "decode": DECODE_WORKLOAD,
-             "varlen": VARLEN_WORKLOAD, "d256": D256_WORKLOAD, "fwdsweep": None}
+             "varlen": VARLEN_WORKLOAD, "d256": D256_WORKLOAD, "d256fwd": D256_WORKLOAD,
+             "fwdsweep": None}
 D256_FWD_METRIC = "attention fwd TFLOPS, head_dim 256, bf16 vs B200 dense BF16 peak"
+D256_METRIC = "attention fwd+bwd TFLOPS, head_dim 256, bf16 vs B200 dense BF16 peak"
 DECODE_METRIC = "KV-cache decode: cached K/V bytes read per second"
 FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "hbm_gbs": 6650.0, "source": "fallback"}
 BWD_KERNEL_SOURCES = ["bwd_sm100.cuh", "ptx.cuh", "common.cuh"]
 FWD_KERNEL_SOURCES = ["fwd_sm100.cuh", "ptx.cuh", "common.cuh"]
+BWD256_KERNEL_SOURCES = ["bwd256_sm100.cuh", "ptx.cuh", "ptx_d256.cuh", "common.cuh"]
+FWD256_KERNEL_SOURCES = ["fwd256_sm100.cuh", "ptx.cuh", "common.cuh"]
+
+
+def kernel_names(w):
+    """(metric, forward kernel, its sources, backward main kernel, its sources) of a workload."""
+    if w["D"] == 256:
+        return (D256_METRIC, "attn_fwd_d256_kernel", FWD256_KERNEL_SOURCES,
+                "attn_bwd_d256_kernel", BWD256_KERNEL_SOURCES)
+    return (METRIC, f"attn_fwd_kernel<{w['D']}>", FWD_KERNEL_SOURCES,
+            f"attn_bwd_main_kernel<{w['D']}>", BWD_KERNEL_SOURCES)
 ORACLE_ROWS_PER_SAMPLE = 512
 
 
@@ -359,7 +372,7 @@ def run_reference(args):
         tot_f += fl
     value = tot_f / tot_s / 1e12
     line = {
-        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "impl": "reference", "metric": kernel_names(w)[0], "value": value, "unit": UNIT, "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": tot_s / args.steps * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic",
@@ -501,6 +514,7 @@ def run_gpu(args):
 
     peaks = load_peaks()
     peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    metric, fwd_name, fwd_src, bwd_name, bwd_src = kernel_names(w)
     bwd_main_tflops = bwd_flops(w) / (per_kernel[2] * 1e-3) / 1e12
     fwd_tflops = fwd_flops(w) / (per_kernel[0] * 1e-3) / 1e12
     kernels = {
@@ -511,22 +525,22 @@ def run_gpu(args):
         "bwd_dq_finalize": {"ms": per_kernel[3]},
     }
     line = {
-        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "metric": metric, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": args.dtype, "data": "synthetic",
         "config": config_dict(w),
-        "roofline": {"bound": "tensor", "kernel": "attn_bwd_main_kernel<128>",
+        "roofline": {"bound": "tensor", "kernel": bwd_name,
                      "achieved": bwd_main_tflops, "peak": peak, "unit": "TFLOP/s",
                      "frac": bwd_main_tflops / peak,
                      "peak_source": f"{peaks.get('source')} bf16_tflops (burst)",
-                     "traffic": committed_traffic(traffic_key("attn_bwd_main_kernel", w, args.dtype),
-                                                  sources_sha(BWD_KERNEL_SOURCES))},
+                     "traffic": committed_traffic(traffic_key(bwd_name.split("<")[0], w, args.dtype),
+                                                  sources_sha(bwd_src))},
         "kernels": kernels,
-        "fwd_roofline": {"bound": "tensor", "kernel": "attn_fwd_kernel<128>",
+        "fwd_roofline": {"bound": "tensor", "kernel": fwd_name,
                          "achieved": fwd_tflops, "peak": peak, "unit": "TFLOP/s",
                          "frac": fwd_tflops / peak,
-                         "traffic": committed_traffic(traffic_key("attn_fwd_kernel", w, args.dtype),
-                                                      sources_sha(FWD_KERNEL_SOURCES))},
+                         "traffic": committed_traffic(traffic_key(fwd_name.split("<")[0], w, args.dtype),
+                                                      sources_sha(fwd_src))},
         "e2e": e2e,
         "gpu_launches": launches,
         "clocks": clocks,
@@ -1163,8 +1177,9 @@ def main(argv=None):
                     help="fwdbwd: the headline fwd+bwd workload (default); gqa: the same sizes "
                          "with 8 K/V heads for 32 query heads; decode: KV-cache decode "
                          "(B8 H32 Hk8, 8192 cached rows, one new row); varlen: a packed batch "
-                         "of 32768 tokens in sequences of 128..4096; d256: head_dim 256 forward, "
-                         "B1 H16 S8192 causal; fwdsweep: the forward alone on C2-C4")
+                         "of 32768 tokens in sequences of 128..4096; d256: head_dim 256 forward + "
+                         "backward, B1 H16 S8192 causal; d256fwd: its forward alone; fwdsweep: "
+                         "the forward alone on C2-C4")
     ap.add_argument("--no-cpu-baseline", action="store_true",
                     help="skip the timed oracle sample (it adds ~15 s of CPU time)")
     ap.add_argument("--no-c3", action="store_true",
@@ -1178,7 +1193,7 @@ def main(argv=None):
         return run_decode_reference(args) if args.impl == "reference" else run_decode(args)
     if args.workload == "varlen":
         return run_varlen_reference(args) if args.impl == "reference" else run_varlen(args)
-    if args.workload == "d256":
+    if args.workload == "d256fwd":
         return run_fwd_only_reference(args) if args.impl == "reference" else run_fwd_only(args)
     if args.workload == "fwdsweep":
         if args.impl == "reference":

@@ -13,6 +13,7 @@
 #include <type_traits>
 
 #include "../../include/attn.h"
+#include "bwd256_sm100.cuh"
 #include "bwd_sm100.cuh"
 #include "decode_sm100.cuh"
 #include "fwd256_sm100.cuh"
@@ -97,6 +98,10 @@ attn_status device_state(DeviceState** out) {
           ok = ok && set_smem(dec::t16::attn_decode_t16_kernel<E>, dec::t16::Cfg::kSmemBytes) ==
                          cudaSuccess;
       };
+      ok = ok &&
+           set_smem(bwd256::attn_bwd_d256_kernel<ElemBF16>, bwd256::Cfg::kSmemBytes) ==
+               cudaSuccess &&
+           set_smem(bwd256::attn_bwd_d256_kernel<ElemF16>, bwd256::Cfg::kSmemBytes) == cudaSuccess;
       prepare(std::integral_constant<int, 64>{}, ElemBF16{});
       prepare(std::integral_constant<int, 128>{}, ElemBF16{});
       prepare(std::integral_constant<int, 64>{}, ElemF16{});
@@ -280,9 +285,10 @@ attn_status launch_bwd_pre(const void* o, const void* dout, const float* lse, in
                            int H, const Workspace& w, cudaStream_t stream) {
   const long long rows = (long long)B * H * w.Sq_pad;
   const unsigned blocks = unsigned((rows + 7) / 8);
+  // head_dim 256 writes dQ rows whole (no reduce-add), so its accumulator needs no clearing
   bwd::attn_bwd_pre_kernel<D, E><<<blocks, 256, 0, stream>>>(
       static_cast<const uint16_t*>(o), static_cast<const uint16_t*>(dout), lse, w.nlse2,
-      w.ndelta, w.dq_acc, B, H, Sq, w.Sq_pad);
+      w.ndelta, D == 256 ? nullptr : w.dq_acc, B, H, Sq, w.Sq_pad);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_LAUNCH;
 }
 
@@ -328,6 +334,51 @@ attn_status launch_bwd_main(const DeviceState& st, const void* q, const void* k,
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_LAUNCH;
 }
 
+// head_dim 256 backward: one launch of dK, dV and dQ tiles (see bwd256_sm100.cuh).
+template <class E>
+attn_status launch_bwd_main_d256(const DeviceState& st, const void* q, const void* k,
+                                 const void* v, const void* dout, void* dk, void* dv, int B,
+                                 int Sq, int Sk, int H, int Hk, float scale, int causal,
+                                 int win_left, int win_right, const Workspace& w,
+                                 cudaStream_t stream) {
+  constexpr CUtensorMapDataType dt = tmap_type<E>();
+  alignas(64) CUtensorMap q128, k128, v128, do128, q64, k64, v64, do64;
+  if (make_map(&q128, q, B, Sq, H, 256, dt, 128) != ATTN_OK ||
+      make_map(&k128, k, B, Sk, Hk, 256, dt, 128) != ATTN_OK ||
+      make_map(&v128, v, B, Sk, Hk, 256, dt, 128) != ATTN_OK ||
+      make_map(&do128, dout, B, Sq, H, 256, dt, 128) != ATTN_OK ||
+      make_map(&q64, q, B, Sq, H, 256, dt, 64) != ATTN_OK ||
+      make_map(&k64, k, B, Sk, Hk, 256, dt, 64) != ATTN_OK ||
+      make_map(&v64, v, B, Sk, Hk, 256, dt, 64) != ATTN_OK ||
+      make_map(&do64, dout, B, Sq, H, 256, dt, 64) != ATTN_OK)
+    return ATTN_ERR_LAUNCH;
+  bwd256::Params p;
+  p.dk = static_cast<uint16_t*>(dk);
+  p.dv = static_cast<uint16_t*>(dv);
+  p.dq_acc = w.dq_acc;
+  p.nlse2 = w.nlse2;
+  p.ndelta = w.ndelta;
+  p.B = B;
+  p.H = H;
+  p.Hk = Hk;
+  p.Sq = Sq;
+  p.Sk = Sk;
+  p.Sq_pad = w.Sq_pad;
+  p.n_ktiles = (Sk + bwd256::BR - 1) / bwd256::BR;
+  p.n_qtiles = (Sq + bwd256::BR - 1) / bwd256::BR;
+  p.scale = scale;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.causal = causal ? 1 : 0;
+  p.win_left = win_left;
+  p.win_right = win_right;
+  p.err = st.err;
+  p.timeout_ns = kTimeoutNs;
+  const dim3 grid(2 * p.n_ktiles + p.n_qtiles, H, B);
+  bwd256::attn_bwd_d256_kernel<E><<<grid, bwd256::kThreads, bwd256::Cfg::kSmemBytes, stream>>>(
+      q128, k128, v128, do128, q64, k64, v64, do64, p);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_LAUNCH;
+}
+
 template <int D, class E>
 attn_status launch_bwd_dq(void* dq, int B, int Sq, int H, float scale, const Workspace& w,
                           cudaStream_t stream) {
@@ -349,6 +400,31 @@ attn_status dispatch(int D, int dtype, F&& f) {
                  : f(std::integral_constant<int, 128>{}, ElemBF16{});
 }
 
+// As dispatch, with head_dim 256 too (the entry points whose kernels have a
+// head_dim 256 form: the forward and the backward stages).
+template <class F>
+attn_status dispatch_d256(int D, int dtype, F&& f) {
+  if (D == 256)
+    return dtype == ATTN_DTYPE_F16 ? f(std::integral_constant<int, 256>{}, ElemF16{})
+                                   : f(std::integral_constant<int, 256>{}, ElemBF16{});
+  return dispatch(D, dtype, f);
+}
+
+// The backward's main stage for any supported head_dim.
+template <int D, class E>
+attn_status launch_bwd_main_any(const DeviceState& st, const void* q, const void* k,
+                                const void* v, const void* dout, void* dk, void* dv, int B,
+                                int Sq, int Sk, int H, int Hk, float scale, int causal,
+                                int win_left, int win_right, const Workspace& w,
+                                cudaStream_t cs) {
+  if constexpr (D == 256)
+    return launch_bwd_main_d256<E>(st, q, k, v, dout, dk, dv, B, Sq, Sk, H, Hk, scale, causal,
+                                   win_left, win_right, w, cs);
+  else
+    return launch_bwd_main<D, E>(st, q, k, v, dout, dk, dv, B, Sq, Sk, H, Hk, scale, causal,
+                                 win_left, win_right, w, cs);
+}
+
 attn_status check_dtype(int dtype) {
   return (dtype == ATTN_DTYPE_BF16 || dtype == ATTN_DTYPE_F16) ? ATTN_OK : ATTN_ERR_DTYPE;
 }
@@ -359,13 +435,13 @@ attn_status run_backward(const DeviceState& st, const void* q, const void* k, co
                          void* dv, int B, int Sq, int Sk, int H, int Hk, int D, int dtype,
                          float scale, int causal, int win_left, int win_right, const Workspace& w,
                          cudaStream_t cs) {
-  return dispatch(D, dtype, [&](auto d, auto e) {
+  return dispatch_d256(D, dtype, [&](auto d, auto e) {
     constexpr int DD = decltype(d)::value;
     using E = decltype(e);
     attn_status s = launch_bwd_pre<DD, E>(o, dout, lse, B, Sq, H, w, cs);
     if (s == ATTN_OK)
-      s = launch_bwd_main<DD, E>(st, q, k, v, dout, dk, dv, B, Sq, Sk, H, Hk, scale, causal,
-                                 win_left, win_right, w, cs);
+      s = launch_bwd_main_any<DD, E>(st, q, k, v, dout, dk, dv, B, Sq, Sk, H, Hk, scale, causal,
+                                     win_left, win_right, w, cs);
     if (s == ATTN_OK) s = launch_bwd_dq<DD, E>(dq, B, Sq, H, scale, w, cs);
     return s;
   });
@@ -685,7 +761,8 @@ const char* attn_status_string(attn_status s) {
     case ATTN_OK: return "ok";
     case ATTN_ERR_NULLPTR: return "a required pointer is NULL";
     case ATTN_ERR_SHAPE: return "bad shape or scale (B, H, Sq, Sk >= 1, sizes < 2^31, scale finite > 0)";
-    case ATTN_ERR_HEADDIM: return "head_dim must be 64 or 128";
+    case ATTN_ERR_HEADDIM:
+      return "head_dim must be 64 or 128 (or 256 for the dense forward and backward)";
     case ATTN_ERR_ALIGN: return "tensor pointers must be 16-byte aligned";
     case ATTN_ERR_WINDOW: return "window sizes must be -1 (unbounded) or >= 0";
     case ATTN_ERR_ARCH: return "the current device is not compute capability 10.0 (sm_100a)";
@@ -740,7 +817,7 @@ attn_status attn_fwd(const void* q, const void* k, const void* v, void* o, float
 }
 
 size_t attn_bwd_workspace_size(int B, int Sq, int H, int D) {
-  if (B < 1 || Sq < 1 || H < 1 || (D != 64 && D != 128)) return 0;
+  if (B < 1 || Sq < 1 || H < 1 || (D != 64 && D != 128 && D != 256)) return 0;
   return workspace_bytes(B, Sq, H, D);
 }
 
@@ -750,7 +827,7 @@ attn_status attn_bwd_ex(const void* q, const void* k, const void* v, const void*
                         int win_left, int win_right, void* workspace, size_t workspace_size,
                         void* stream) {
   if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv) return ATTN_ERR_NULLPTR;
-  attn_status s = check_common(B, Sq, Sk, H, D, scale, win_left, win_right, Hk);
+  attn_status s = check_common(B, Sq, Sk, H, D, scale, win_left, win_right, Hk, true);
   if (s != ATTN_OK) return s;
   if ((s = check_dtype(dtype)) != ATTN_OK) return s;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) ||
@@ -846,7 +923,7 @@ attn_status attn_bwd_preprocess_ex(const void* o, const void* dout, const float*
                                    int Sq, int H, int D, int dtype, void* workspace,
                                    size_t workspace_size, void* stream) {
   if (!o || !dout || !lse) return ATTN_ERR_NULLPTR;
-  attn_status s = check_common(B, Sq, 1, H, D, 1.0f, -1, -1);
+  attn_status s = check_common(B, Sq, 1, H, D, 1.0f, -1, -1, -1, true);
   if (s != ATTN_OK) return s;
   if ((s = check_dtype(dtype)) != ATTN_OK) return s;
   if (!aligned16(o) || !aligned16(dout) || (reinterpret_cast<uintptr_t>(lse) & 3u))
@@ -859,7 +936,7 @@ attn_status attn_bwd_preprocess_ex(const void* o, const void* dout, const float*
   if (!all_on_device({o, dout, lse, workspace})) return ATTN_ERR_DEVICE;
   const Workspace w = carve(workspace, B, Sq, H, D);
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
-  return dispatch(D, dtype, [&](auto d, auto e) {
+  return dispatch_d256(D, dtype, [&](auto d, auto e) {
     return launch_bwd_pre<decltype(d)::value, decltype(e)>(o, dout, lse, B, Sq, H, w, cs);
   });
 }
@@ -876,7 +953,7 @@ attn_status attn_bwd_main_ex(const void* q, const void* k, const void* v, const 
                              int dtype, float scale, int causal, int win_left, int win_right,
                              void* workspace, size_t workspace_size, void* stream) {
   if (!q || !k || !v || !dout || !dk || !dv) return ATTN_ERR_NULLPTR;
-  attn_status s = check_common(B, Sq, Sk, H, D, scale, win_left, win_right, Hk);
+  attn_status s = check_common(B, Sq, Sk, H, D, scale, win_left, win_right, Hk, true);
   if (s != ATTN_OK) return s;
   if ((s = check_dtype(dtype)) != ATTN_OK) return s;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dout) || !aligned16(dk) ||
@@ -890,8 +967,8 @@ attn_status attn_bwd_main_ex(const void* q, const void* k, const void* v, const 
   if (!all_on_device({q, k, v, dout, dk, dv, workspace})) return ATTN_ERR_DEVICE;
   const Workspace w = carve(workspace, B, Sq, H, D);
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
-  return dispatch(D, dtype, [&](auto d, auto e) {
-    return launch_bwd_main<decltype(d)::value, decltype(e)>(*st, q, k, v, dout, dk, dv, B, Sq,
+  return dispatch_d256(D, dtype, [&](auto d, auto e) {
+    return launch_bwd_main_any<decltype(d)::value, decltype(e)>(*st, q, k, v, dout, dk, dv, B, Sq,
                                                             Sk, H, Hk, scale, causal, win_left,
                                                             win_right, w, cs);
   });
@@ -909,7 +986,7 @@ attn_status attn_bwd_dq_finalize_ex(void* dq, int B, int Sq, int H, int D, int d
                                     float scale, void* workspace, size_t workspace_size,
                                     void* stream) {
   if (!dq) return ATTN_ERR_NULLPTR;
-  attn_status s = check_common(B, Sq, 1, H, D, scale, -1, -1);
+  attn_status s = check_common(B, Sq, 1, H, D, scale, -1, -1, -1, true);
   if (s != ATTN_OK) return s;
   if ((s = check_dtype(dtype)) != ATTN_OK) return s;
   if (!aligned16(dq)) return ATTN_ERR_ALIGN;
@@ -921,7 +998,7 @@ attn_status attn_bwd_dq_finalize_ex(void* dq, int B, int Sq, int H, int D, int d
   if (!all_on_device({dq, workspace})) return ATTN_ERR_DEVICE;
   const Workspace w = carve(workspace, B, Sq, H, D);
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
-  return dispatch(D, dtype, [&](auto d, auto e) {
+  return dispatch_d256(D, dtype, [&](auto d, auto e) {
     return launch_bwd_dq<decltype(d)::value, decltype(e)>(dq, B, Sq, H, scale, w, cs);
   });
 }
@@ -937,7 +1014,7 @@ attn_status attn_bwd_noalloc(const void* q, const void* k, const void* v, const 
                              int B, int Sq, int Sk, int H, int D, float scale, int causal,
                              int win_left, int win_right, void* stream) {
   if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv) return ATTN_ERR_NULLPTR;
-  attn_status s = check_common(B, Sq, Sk, H, D, scale, win_left, win_right);
+  attn_status s = check_common(B, Sq, Sk, H, D, scale, win_left, win_right, -1, true);
   if (s != ATTN_OK) return s;
   if (workspace_bytes(B, Sq, H, D) > ATTN_NOALLOC_SCRATCH_BYTES) return ATTN_ERR_SCRATCH;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) ||

@@ -145,9 +145,14 @@ __global__ void __launch_bounds__(256) attn_bwd_pre_kernel(
   float dot = 0.f;
   if (i < Sq) {
     const size_t base = ((size_t(b) * Sq + i) * H + h) * D;
-    constexpr int kPer = D / 32;  // 16-bit elements per lane (2 or 4)
+    constexpr int kPer = D / 32;  // 16-bit elements per lane (2, 4 or 8)
     uint32_t ow[kPer / 2], dw[kPer / 2];
-    if constexpr (kPer == 4) {
+    if constexpr (kPer == 8) {
+      const uint4 ov = *reinterpret_cast<const uint4*>(o + base + lane * 8);
+      const uint4 dv = *reinterpret_cast<const uint4*>(dout + base + lane * 8);
+      ow[0] = ov.x; ow[1] = ov.y; ow[2] = ov.z; ow[3] = ov.w;
+      dw[0] = dv.x; dw[1] = dv.y; dw[2] = dv.z; dw[3] = dv.w;
+    } else if constexpr (kPer == 4) {
       const uint2 ov = *reinterpret_cast<const uint2*>(o + base + lane * 4);
       const uint2 dv = *reinterpret_cast<const uint2*>(dout + base + lane * 4);
       ow[0] = ov.x; ow[1] = ov.y;
@@ -177,6 +182,8 @@ __global__ void __launch_bounds__(256) attn_bwd_pre_kernel(
     nlse2[r] = nl2;
     ndelta[r] = -dot;
   }
+  // (no accumulator to clear when dQ is written whole rather than reduced into)
+  if (dq_acc == nullptr) return;
   float4* acc = reinterpret_cast<float4*>(dq_acc + (size_t(bh) * Sq_pad + i) * D);
   for (int c = lane; c < D / 4; c += 32) acc[c] = make_float4(0.f, 0.f, 0.f, 0.f);
 }

@@ -10,7 +10,7 @@
 // tensor-memory columns, so a CTA owns one 128-row query tile, and the other
 // 256 columns hold two 128-key score buffers, S0 and S1:
 //   S(t) = Q K_t^T     (M = 128, N = 128, K = 256: two chains of 8 steps)
-//   O   += P(t) V_t    (M = 128, N = 2 x 128, K = 128: P read from tensor memory)
+//   O   += P(t) V_t    (M = 128, N = 256, K = 128: P read from tensor memory)
 // The tensor core computes S(t + 1) while the softmax works on S(t), and per
 // key tile the products (2048 tensor-core cycles) outlast the softmax, so the
 // tensor core, not the exponentials, sets the pace.  Tensor memory: S0 [0,128),
@@ -26,8 +26,13 @@
 //    128 columns of O;
 //  * warp 8: one thread issues the tcgen05 products; warp 9: one thread loads
 //    Q once (four 128 x 64 boxes) and then, per key tile, the halves
-//    K[:, 0:128], K[:, 128:256], V[:, 0:128], V[:, 128:256] into a ring of five
-//    32 KB slots (a slot is handed back as soon as the product reading it is done);
+//    K[:, 0:128], K[:, 128:256], V[:, 0:128], V[:, 128:256] into a ring of four
+//    32 KB slots in the order the products read them (a slot is handed back as
+//    soon as the product reading it is done).  With four slots the two halves
+//    of every V tile land in adjacent slots, so P V is one N = 256 product per
+//    16 keys: a tensor-memory A operand costs a fixed ~107 cycles per
+//    instruction up to N = 128 (measured), so two N = 128 halves would take
+//    1.6x as long as one N = 256 product;
 //  * epilogue: O / l in the input format and LSE = (m + log2 l) ln 2, after a
 //    barrier committed once behind the last P V.
 #pragma once
@@ -58,7 +63,7 @@ struct Cfg {
   static constexpr int kBox = 128 * 128;          // 128 rows x 64 columns of 16-bit (16 KB)
   static constexpr int kQBytes = 4 * kBox;        // 64 KB
   static constexpr int kSlotBytes = 2 * kBox;     // 128 rows x 128 columns (32 KB)
-  static constexpr int kSlots = 5;
+  static constexpr int kSlots = 4;  // even: a V tile's halves stay adjacent
   static constexpr int kQOff = 0;
   static constexpr int kRingOff = kQBytes;
   static constexpr int kRedOff = kRingOff + kSlots * kSlotBytes;  // [2][2][128] f32 row maxima
@@ -372,7 +377,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ tcgen05 issue
     if (lane == 0 && n_kv > 0) {
       constexpr uint32_t idesc_s = idesc_f32acc(BM, BN, false, false, E::kFmt);
-      constexpr uint32_t idesc_o = idesc_f32acc(BM, 128, false, true, E::kFmt);
+      constexpr uint32_t idesc_o = idesc_f32acc(BM, D, false, true, E::kFmt);
       bool ok = bw.wait(bar(C::kBarQ), 0, 84);
       auto slot_of = [&](int L) { return L % C::kSlots; };
       // ring positions of the K and V halves of key tile t (the loader's order)
@@ -402,19 +407,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (ok && n_kv > 1) ok = issue_s(1);
       for (int t = 0; ok && t < n_kv; ++t) {
         if (!bw.wait(bar(C::kBarP), t & 1, 86)) break;
+        // V(t)'s halves sit in adjacent slots (L even): one N = 256 product whose
+        // four 64-column boxes lie 16 KB apart
         const int L = pos_v(t);
-        if (!ready(L)) break;
+        if (!ready(L) || !ready(L + 1)) break;
         tc_fence_after();
         mma_chain_ts_mn8(tmem + C::kColO, tmem + C::col_s(t),
                          sdesc_sw128(slot_addr(slot_of(L)), C::kBox), idesc_o, t > 0 ? 1u : 0u);
         tc_commit(bar(C::kBarEmpty + slot_of(L)));
-        if (!ready(L + 1)) break;
-        tc_fence_after();
-        mma_chain_ts_mn8(tmem + C::kColO + 128, tmem + C::col_s(t),
-                         sdesc_sw128(slot_addr(slot_of(L + 1)), C::kBox), idesc_o,
-                         t > 0 ? 1u : 0u);
-        tc_commit(bar(C::kBarO));
         tc_commit(bar(C::kBarEmpty + slot_of(L + 1)));
+        tc_commit(bar(C::kBarO));
         if (t == n_kv - 1) tc_commit(bar(C::kBarOFinal));
         if (t + 2 < n_kv) ok = issue_s(t + 2);
       }

@@ -64,7 +64,7 @@ def test_fwd_validation_order_and_codes():
     assert _fwd(lib, Sq=1 << 20, H=32, D=128) == SHAPE       # 2^32 elements
     assert _fwd(lib, D=96) == HEADDIM
     assert _fwd(lib, D=512) == HEADDIM
-    assert _fwd(lib, D=256) in (ARCH, DEVICE)   # head_dim 256: forward only
+    assert _fwd(lib, D=256) in (ARCH, DEVICE)   # head_dim 256 passes validation
     assert _fwd(lib, scale=0.0) == SHAPE
     assert _fwd(lib, scale=float("nan")) == SHAPE
     assert _fwd(lib, scale=float("inf")) == SHAPE
@@ -80,6 +80,8 @@ def test_bwd_validation_and_workspace_size():
     assert lib.attn_bwd_workspace_size(1, 129, 2, 128) == 256 * 2 * (128 * 4 + 8)
     assert lib.attn_bwd_workspace_size(0, 128, 2, 64) == 0
     assert lib.attn_bwd_workspace_size(1, 128, 2, 80) == 0
+    # head_dim 256: the same layout (float32 dQ rows, then the two row values)
+    assert lib.attn_bwd_workspace_size(2, 200, 3, 256) == 2 * 3 * 256 * (256 * 4 + 8)
     p = [0x1000 * (i + 1) for i in range(9)]
     ws = lib.attn_bwd_workspace_size(1, 128, 2, 128)
 
@@ -89,7 +91,10 @@ def test_bwd_validation_and_workspace_size():
     assert bwd(ptrs=[None] + p[1:]) == NULLPTR
     assert bwd(B=0) == SHAPE
     assert bwd(D=32) == HEADDIM
-    assert bwd(D=256) == HEADDIM            # head_dim 256 has a forward only
+    assert bwd(D=256) == 10                 # head_dim 256 needs a larger workspace
+    ws256 = lib.attn_bwd_workspace_size(1, 128, 2, 256)
+    assert bwd(D=256, wsz=ws256) in (ARCH, DEVICE)  # then passes validation
+    assert bwd(D=512, wsz=ws256) == HEADDIM
     assert bwd(wl=-3) == WINDOW
     assert bwd(ptrs=p[:6] + [0x7004] + p[7:]) == ALIGN
     assert bwd(wsp=None) == 10
