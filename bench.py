@@ -43,6 +43,9 @@ GQA_WORKLOAD = dict(name="gqa_b1h32hk8s8192d128_fwdbwd", B=1, H=32, Hk=8, Sq=819
 # KV-cache decode: one new query row per sequence over a full 8192-row cache
 DECODE_WORKLOAD = dict(name="decode_b8h32hk8l8192d128", B=8, Sq=1, H=32, Hk=8, Smax=8192,
                        D=128, causal=0, input_scale=0.5, seed=1007)
+# the same step at head_dim 64, which runs the rows-on-lanes decode kernel
+DECODE64_WORKLOAD = dict(name="decode_b8h32hk8l8192d64", B=8, Sq=1, H=32, Hk=8, Smax=8192,
+                         D=64, causal=0, input_scale=0.5, seed=1010)
 # packed variable-length batch: 32768 tokens in sequences of 128..4096 tokens
 VARLEN_WORKLOAD = dict(name="varlen_t32768h32d128_fwdbwd", total=32768, len_lo=128,
                        len_hi=4096, H=32, Hk=32, D=128, causal=1, input_scale=0.5, seed=1008)
@@ -57,6 +60,7 @@ FWD_SWEEP = [
     ("c3_b1h32s8192d128", 1, 32, 8192, 0, (-1, -1), 1099.51),
     ("c4_b1h32s32768d128_causal", 1, 32, 32768, 1, (-1, -1), 8796.09),
     ("c4_b1h32s32768d128_window4096", 1, 32, 32768, 1, (4096, 0), 2062.09),
+    ("b2h32s8192d64_causal", 2, 32, 8192, 1, (-1, -1), 549.76),
 ]
 # the forward alone on the causal 7B-decoder-like layer (B1 H32 Sq=Sk=8192 D128,
 # inputs N(0,1)*0.5), timed by itself inside the default run
@@ -71,6 +75,7 @@ ORACLE_FULL = [
          win_left=-1, win_right=-1, input_scale=1.0, seed=1002),
 ]
 WORKLOADS = {"fwdbwd": WORKLOAD, "gqa": GQA_WORKLOAD, "decode": DECODE_WORKLOAD,
+             "decode64": DECODE64_WORKLOAD,
              "varlen": VARLEN_WORKLOAD, "d256": D256_WORKLOAD, "d256fwd": D256_WORKLOAD,
              "fwdsweep": None}
 D256_FWD_METRIC = "attention fwd TFLOPS, head_dim 256, bf16 vs B200 dense BF16 peak"
@@ -614,7 +619,7 @@ def run_decode_reference(args):
     rank, _, _ = dist_env()
     if rank != 0:
         return 0
-    w = DECODE_WORKLOAD
+    w = WORKLOADS[args.workload]
     inputs = decode_oracle_inputs(w)
     for _ in range(args.warmup):
         decode_oracle_step(inputs, w)
@@ -648,7 +653,7 @@ def run_decode(args):
     from exact_attention_156_b200 import (attn_decode, attn_decode_workspace_size,
                                           get_last_device_error)
     from synth import make_inputs
-    w = DECODE_WORKLOAD
+    w = WORKLOADS[args.workload]
     B, Sq, H, Hk, Smax, D = w["B"], w["Sq"], w["H"], w["Hk"], w["Smax"], w["D"]
     bits = make_inputs(B, Sq, Smax, H, D, w["seed"] + rank, w["input_scale"], Hk=Hk,
                        fmt=args.dtype)
@@ -1121,7 +1126,8 @@ def run_fwd_sweep(args):
     rows = []
     for name, B, H, S, causal, win, gflop in FWD_SWEEP:
         gen.manual_seed(1000 + len(rows))
-        q, k, v = ((torch.randn(B, S, H, 128, device="cuda", generator=gen) * 0.5).bfloat16()
+        D = 64 if name.endswith("d64_causal") else 128
+        q, k, v = ((torch.randn(B, S, H, D, device="cuda", generator=gen) * 0.5).bfloat16()
                    for _ in range(3))
         o = torch.empty_like(q)
         lse = torch.empty((B, H, S), dtype=torch.float32, device="cuda")
@@ -1189,7 +1195,7 @@ def main(argv=None):
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
-    if args.workload == "decode":
+    if args.workload in ("decode", "decode64"):
         return run_decode_reference(args) if args.impl == "reference" else run_decode(args)
     if args.workload == "varlen":
         return run_varlen_reference(args) if args.impl == "reference" else run_varlen(args)

@@ -78,6 +78,16 @@ def _load() -> ctypes.CDLL:
     lib.attn_bwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, i,
                                      i, vp]
     lib.attn_bwd_noalloc.restype = i
+    lib.attn_fwd_padded_workspace_size.argtypes = [i, i, i, i, i, i]
+    lib.attn_fwd_padded_workspace_size.restype = sz
+    lib.attn_bwd_padded_workspace_size.argtypes = [i, i, i, i, i, i]
+    lib.attn_bwd_padded_workspace_size.restype = sz
+    lib.attn_fwd_padded.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, f, i, i, i,
+                                    vp, sz, vp]
+    lib.attn_fwd_padded.restype = i
+    lib.attn_bwd_padded.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i,
+                                    i, f, i, i, i, vp, sz, vp]
+    lib.attn_bwd_padded.restype = i
     lib.attn_bwd_workspace_size.argtypes = [i, i, i, i]
     lib.attn_bwd_workspace_size.restype = sz
     lib.attn_status_string.argtypes = [i]
@@ -406,6 +416,89 @@ def attn_bwd_varlen(q, k, v, out, dout, lse, cu_seqlens_q, cu_seqlens_k, max_seq
                              _stream_handle(stream, q.device))
     if st != 0:
         raise AttnError(st, "attn_bwd_varlen")
+    return dq, dk, dv
+
+
+def attn_fwd_padded_workspace_size(B: int, Sq: int, Sk: int, H: int, Hk: int, D: int) -> int:
+    return int(lib.attn_fwd_padded_workspace_size(B, Sq, Sk, H, Hk, D))
+
+
+def attn_bwd_padded_workspace_size(B: int, Sq: int, Sk: int, H: int, Hk: int, D: int) -> int:
+    return int(lib.attn_bwd_padded_workspace_size(B, Sq, Sk, H, Hk, D))
+
+
+def _check_seqlens(t, name, B):
+    import torch
+    _check(t, name, torch.int32, 1)
+    if t.numel() != B:
+        raise ValueError(f"{name} must hold one length per sequence ({B}), got {t.numel()}")
+
+
+def attn_fwd_padded(q, k, v, seqlens_q, seqlens_k, softmax_scale: Optional[float] = None,
+                    causal: bool = False, window_size: Optional[Tuple[int, int]] = None,
+                    out=None, lse=None, workspace=None, stream=None):
+    """Exact attention of a padded batch: q (B, Sq, H, D), k, v (B, Sk, Hk, D);
+    sequence b's real rows are its first seqlens_q[b] / seqlens_k[b] rows (int32
+    CUDA tensors of B lengths).  Padding rows are never read; those of the
+    output are zero and their LSE -inf.  Returns (o (B, Sq, H, D), lse (B, H, Sq))."""
+    import torch
+    dt = _dtype_code(q)
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _check(t, n, q.dtype, 4)
+    B, Sq, H, D = q.shape
+    Sk = k.shape[1]
+    Hk = _kv_heads(q, k, v)
+    _check_seqlens(seqlens_q, "seqlens_q", B)
+    _check_seqlens(seqlens_k, "seqlens_k", B)
+    out = torch.empty_like(q) if out is None else out
+    lse = torch.empty((B, H, Sq), dtype=torch.float32, device=q.device) if lse is None else lse
+    _check(out, "out", q.dtype, 4)
+    _check(lse, "lse", torch.float32, 3)
+    if workspace is None:
+        workspace = torch.empty(max(attn_fwd_padded_workspace_size(B, Sq, Sk, H, Hk, D), 256),
+                                dtype=torch.uint8, device=q.device)
+    c, wl, wr = _window(causal, window_size)
+    st = lib.attn_fwd_padded(q.data_ptr(), k.data_ptr(), v.data_ptr(), seqlens_q.data_ptr(),
+                             seqlens_k.data_ptr(), out.data_ptr(), lse.data_ptr(), B, Sq, Sk, H,
+                             Hk, D, dt, _scale(softmax_scale, D), c, wl, wr,
+                             workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                             _stream_handle(stream, q.device))
+    if st != 0:
+        raise AttnError(st, "attn_fwd_padded")
+    return out, lse
+
+
+def attn_bwd_padded(q, k, v, out, dout, lse, seqlens_q, seqlens_k,
+                    softmax_scale: Optional[float] = None, causal: bool = False,
+                    window_size: Optional[Tuple[int, int]] = None, dq=None, dk=None, dv=None,
+                    workspace=None, stream=None):
+    """dQ, dK, dV of ``attn_fwd_padded`` (same padded layout) given its O and
+    LSE and dO; padding rows of the gradients are zero.  Returns (dq, dk, dv)."""
+    import torch
+    dt = _dtype_code(q)
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (out, "out"), (dout, "dout")):
+        _check(t, n, q.dtype, 4)
+    _check(lse, "lse", torch.float32, 3)
+    B, Sq, H, D = q.shape
+    Sk = k.shape[1]
+    Hk = _kv_heads(q, k, v)
+    _check_seqlens(seqlens_q, "seqlens_q", B)
+    _check_seqlens(seqlens_k, "seqlens_k", B)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    if workspace is None:
+        workspace = torch.empty(max(attn_bwd_padded_workspace_size(B, Sq, Sk, H, Hk, D), 256),
+                                dtype=torch.uint8, device=q.device)
+    c, wl, wr = _window(causal, window_size)
+    st = lib.attn_bwd_padded(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                             dout.data_ptr(), lse.data_ptr(), seqlens_q.data_ptr(),
+                             seqlens_k.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B,
+                             Sq, Sk, H, Hk, D, dt, _scale(softmax_scale, D), c, wl, wr,
+                             workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                             _stream_handle(stream, q.device))
+    if st != 0:
+        raise AttnError(st, "attn_bwd_padded")
     return dq, dk, dv
 
 

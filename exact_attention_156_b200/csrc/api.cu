@@ -18,6 +18,7 @@
 #include "decode_sm100.cuh"
 #include "fwd256_sm100.cuh"
 #include "fwd_sm100.cuh"
+#include "padded.cuh"
 
 using namespace attn156;
 
@@ -709,6 +710,81 @@ bool all_on_device(std::initializer_list<const void*> ptrs) {
 }
 
 // ---------------------------------------------------------------------------
+// Padded batches: the real rows gathered into packed tensors in the caller's
+// workspace, the variable-length kernels run on those, the results scattered
+// back with padding rows cleared.
+// ---------------------------------------------------------------------------
+constexpr int kPackTail = 128;  // cleared rows after the last packed row (a ragged tile's reach)
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// Workspace of a padded call: [cu_q][cu_k][packed tensors ...][varlen backward workspace].
+struct PaddedLayout {
+  size_t cu_q, cu_k, q, k, v, o, lse, dout, dq, dk, dv, bwd_ws, total;
+};
+
+PaddedLayout padded_layout(int B, int Sq, int Sk, int H, int Hk, int D, bool backward) {
+  PaddedLayout L{};
+  const size_t nq = size_t(B) * Sq * H * D * 2, nk = size_t(B) * Sk * Hk * D * 2;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = off;
+    off += align256(bytes);
+    return at;
+  };
+  L.cu_q = take(size_t(B + 2) * 4);
+  L.cu_k = take(size_t(B + 2) * 4);
+  L.q = take(nq);
+  L.k = take(nk);
+  L.v = take(nk);
+  L.o = take(nq);
+  L.lse = take(size_t(H) * B * Sq * 4);
+  if (backward) {
+    L.dout = take(nq);
+    L.dq = take(nq);
+    L.dk = take(nk);
+    L.dv = take(nk);
+    L.bwd_ws = take(varlen_workspace_bytes(B, B * Sq, H, D));
+  }
+  L.total = off;
+  return L;
+}
+
+attn_status check_padded(int B, int Sq, int Sk, int H, int Hk, int D, float scale, int win_left,
+                         int win_right) {
+  attn_status s = check_common(B, Sq, Sk, H, D, scale, win_left, win_right, Hk);
+  if (s != ATTN_OK) return s;
+  // the packed tensors and the varlen row layout must stay below 2^31 elements
+  return check_varlen(B, B * Sq, B * Sk, Sq, Sk, H, Hk, D, scale, win_left, win_right);
+}
+
+template <int D>
+attn_status launch_pack(const void* src, void* dst, const int* cu, int B, int S, int NH,
+                        cudaStream_t cs) {
+  const long long warps = (long long)B * S + kPackTail;
+  padded::pack_rows_kernel<D><<<unsigned((warps + 7) / 8), 256, 0, cs>>>(
+      static_cast<const uint16_t*>(src), static_cast<uint16_t*>(dst), cu, B, S, NH,
+      (long long)B * S, kPackTail);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_LAUNCH;
+}
+
+template <int D>
+attn_status launch_unpack(const void* src, void* dst, const int* cu, int B, int S, int NH,
+                          cudaStream_t cs) {
+  const long long warps = (long long)B * S;
+  padded::unpack_rows_kernel<D><<<unsigned((warps + 7) / 8), 256, 0, cs>>>(
+      static_cast<const uint16_t*>(src), static_cast<uint16_t*>(dst), cu, B, S, NH);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_LAUNCH;
+}
+
+attn_status launch_scans(const int* len_q, const int* len_k, int* cu_q, int* cu_k, int B, int Sq,
+                         int Sk, uint32_t* err, cudaStream_t cs) {
+  padded::seqlens_scan_kernel<<<1, 32, 0, cs>>>(len_q, B, Sq, cu_q, err);
+  padded::seqlens_scan_kernel<<<1, 32, 0, cs>>>(len_k, B, Sk, cu_k, err);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_LAUNCH;
+}
+
+// ---------------------------------------------------------------------------
 // Scratch for attn_bwd_noalloc: one statically declared device array per GPU.
 // In host code `g_noalloc_scratch` is only a host-side stand-in for the
 // symbol, never a device address; its device address is looked up once per
@@ -1077,6 +1153,119 @@ attn_status attn_decode_split_plan(int B, int Smax, int Hk, int num_sms, int* ns
   *nsplit = plan.nsplit;
   *tiles_per_split = plan.tiles_per_split;
   return ATTN_OK;
+}
+
+size_t attn_fwd_padded_workspace_size(int B, int Sq, int Sk, int H, int Hk, int D) {
+  if (check_padded(B, Sq, Sk, H, Hk, D, 1.0f, -1, -1) != ATTN_OK) return 0;
+  return padded_layout(B, Sq, Sk, H, Hk, D, false).total;
+}
+
+size_t attn_bwd_padded_workspace_size(int B, int Sq, int Sk, int H, int Hk, int D) {
+  if (check_padded(B, Sq, Sk, H, Hk, D, 1.0f, -1, -1) != ATTN_OK) return 0;
+  return padded_layout(B, Sq, Sk, H, Hk, D, true).total;
+}
+
+attn_status attn_fwd_padded(const void* q, const void* k, const void* v, const int* seqlens_q,
+                            const int* seqlens_k, void* o, float* lse, int B, int Sq, int Sk,
+                            int H, int Hk, int D, int dtype, float scale, int causal,
+                            int win_left, int win_right, void* workspace, size_t workspace_size,
+                            void* stream) {
+  if (!q || !k || !v || !seqlens_q || !seqlens_k || !o || !lse) return ATTN_ERR_NULLPTR;
+  attn_status s = check_padded(B, Sq, Sk, H, Hk, D, scale, win_left, win_right);
+  if (s != ATTN_OK) return s;
+  if ((s = check_dtype(dtype)) != ATTN_OK) return s;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned4(lse) ||
+      !aligned4(seqlens_q) || !aligned4(seqlens_k))
+    return ATTN_ERR_ALIGN;
+  const PaddedLayout L = padded_layout(B, Sq, Sk, H, Hk, D, false);
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) || workspace_size < L.total)
+    return ATTN_ERR_WORKSPACE;
+  DeviceState* st = nullptr;
+  s = device_state(&st);
+  if (s != ATTN_OK) return s;
+  if (!all_on_device({q, k, v, o, lse, seqlens_q, seqlens_k, workspace})) return ATTN_ERR_DEVICE;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  int* cu_q = reinterpret_cast<int*>(ws + L.cu_q);
+  int* cu_k = reinterpret_cast<int*>(ws + L.cu_k);
+  const Varlen vl{cu_q, cu_k, B * Sq, B * Sk, Sq, Sk};
+  if ((s = launch_scans(seqlens_q, seqlens_k, cu_q, cu_k, B, Sq, Sk, st->err, cs)) != ATTN_OK)
+    return s;
+  return dispatch(D, dtype, [&](auto d, auto e) {
+    constexpr int DD = decltype(d)::value;
+    using E = decltype(e);
+    attn_status r = launch_pack<DD>(q, ws + L.q, cu_q, B, Sq, H, cs);
+    if (r == ATTN_OK) r = launch_pack<DD>(k, ws + L.k, cu_k, B, Sk, Hk, cs);
+    if (r == ATTN_OK) r = launch_pack<DD>(v, ws + L.v, cu_k, B, Sk, Hk, cs);
+    if (r == ATTN_OK)
+      r = launch_fwd_varlen<DD, E>(*st, ws + L.q, ws + L.k, ws + L.v, ws + L.o,
+                                   reinterpret_cast<float*>(ws + L.lse), vl, B, H, Hk, scale,
+                                   causal, win_left, win_right, cs);
+    if (r == ATTN_OK) r = launch_unpack<DD>(ws + L.o, o, cu_q, B, Sq, H, cs);
+    if (r == ATTN_OK) {
+      const long long n = (long long)B * H * Sq;
+      padded::unpack_lse_kernel<<<unsigned((n + 255) / 256), 256, 0, cs>>>(
+          reinterpret_cast<const float*>(ws + L.lse), lse, cu_q, B, Sq, H, (long long)B * Sq);
+      if (cudaGetLastError() != cudaSuccess) r = ATTN_ERR_LAUNCH;
+    }
+    return r;
+  });
+}
+
+attn_status attn_bwd_padded(const void* q, const void* k, const void* v, const void* o,
+                            const void* dout, const float* lse, const int* seqlens_q,
+                            const int* seqlens_k, void* dq, void* dk, void* dv, int B, int Sq,
+                            int Sk, int H, int Hk, int D, int dtype, float scale, int causal,
+                            int win_left, int win_right, void* workspace, size_t workspace_size,
+                            void* stream) {
+  if (!q || !k || !v || !o || !dout || !lse || !seqlens_q || !seqlens_k || !dq || !dk || !dv)
+    return ATTN_ERR_NULLPTR;
+  attn_status s = check_padded(B, Sq, Sk, H, Hk, D, scale, win_left, win_right);
+  if (s != ATTN_OK) return s;
+  if ((s = check_dtype(dtype)) != ATTN_OK) return s;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) ||
+      !aligned16(dq) || !aligned16(dk) || !aligned16(dv) || !aligned4(lse) ||
+      !aligned4(seqlens_q) || !aligned4(seqlens_k))
+    return ATTN_ERR_ALIGN;
+  const PaddedLayout L = padded_layout(B, Sq, Sk, H, Hk, D, true);
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) || workspace_size < L.total)
+    return ATTN_ERR_WORKSPACE;
+  DeviceState* st = nullptr;
+  s = device_state(&st);
+  if (s != ATTN_OK) return s;
+  if (!all_on_device({q, k, v, o, dout, lse, seqlens_q, seqlens_k, dq, dk, dv, workspace}))
+    return ATTN_ERR_DEVICE;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  int* cu_q = reinterpret_cast<int*>(ws + L.cu_q);
+  int* cu_k = reinterpret_cast<int*>(ws + L.cu_k);
+  const Varlen vl{cu_q, cu_k, B * Sq, B * Sk, Sq, Sk};
+  if ((s = launch_scans(seqlens_q, seqlens_k, cu_q, cu_k, B, Sq, Sk, st->err, cs)) != ATTN_OK)
+    return s;
+  float* lse_p = reinterpret_cast<float*>(ws + L.lse);
+  return dispatch(D, dtype, [&](auto d, auto e) {
+    constexpr int DD = decltype(d)::value;
+    using E = decltype(e);
+    attn_status r = launch_pack<DD>(q, ws + L.q, cu_q, B, Sq, H, cs);
+    if (r == ATTN_OK) r = launch_pack<DD>(k, ws + L.k, cu_k, B, Sk, Hk, cs);
+    if (r == ATTN_OK) r = launch_pack<DD>(v, ws + L.v, cu_k, B, Sk, Hk, cs);
+    if (r == ATTN_OK) r = launch_pack<DD>(o, ws + L.o, cu_q, B, Sq, H, cs);
+    if (r == ATTN_OK) r = launch_pack<DD>(dout, ws + L.dout, cu_q, B, Sq, H, cs);
+    if (r == ATTN_OK) {
+      const long long n = (long long)B * H * Sq;
+      padded::pack_lse_kernel<<<unsigned((n + 255) / 256), 256, 0, cs>>>(
+          lse, lse_p, cu_q, B, Sq, H, (long long)B * Sq);
+      if (cudaGetLastError() != cudaSuccess) r = ATTN_ERR_LAUNCH;
+    }
+    if (r == ATTN_OK)
+      r = run_backward_varlen<DD, E>(*st, ws + L.q, ws + L.k, ws + L.v, ws + L.o, ws + L.dout,
+                                     lse_p, ws + L.dq, ws + L.dk, ws + L.dv, vl, B, H, Hk, scale,
+                                     causal, win_left, win_right, ws + L.bwd_ws, cs);
+    if (r == ATTN_OK) r = launch_unpack<DD>(ws + L.dq, dq, cu_q, B, Sq, H, cs);
+    if (r == ATTN_OK) r = launch_unpack<DD>(ws + L.dk, dk, cu_k, B, Sk, Hk, cs);
+    if (r == ATTN_OK) r = launch_unpack<DD>(ws + L.dv, dv, cu_k, B, Sk, Hk, cs);
+    return r;
+  });
 }
 
 attn_status attn_get_last_device_error(void) {

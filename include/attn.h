@@ -37,8 +37,9 @@
  *     bottom-right corner when Sq != Sk.
  *   - scale must be finite and > 0 (callers wanting the default pass
  *     1/sqrt(head_dim)).
- *   - head_dim D must be 64 or 128; the forward entry points attn_fwd and
- *     attn_fwd_ex also take 256 (the backward, the varlen and the decode entry
+ *   - head_dim D must be 64 or 128; the dense forward and backward entry points
+ *     (attn_fwd, attn_bwd, their _ex forms, the three backward stages and
+ *     attn_bwd_noalloc) also take 256 (the varlen, padded and decode entry
  *     points do not).  B, H, Sq, Sk must be >= 1 and every
  *     tensor must hold fewer than 2^31 elements.
  *   - The device must be compute capability 10.0 (B200, sm_100a).
@@ -66,7 +67,7 @@ typedef enum {
     ATTN_OK = 0,
     ATTN_ERR_NULLPTR = 1,   /* a required pointer is NULL                         */
     ATTN_ERR_SHAPE = 2,     /* B, H, Sq or Sk < 1, a size overflows, or bad scale */
-    ATTN_ERR_HEADDIM = 3,   /* head_dim not in {64, 128} (forward: {64, 128, 256}) */
+    ATTN_ERR_HEADDIM = 3,   /* head_dim not in {64, 128} (dense: {64, 128, 256})  */
     ATTN_ERR_ALIGN = 4,     /* a tensor pointer is not 16-byte aligned            */
     ATTN_ERR_WINDOW = 5,    /* win_left or win_right < -1                         */
     ATTN_ERR_ARCH = 6,      /* current device is not compute capability 10.0      */
@@ -141,7 +142,9 @@ ATTN_API attn_status attn_bwd(const void* q, const void* k, const void* v, const
  * attn_bwd_main - for every 128-key tile: recomputes P from Q, K and the
  *   workspace LSE, accumulates dV = P^T dO and dK = scale dS^T Q in tensor
  *   memory and writes them (bf16), and adds dS K into the workspace dQ
- *   accumulator with float32 bulk reduce-adds.
+ *   accumulator with float32 bulk reduce-adds.  At head_dim 256 dK, dV and dQ
+ *   are accumulated by separate tiles of one launch, and dS K is written into
+ *   the accumulator whole, row by row (the preprocess then does not clear it).
  * attn_bwd_dq_finalize - dq = bf16(scale * accumulator).
  */
 ATTN_API attn_status attn_bwd_preprocess(const void* o, const void* dout, const float* lse,
@@ -259,6 +262,49 @@ ATTN_API attn_status attn_decode(const void* q, const void* k_cache, const void*
                                  int Smax, int H, int Hk, int D, int dtype, float scale,
                                  int causal, void* workspace, size_t workspace_bytes,
                                  void* stream);
+
+/*
+ * attn_fwd_padded / attn_bwd_padded - a padded batch: B sequences stored in
+ * (B, S, H, D) tensors of one padded length, sequence b's real rows being
+ * rows 0 .. seqlens[b] - 1 (the pages name the upstream padded-batch test,
+ * FlashAttention-2 overview, lshu.cn, section 3.2, and say nothing more).
+ * The result is that of the packed batch of the real rows (attn_fwd_varlen /
+ * attn_bwd_varlen); padding rows of the inputs are never read and may hold
+ * anything, non-finite values included; padding rows of the outputs are
+ * written as zeros (o, dq for rows >= seqlens_q[b]; dk, dv for rows >=
+ * seqlens_k[b]) and their LSE as -inf.  The real rows are gathered into
+ * packed copies in the workspace, the variable-length kernels run on those,
+ * and the results are scattered back.
+ *
+ *   q, o, dout, dq  [B, Sq, H, D]        k, v, dk, dv [B, Sk, Hk, D]
+ *   lse             [B, H, Sq] float32 (out of attn_fwd_padded, in of bwd)
+ *   seqlens_q / _k  [B] int32, device: 0 <= seqlens_q[b] <= Sq, 0 <= seqlens_k[b] <= Sk.
+ *                   They live on the device, so they are checked there: a
+ *                   length outside its range is taken as 0 (the sequence's
+ *                   output rows are zeros) and the next
+ *                   attn_get_last_device_error returns ATTN_ERR_SEQLENS.
+ *   workspace       at least attn_fwd_padded_workspace_size / 
+ *                   attn_bwd_padded_workspace_size(B, Sq, Sk, H, Hk, D) bytes,
+ *                   256-byte aligned, contents ignored (0 from the size
+ *                   functions means the arguments are invalid).
+ * head_dim 64 or 128; grouped K/V heads and dtype as in the _ex entry points.
+ * Errors: as attn_fwd_ex / attn_bwd_ex; ATTN_ERR_ALIGN if lse or a seqlens
+ * pointer is not 4-byte aligned.
+ */
+ATTN_API size_t attn_fwd_padded_workspace_size(int B, int Sq, int Sk, int H, int Hk, int D);
+ATTN_API attn_status attn_fwd_padded(const void* q, const void* k, const void* v,
+                                     const int* seqlens_q, const int* seqlens_k, void* o,
+                                     float* lse, int B, int Sq, int Sk, int H, int Hk, int D,
+                                     int dtype, float scale, int causal, int win_left,
+                                     int win_right, void* workspace, size_t workspace_bytes,
+                                     void* stream);
+ATTN_API size_t attn_bwd_padded_workspace_size(int B, int Sq, int Sk, int H, int Hk, int D);
+ATTN_API attn_status attn_bwd_padded(const void* q, const void* k, const void* v, const void* o,
+                                     const void* dout, const float* lse, const int* seqlens_q,
+                                     const int* seqlens_k, void* dq, void* dk, void* dv, int B,
+                                     int Sq, int Sk, int H, int Hk, int D, int dtype, float scale,
+                                     int causal, int win_left, int win_right, void* workspace,
+                                     size_t workspace_bytes, void* stream);
 
 /*
  * attn_fwd_varlen / attn_bwd_varlen - a batch of B sequences of different

@@ -294,3 +294,37 @@ def test_decode_split_plan():
                     cost = lambda t: math.ceil(B * Hk * math.ceil(tiles / t) / sms) * (t + 3)
                     best = min(cost(t) for t in range(2 if tiles > 1 else 1, tiles + 1))
                     assert cost(tps) == best, (B, Smax, Hk, sms, ns, tps)
+
+
+def test_padded_validation_and_workspace_size():
+    from exact_attention_156_b200 import lib
+    wsf = lib.attn_fwd_padded_workspace_size(2, 300, 400, 4, 2, 128)
+    wsb = lib.attn_bwd_padded_workspace_size(2, 300, 400, 4, 2, 128)
+    # the backward also holds dO, dQ, dK, dV and the packed backward's own workspace
+    assert 0 < wsf < wsb
+    assert wsb - wsf >= lib.attn_bwd_varlen_workspace_size(2, 600, 4, 128)
+    assert lib.attn_fwd_padded_workspace_size(2, 300, 400, 4, 2, 256) == 0   # head_dim 256
+    assert lib.attn_fwd_padded_workspace_size(2, 300, 400, 4, 3, 128) == 0   # Hk must divide H
+    assert lib.attn_bwd_padded_workspace_size(0, 300, 400, 4, 2, 128) == 0
+    p = [0x1000 * (i + 1) for i in range(11)]
+    f = ctypes.c_float
+
+    def fwd(ptrs=p[:7], D=128, Hk=2, ws=0x200000, wsz=wsf, dtype=0):
+        return lib.attn_fwd_padded(*ptrs, 2, 300, 400, 4, Hk, D, dtype, f(0.1), 1, -1, -1, ws,
+                                   wsz, None)
+
+    def bwd(ptrs=p, D=128, ws=0x200000, wsz=wsb):
+        return lib.attn_bwd_padded(*ptrs, 2, 300, 400, 4, 2, D, 0, f(0.1), 1, -1, -1, ws, wsz,
+                                   None)
+
+    assert fwd(ptrs=p[:3] + [None] + p[4:7]) == NULLPTR
+    assert fwd(D=256) == HEADDIM
+    assert fwd(Hk=3) == SHAPE
+    assert fwd(dtype=7) == 12
+    assert fwd(ptrs=p[:3] + [0x3002] + p[4:7]) == ALIGN     # seqlens not 4-byte aligned
+    assert fwd(ws=0x200010) == 10
+    assert fwd(wsz=wsf - 1) == 10
+    assert fwd() in (ARCH, DEVICE)
+    assert bwd(ptrs=p[:10] + [None]) == NULLPTR
+    assert bwd(wsz=wsb - 256) == 10
+    assert bwd() in (ARCH, DEVICE)
