@@ -49,7 +49,10 @@ DECODE64_WORKLOAD = dict(name="decode_b8h32hk8l8192d64", B=8, Sq=1, H=32, Hk=8, 
 # packed variable-length batch: 32768 tokens in sequences of 128..4096 tokens
 VARLEN_WORKLOAD = dict(name="varlen_t32768h32d128_fwdbwd", total=32768, len_lo=128,
                        len_hi=4096, H=32, Hk=32, D=128, causal=1, input_scale=0.5, seed=1008)
-# head_dim 256 (forward only): B1 H16 S8192 causal
+# head_dim 64 forward alone: B2 H32 S8192 causal (inputs 192 MiB, larger than L2)
+FWD64_WORKLOAD = dict(name="fwd_b2h32s8192d64_causal", B=2, H=32, Hk=32, Sq=8192, Sk=8192,
+                      D=64, causal=1, win_left=-1, win_right=-1, input_scale=0.5, seed=1011)
+# head_dim 256: B1 H16 S8192 causal
 D256_WORKLOAD = dict(name="fwd_b1h16s8192d256_causal", B=1, H=16, Hk=16, Sq=8192, Sk=8192,
                      D=256, causal=1, win_left=-1, win_right=-1, input_scale=0.5, seed=1009)
 # forward alone on the attention configurations (name, B, H, S, causal, window, counted
@@ -77,8 +80,10 @@ ORACLE_FULL = [
 WORKLOADS = {"fwdbwd": WORKLOAD, "gqa": GQA_WORKLOAD, "decode": DECODE_WORKLOAD,
              "decode64": DECODE64_WORKLOAD,
              "varlen": VARLEN_WORKLOAD, "d256": D256_WORKLOAD, "d256fwd": D256_WORKLOAD,
+             "fwd64": FWD64_WORKLOAD,
              "fwdsweep": None}
 D256_FWD_METRIC = "attention fwd TFLOPS, head_dim 256, bf16 vs B200 dense BF16 peak"
+FWD64_METRIC = "attention fwd TFLOPS, head_dim 64, bf16 vs B200 dense BF16 peak"
 D256_METRIC = "attention fwd+bwd TFLOPS, head_dim 256, bf16 vs B200 dense BF16 peak"
 DECODE_METRIC = "KV-cache decode: cached K/V bytes read per second"
 FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "hbm_gbs": 6650.0, "source": "fallback"}
@@ -955,7 +960,7 @@ def run_varlen(args):
 
 
 def run_fwd_only(args):
-    """Forward-only workload (head_dim 256, which has no backward here)."""
+    """Forward-only workloads (head_dim 256 or 64, the forward alone)."""
     import torch
     rank, world, local = dist_env()
     if world > 1:
@@ -967,7 +972,8 @@ def run_fwd_only(args):
     torch.cuda.set_device(device)
     from exact_attention_156_b200 import attn_fwd, get_last_device_error
     from synth import make_inputs
-    w = D256_WORKLOAD
+    w = WORKLOADS[args.workload]
+    fwd_metric = D256_FWD_METRIC if w["D"] == 256 else FWD64_METRIC
     B, H, Sq, Sk, D = w["B"], w["H"], w["Sq"], w["Sk"], w["D"]
     bits = make_inputs(B, Sq, Sk, H, D, w["seed"] + rank, w["input_scale"], Hk=w["Hk"],
                        fmt=args.dtype)
@@ -1026,14 +1032,17 @@ def run_fwd_only(args):
     peaks = load_peaks()
     peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
     line = {
-        "metric": D256_FWD_METRIC, "value": world * tf, "unit": UNIT, "n_gpus": world,
+        "metric": fwd_metric, "value": world * tf, "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": args.dtype, "data": "synthetic",
         "config": {"workload": f"{w['name']}: forward, B={B} H={H} Sq=Sk={Sq} D={D} causal, "
                                f"inputs N(0,1)*{w['input_scale']}", "B": B, "H": H, "Sq": Sq,
                    "Sk": Sk, "D": D, "causal": causal,
-                   "l2": "no flush: inputs (Q,K,V 384 MiB) exceed the 126 MB L2"},
-        "roofline": {"bound": "tensor", "kernel": "attn_fwd_d256_kernel", "achieved": tf,
+                   "l2": f"no flush: inputs (Q,K,V {3 * B * Sq * H * D * 2 / 2**20:.0f} MiB) "
+                         "exceed the 126 MB L2"},
+        "roofline": {"bound": "tensor",
+                     "kernel": "attn_fwd_d256_kernel" if D == 256 else f"attn_fwd_kernel<{D}>",
+                     "achieved": tf,
                      "peak": peak, "unit": "TFLOP/s", "frac": tf / peak,
                      "peak_source": f"{peaks.get('source')} bf16_tflops (burst)",
                      "traffic": None},
@@ -1086,7 +1095,7 @@ def run_fwd_only_reference(args):
     rank, _, _ = dist_env()
     if rank != 0:
         return 0
-    w = D256_WORKLOAD
+    w = WORKLOADS[args.workload]
     inputs = oracle_sample_inputs(w)
     for i in range(args.warmup):
         fwd_oracle_sample(inputs, w, 1000 + i)
@@ -1097,7 +1106,8 @@ def run_fwd_only_reference(args):
         tot_f += fl
     value = tot_f / tot_s / 1e12
     print(json.dumps({
-        "impl": "reference", "metric": D256_FWD_METRIC, "value": value, "unit": UNIT,
+        "impl": "reference",
+        "metric": D256_FWD_METRIC if w["D"] == 256 else FWD64_METRIC, "value": value, "unit": UNIT,
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": tot_s / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
@@ -1184,8 +1194,9 @@ def main(argv=None):
                          "with 8 K/V heads for 32 query heads; decode: KV-cache decode "
                          "(B8 H32 Hk8, 8192 cached rows, one new row); varlen: a packed batch "
                          "of 32768 tokens in sequences of 128..4096; d256: head_dim 256 forward + "
-                         "backward, B1 H16 S8192 causal; d256fwd: its forward alone; fwdsweep: "
-                         "the forward alone on C2-C4")
+                         "backward, B1 H16 S8192 causal; d256fwd: its forward alone; fwd64: the "
+                         "head_dim 64 forward alone, B2 H32 S8192 causal; decode64: the decode "
+                         "step at head_dim 64; fwdsweep: the forward alone on C2-C4")
     ap.add_argument("--no-cpu-baseline", action="store_true",
                     help="skip the timed oracle sample (it adds ~15 s of CPU time)")
     ap.add_argument("--no-c3", action="store_true",
@@ -1199,7 +1210,7 @@ def main(argv=None):
         return run_decode_reference(args) if args.impl == "reference" else run_decode(args)
     if args.workload == "varlen":
         return run_varlen_reference(args) if args.impl == "reference" else run_varlen(args)
-    if args.workload == "d256fwd":
+    if args.workload in ("d256fwd", "fwd64"):
         return run_fwd_only_reference(args) if args.impl == "reference" else run_fwd_only(args)
     if args.workload == "fwdsweep":
         if args.impl == "reference":

@@ -162,6 +162,71 @@ constexpr CUtensorMapDataType tmap_type() {
                                           : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
 }
 
+// Encoded tensor maps, cached per (device, base address, element type, rank,
+// extents, strides, box): a map is a pure function of these, so a cached one
+// stays valid for as long as the same arguments come back (a buffer freed and
+// reallocated at the same address with the same shape gets the same map).
+// Small and round-robin: one call needs at most eight maps.  Every map in this
+// library uses 128-byte swizzle, no interleave, 256-byte L2 promotion, zero
+// fill out of bounds and unit element strides.
+struct MapKey {
+  int dev, rank;
+  CUtensorMapDataType dtype;
+  const void* base;
+  cuuint64_t dims[4], strides[3];
+  cuuint32_t box[4];
+  bool operator==(const MapKey& o) const {
+    if (dev != o.dev || rank != o.rank || dtype != o.dtype || base != o.base) return false;
+    for (int i = 0; i < rank; ++i)
+      if (dims[i] != o.dims[i] || box[i] != o.box[i]) return false;
+    for (int i = 0; i + 1 < rank; ++i)
+      if (strides[i] != o.strides[i]) return false;
+    return true;
+  }
+};
+constexpr int kMapCacheSize = 64;
+struct MapCache {
+  MapKey key[kMapCacheSize];
+  alignas(64) CUtensorMap map[kMapCacheSize];
+  bool used[kMapCacheSize] = {};
+  int next = 0;
+};
+MapCache g_maps;
+std::mutex g_maps_mu;
+
+attn_status encode_cached(CUtensorMap* out, CUtensorMapDataType dtype, int rank, const void* base,
+                          const cuuint64_t* dims, const cuuint64_t* strides,
+                          const cuuint32_t* box) {
+  MapKey k{};
+  if (cudaGetDevice(&k.dev) != cudaSuccess) return ATTN_ERR_DEVICE;
+  k.rank = rank;
+  k.dtype = dtype;
+  k.base = base;
+  for (int i = 0; i < rank; ++i) {
+    k.dims[i] = dims[i];
+    k.box[i] = box[i];
+  }
+  for (int i = 0; i + 1 < rank; ++i) k.strides[i] = strides[i];
+  std::lock_guard<std::mutex> lock(g_maps_mu);
+  for (int i = 0; i < kMapCacheSize; ++i)
+    if (g_maps.used[i] && g_maps.key[i] == k) {
+      *out = g_maps.map[i];
+      return ATTN_OK;
+    }
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  const CUresult r =
+      g_encode(out, dtype, cuuint32_t(rank), const_cast<void*>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return ATTN_ERR_LAUNCH;
+  const int slot = g_maps.next;
+  g_maps.next = (slot + 1) % kMapCacheSize;
+  g_maps.key[slot] = k;
+  g_maps.map[slot] = *out;
+  g_maps.used[slot] = true;
+  return ATTN_OK;
+}
+
 // 4-D map over a (B, S, H, D) tensor of 16-bit elements, box = 64 x 1 x rows x 1
 // (rows = 128 unless given), 128-byte swizzle.
 attn_status make_map(CUtensorMap* map, const void* base, int B, int S, int H, int D,
@@ -170,12 +235,7 @@ attn_status make_map(CUtensorMap* map, const void* base, int B, int S, int H, in
   const cuuint64_t strides[3] = {cuuint64_t(D) * 2, cuuint64_t(H) * D * 2,
                                  cuuint64_t(S) * H * D * 2};
   const cuuint32_t box[4] = {64, 1, cuuint32_t(box_rows), 1};
-  const cuuint32_t estr[4] = {1, 1, 1, 1};
-  const CUresult r =
-      g_encode(map, dtype, 4, const_cast<void*>(base), dims, strides,
-               box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS ? ATTN_OK : ATTN_ERR_LAUNCH;
+  return encode_cached(map, dtype, 4, base, dims, strides, box);
 }
 
 // 2-D fp32 map over the dQ accumulator [rows][D], box = 32 x 128, 128-byte swizzle
@@ -184,12 +244,7 @@ attn_status make_dq_map(CUtensorMap* map, const float* base, long long rows, int
   const cuuint64_t dims[2] = {cuuint64_t(D), cuuint64_t(rows)};
   const cuuint64_t strides[1] = {cuuint64_t(D) * 4};
   const cuuint32_t box[2] = {32, 128};
-  const cuuint32_t estr[2] = {1, 1};
-  const CUresult r =
-      g_encode(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(base), dims, strides,
-               box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS ? ATTN_OK : ATTN_ERR_LAUNCH;
+  return encode_cached(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, base, dims, strides, box);
 }
 
 int sq_pad(int Sq) { return ((Sq + 127) / 128) * 128; }
@@ -634,12 +689,7 @@ attn_status launch_decode(const DeviceState& st, const void* q, const void* kc, 
     const cuuint64_t strides[3] = {cuuint64_t(D) * 2, cuuint64_t(H) * D * 2,
                                    cuuint64_t(Sq) * H * D * 2};
     const cuuint32_t box[4] = {64, cuuint32_t(group), cuuint32_t(Sq), 1};
-    const cuuint32_t estr[4] = {1, 1, 1, 1};
-    if (g_encode(&mq, dt, 4, const_cast<void*>(q), dims, strides, box, estr,
-                 CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                 CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-      return ATTN_ERR_LAUNCH;
+    if (encode_cached(&mq, dt, 4, q, dims, strides, box) != ATTN_OK) return ATTN_ERR_LAUNCH;
   }
   if (make_map(&mk, kc, B, Smax, Hk, D, dt) != ATTN_OK ||
       make_map(&mv, vc, B, Smax, Hk, D, dt) != ATTN_OK)
