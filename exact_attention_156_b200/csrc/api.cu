@@ -280,6 +280,7 @@ attn_status launch_fwd(const DeviceState& st, const void* q, const void* k, cons
   p.total_q = 0;
   p.total_k = 0;
   p.num_mblocks = (Sq + fwd::NQ * fwd::BM - 1) / (fwd::NQ * fwd::BM);
+  p.compact = 0;
   p.err = st.err;
   p.timeout_ns = kTimeoutNs;
   dim3 grid(p.num_mblocks, H, B);
@@ -376,6 +377,7 @@ attn_status launch_bwd_main(const DeviceState& st, const void* q, const void* k,
   p.total_q = 0;
   p.total_k = 0;
   p.R = 0;
+  p.compact = 0;
   p.Hk = Hk;
   p.scale = scale;
   p.scale_log2 = scale * 1.4426950408889634f;
@@ -572,7 +574,13 @@ attn_status launch_fwd_varlen(const DeviceState& st, const void* q, const void* 
   p.num_mblocks = (vl.max_q + fwd::NQ * fwd::BM - 1) / (fwd::NQ * fwd::BM);
   p.err = st.err;
   p.timeout_ns = kTimeoutNs;
-  dim3 grid(p.num_mblocks, H, B);
+  // Up to kCompactMaxB sequences: one CTA per query-tile pair that has work
+  // (at most ceil(total_q / 256) + B of them); otherwise the longest sequence's
+  // pair count for every sequence.
+  p.compact = B <= kCompactMaxB ? 1 : 0;
+  const int rows = fwd::NQ * fwd::BM;
+  dim3 grid = p.compact ? dim3((vl.total_q + rows - 1) / rows + B, H, 1)
+                        : dim3(p.num_mblocks, H, B);
   fwd::attn_fwd_kernel<D, E, true><<<grid, fwd::kThreads, fwd::Cfg<D>::kSmemBytes, stream>>>(mq, mk, mv,
                                                                                        p);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_LAUNCH;
@@ -629,7 +637,12 @@ attn_status run_backward_varlen(const DeviceState& st, const void* q, const void
   p.win_right = win_right;
   p.err = st.err;
   p.timeout_ns = kTimeoutNs;
-  dim3 grid((vl.max_k + bwd::BN - 1) / bwd::BN, Hk, B);
+  // Up to kCompactMaxB sequences: one CTA per key tile that has work (at most
+  // ceil(total_k / 128) + B of them); otherwise the longest sequence's tile
+  // count for every sequence.
+  p.compact = B <= kCompactMaxB ? 1 : 0;
+  dim3 grid = p.compact ? dim3((vl.total_k + bwd::BN - 1) / bwd::BN + B, Hk, 1)
+                        : dim3((vl.max_k + bwd::BN - 1) / bwd::BN, Hk, B);
   bwd::attn_bwd_main_kernel<D, E, true>
       <<<grid, bwd::kThreads, bwd::Cfg<D>::kSmemBytes, stream>>>(mq, mk, mv, mdo, mdq, p);
   if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_LAUNCH;

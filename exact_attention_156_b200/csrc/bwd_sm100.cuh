@@ -118,6 +118,7 @@ struct Params {
   const int* cu_q;
   const int* cu_k;
   int total_q, total_k, R;
+  int compact;  // packed batches: blockIdx.x numbers the key tiles that have work (compact_tile)
   int Hk;  // key/value heads: the CTA's K/V head is shared by H / Hk query heads
   float scale;
   float scale_log2;
@@ -373,9 +374,21 @@ __global__ void __launch_bounds__(kThreads, 1)
   // Grid: (key tile, K/V head, batch).  The key tiles of one head run side by
   // side, so they share that head's Q and dO tiles in L2; low key tiles (the
   // most query tiles when causal) start first.
-  const int kt = blockIdx.x;
+  int kt = blockIdx.x;
   const int hk = blockIdx.y;  // key/value head
-  const int b = blockIdx.z;
+  int b = blockIdx.z;
+  if constexpr (kVarlen) {
+    if (p.compact) {
+      // one CTA per key tile that has work, low key tiles (the heaviest when
+      // causal) first
+      b = compact_tile(p.cu_q, p.cu_k, p.B, p.total_q, p.total_k, p.Sq, p.Sk, true, BN,
+                       int(blockIdx.x), kt);
+      if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x < 32)
+        compact_check(p.cu_q, p.cu_k, p.B, p.total_q, p.total_k, p.Sq, p.Sk, true, BN,
+                      (long long)gridDim.x, p.err);
+      if (b < 0) return;
+    }
+  }
   const int group = p.H / p.Hk;  // query heads sharing this K/V head
   // This sequence's lengths, first rows, TMA batch coordinate and row-value base.
   int Lq = p.Sq, Lk = p.Sk, q_row0 = 0, k_row0 = 0, bc = b;

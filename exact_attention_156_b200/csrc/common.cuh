@@ -73,4 +73,79 @@ __device__ __forceinline__ SeqSpan seq_span(const int* cu_q, const int* cu_k, in
   return s;
 }
 
+// Packed batches of at most kCompactMaxB sequences run on a compact grid: one
+// CTA per (tile, sequence) that has work, instead of the longest sequence's tile
+// count for every sequence (CTAs that only find their sequence too short to
+// reach them still cost a launch and a shared-memory allocation each).
+// Tiles are numbered level by level: level l holds tile l of every sequence
+// that has more than l tiles, in sequence order, so the first level (each
+// sequence's heaviest tile) starts first and the light tiles form the tail.
+// A malformed sequence has no tiles.
+constexpr int kCompactMaxB = 256;
+
+// Tile `idx` of that numbering: returns the sequence (and its tile, 0 = the
+// first level) or -1 past the last tile.  Every thread of a warp calls it
+// (warp shuffles); lane i holds the tile counts of sequences i, i + 32, ....
+// `rows`: rows per tile of the query axis (by_keys = 0) or the key axis.
+__device__ __forceinline__ int compact_tile(const int* cu_q, const int* cu_k, int B, int total_q,
+                                           int total_k, int max_q, int max_k, bool by_keys,
+                                           int rows, int idx, int& tile) {
+  const int lane = threadIdx.x & 31;
+  constexpr int kPer = kCompactMaxB / 32;
+  int cnt[kPer];
+  int tmax = 0;
+#pragma unroll
+  for (int r = 0; r < kPer; ++r) {
+    const int b = r * 32 + lane;
+    cnt[r] = 0;
+    if (b < B) {
+      const SeqSpan sp = seq_span(cu_q, cu_k, b, total_q, total_k, max_q, max_k);
+      cnt[r] = ((by_keys ? sp.Lk : sp.Lq) + rows - 1) / rows;
+    }
+    tmax = max(tmax, cnt[r]);
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) tmax = max(tmax, __shfl_xor_sync(0xffffffffu, tmax, off));
+  for (int l = 0; l < tmax; ++l) {
+#pragma unroll
+    for (int r = 0; r < kPer; ++r) {
+      if (r * 32 >= B) break;
+      const unsigned has = __ballot_sync(0xffffffffu, cnt[r] > l);
+      const int n = __popc(has);
+      if (idx < n) {
+        // the idx-th set bit of `has`
+        unsigned m = has;
+        for (int j = 0; j < idx; ++j) m &= m - 1;
+        tile = l;
+        return r * 32 + __ffs(m) - 1;
+      }
+      idx -= n;
+    }
+  }
+  tile = 0;
+  return -1;
+}
+
+// Run by one full warp of one CTA of a compact grid: a malformed sequence has
+// no tiles, so no CTA of its own reports it; and with malformed (overlapping)
+// boundaries the valid sequences' tiles could outnumber the grid.  Either sets
+// the device error word.
+__device__ __forceinline__ void compact_check(const int* cu_q, const int* cu_k, int B,
+                                              int total_q, int total_k, int max_q, int max_k,
+                                              bool by_keys, int rows, long long grid,
+                                              uint32_t* err) {
+  const int lane = threadIdx.x & 31;
+  long long tiles = 0;
+  bool bad = false;
+  for (int b = lane; b < B; b += 32) {
+    const SeqSpan sp = seq_span(cu_q, cu_k, b, total_q, total_k, max_q, max_k);
+    bad = bad || !sp.ok;
+    tiles += ((by_keys ? sp.Lk : sp.Lq) + rows - 1) / rows;
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) tiles += __shfl_xor_sync(0xffffffffu, tiles, off);
+  bad = __any_sync(0xffffffffu, bad) != 0;
+  if (lane == 0 && (bad || tiles > grid)) atomicCAS(err, 0u, kErrSeqlens);
+}
+
 }  // namespace attn156

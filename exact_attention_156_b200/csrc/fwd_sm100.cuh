@@ -92,6 +92,7 @@ struct Params {
   float scale_log2;  // scale * log2(e)
   int causal, win_left, win_right;
   int num_mblocks;   // ceil(Sq / (NQ * BM))
+  int compact;       // packed batches: blockIdx.x numbers the tiles that have work (compact_tile)
   uint32_t* err;
   uint64_t timeout_ns;
 };
@@ -134,10 +135,26 @@ __global__ void __launch_bounds__(kThreads, 1)
   // Grid: (query-tile pair, head, batch).  The pairs of one head run side by
   // side, so they share that head's K/V tiles in L2; causal launches each
   // head's pairs with the most keys first.
-  const int mb = p.causal ? (p.num_mblocks - 1 - int(blockIdx.x)) : int(blockIdx.x);
+  int mb = p.causal ? (p.num_mblocks - 1 - int(blockIdx.x)) : int(blockIdx.x);
   const int h = blockIdx.y;
   const int hk = h / (p.H / p.Hk);  // the key/value head this query head reads
-  const int b = blockIdx.z;
+  int b = blockIdx.z;
+  if constexpr (kVarlen) {
+    if (p.compact) {
+      // one CTA per query-tile pair that has work, the heaviest pairs first
+      int tile = 0;
+      b = compact_tile(p.cu_q, p.cu_k, p.B, p.total_q, p.total_k, p.Sq, p.Sk, false, NQ * BM,
+                       int(blockIdx.x), tile);
+      if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x < 32)
+        compact_check(p.cu_q, p.cu_k, p.B, p.total_q, p.total_k, p.Sq, p.Sk, false, NQ * BM,
+                      (long long)gridDim.x, p.err);
+      if (b < 0) return;
+      const int pairs =
+          (seq_span(p.cu_q, p.cu_k, b, p.total_q, p.total_k, p.Sq, p.Sk).Lq + NQ * BM - 1) /
+          (NQ * BM);
+      mb = p.causal ? pairs - 1 - tile : tile;
+    }
+  }
   // This sequence's lengths, first rows and TMA batch coordinate.
   int Lq = p.Sq, Lk = p.Sk, q_row0 = 0, k_row0 = 0, bc = b;
   if constexpr (kVarlen) {

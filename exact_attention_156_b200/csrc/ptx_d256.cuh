@@ -92,4 +92,30 @@ __device__ __forceinline__ void mma_chain_ts_mn4(uint32_t d_tmem, uint32_t a_tme
       : "memory");
 }
 
+// 4 chained K-steps (K = 64), A from tensor memory in two 16-column pieces 32
+// columns apart (steps at +0, +8, +32, +40), B MN-major (TS form).
+__device__ __forceinline__ void mma_chain_ts_mn4_split32(uint32_t d_tmem, uint32_t a_tmem,
+                                                        uint64_t b_desc, uint32_t idesc,
+                                                        uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .b32 blo, bhi, bl, at;\n\t.reg .b64 bd;\n\t.reg .pred pa, pt;\n\t"
+      "mov.b64 {blo, bhi}, %2;\n\t"
+      "setp.ne.b32 pa, %4, 0;\n\tsetp.eq.b32 pt, 0, 0;\n\t"
+      "add.u32 at, %1, 0;\n\tadd.u32 bl, blo, 0;\n\t"
+      "mov.b64 bd, {bl, bhi};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [at], bd, %3, pa;\n\t"
+      "add.u32 at, %1, 8;\n\tadd.u32 bl, blo, 128;\n\t"
+      "mov.b64 bd, {bl, bhi};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [at], bd, %3, pt;\n\t"
+      "add.u32 at, %1, 32;\n\tadd.u32 bl, blo, 256;\n\t"
+      "mov.b64 bd, {bl, bhi};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [at], bd, %3, pt;\n\t"
+      "add.u32 at, %1, 40;\n\tadd.u32 bl, blo, 384;\n\t"
+      "mov.b64 bd, {bl, bhi};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [at], bd, %3, pt;\n\t"
+      "}"
+      :: "r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 }  // namespace attn156
