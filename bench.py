@@ -580,6 +580,15 @@ def decode_bytes(w) -> float:
 DECODE_KERNEL_SOURCES = ["decode_sm100.cuh", "ptx.cuh", "common.cuh"]
 
 
+def decode_kernel_name(w) -> str:
+    """The split kernel attn_decode runs for a workload: keys on the lanes for
+    head_dim 128 with at most 16 query rows per K/V head, else rows on the lanes."""
+    if w["D"] == 128 and (w["H"] // w["Hk"]) * w["Sq"] <= 16:
+        return "attn_decode_t16_kernel"
+    return "attn_decode_kernel"
+
+
+
 def decode_oracle_inputs(w, rank: int = 0):
     from synth import bits_to_f32, make_inputs
     bits = make_inputs(w["B"], w["Sq"], w["Smax"], w["H"], w["D"], w["seed"] + rank,
@@ -717,11 +726,11 @@ def run_decode(args):
         "scaling": "weak", "vs_baseline": None, "dtype": args.dtype, "data": "synthetic",
         "config": decode_config(w),
         "roofline": {"bound": "hbm",
-                     "kernel": "attn_decode_t16_kernel (timed with its combine launch)",
+                     "kernel": f"{decode_kernel_name(w)} (timed with its combine launch)",
                      "achieved": decode_bytes(w) / (ms * 1e-3) / 1e9, "peak": peak,
                      "unit": "GB/s", "frac": decode_bytes(w) / (ms * 1e-3) / 1e9 / peak,
                      "peak_source": f"{peaks.get('source')} hbm_gbs",
-                     "traffic": committed_traffic(traffic_key("attn_decode_t16_kernel", w,
+                     "traffic": committed_traffic(traffic_key(decode_kernel_name(w), w,
                                                               args.dtype),
                                                   sources_sha(DECODE_KERNEL_SOURCES))},
         "e2e": {"value": world * decode_bytes(w) / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",

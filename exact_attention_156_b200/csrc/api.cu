@@ -28,6 +28,9 @@ namespace {
 __device__ uint32_t g_attn_err = 0;
 
 constexpr uint64_t kTimeoutNs = 1000000000ull;  // 1 s per device-side wait
+// Forward block order: pair-major while the K and V of all heads take at most
+// this many bytes (well inside the 126 MB L2, next to Q and O traffic).
+constexpr double kPairMajorMaxKV = 48.0 * 1024 * 1024;
 constexpr int kMaxDevices = 64;
 
 struct DeviceState {
@@ -95,9 +98,8 @@ attn_status device_state(DeviceState** out) {
         ok = ok &&
              set_smem(dec::attn_decode_kernel<D, E>, dec::Cfg<D>::kSmemBytes) == cudaSuccess &&
              set_smem(fwd256::attn_fwd_d256_kernel<E>, fwd256::Cfg::kSmemBytes) == cudaSuccess;
-        if constexpr (D == 128)
-          ok = ok && set_smem(dec::t16::attn_decode_t16_kernel<E>, dec::t16::Cfg::kSmemBytes) ==
-                         cudaSuccess;
+        ok = ok && set_smem(dec::t16::attn_decode_t16_kernel<D, E>, dec::t16::Cfg::kSmemBytes) ==
+                       cudaSuccess;
       };
       ok = ok &&
            set_smem(bwd256::attn_bwd_d256_kernel<ElemBF16>, bwd256::Cfg::kSmemBytes) ==
@@ -281,6 +283,12 @@ attn_status launch_fwd(const DeviceState& st, const void* q, const void* k, cons
   p.total_k = 0;
   p.num_mblocks = (Sq + fwd::NQ * fwd::BM - 1) / (fwd::NQ * fwd::BM);
   p.compact = 0;
+  // Block order: while every head's K and V fit in L2 together, nothing is lost
+  // by running the pairs of many heads at once, and pair-major order starts the
+  // longest causal CTAs of all heads first; larger problems keep the pairs of
+  // one head side by side so that they share its K/V tiles in L2.
+  const double kv_bytes = 2.0 * B * double(Sk) * Hk * D * 2.0;
+  p.pair_major = kv_bytes <= kPairMajorMaxKV ? 1 : 0;
   p.err = st.err;
   p.timeout_ns = kTimeoutNs;
   dim3 grid(p.num_mblocks, H, B);
@@ -289,7 +297,7 @@ attn_status launch_fwd(const DeviceState& st, const void* q, const void* k, cons
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_LAUNCH;
 }
 
-// head_dim 256 forward: one 128-row query tile per CTA, 64-key K/V tiles.
+// head_dim 256 forward: one 128-row query tile per CTA, 128-key K/V tiles.
 template <class E>
 attn_status launch_fwd_d256(const DeviceState& st, const void* q, const void* k, const void* v,
                             void* o, float* lse, int B, int Sq, int Sk, int H, int Hk, float scale,
@@ -341,7 +349,8 @@ template <int D, class E>
 attn_status launch_bwd_pre(const void* o, const void* dout, const float* lse, int B, int Sq,
                            int H, const Workspace& w, cudaStream_t stream) {
   const long long rows = (long long)B * H * w.Sq_pad;
-  const unsigned blocks = unsigned((rows + 7) / 8);
+  const long long per_block = 8LL * bwd::kPreRows;  // 8 warps of kPreRows rows
+  const unsigned blocks = unsigned((rows + per_block - 1) / per_block);
   // head_dim 256 writes dQ rows whole (no reduce-add), so its accumulator needs no clearing
   bwd::attn_bwd_pre_kernel<D, E><<<blocks, 256, 0, stream>>>(
       static_cast<const uint16_t*>(o), static_cast<const uint16_t*>(dout), lse, w.nlse2,
@@ -378,6 +387,10 @@ attn_status launch_bwd_main(const DeviceState& st, const void* q, const void* k,
   p.total_k = 0;
   p.R = 0;
   p.compact = 0;
+  // Block order (as in the forward): tile-major while the operands every CTA
+  // streams (Q, dO, the fp32 dQ accumulator) of all heads fit in L2 together.
+  const double stream_bytes = double(B) * H * double(Sq) * D * (2.0 + 2.0 + 4.0);
+  p.tile_major = stream_bytes <= kPairMajorMaxKV ? 1 : 0;
   p.Hk = Hk;
   p.scale = scale;
   p.scale_log2 = scale * 1.4426950408889634f;
@@ -578,6 +591,7 @@ attn_status launch_fwd_varlen(const DeviceState& st, const void* q, const void* 
   // (at most ceil(total_q / 256) + B of them); otherwise the longest sequence's
   // pair count for every sequence.
   p.compact = B <= kCompactMaxB ? 1 : 0;
+  p.pair_major = 0;
   const int rows = fwd::NQ * fwd::BM;
   dim3 grid = p.compact ? dim3((vl.total_q + rows - 1) / rows + B, H, 1)
                         : dim3(p.num_mblocks, H, B);
@@ -599,7 +613,8 @@ attn_status run_backward_varlen(const DeviceState& st, const void* q, const void
   float* nlse2 = dq_acc + rows * D;
   float* ndelta = nlse2 + rows;
   {
-    const unsigned blocks = unsigned((rows + 7) / 8);
+    const size_t per_block = 8 * bwd::kPreRows;  // 8 warps of kPreRows rows (R is a multiple of 4)
+    const unsigned blocks = unsigned((rows + per_block - 1) / per_block);
     bwd::attn_bwd_pre_varlen_kernel<D, E><<<blocks, 256, 0, stream>>>(
         static_cast<const uint16_t*>(o), static_cast<const uint16_t*>(dout), lse, nlse2, ndelta,
         dq_acc, vl.cu_q, vl.cu_k, B, H, vl.total_q, vl.total_k, vl.max_q, vl.max_k, int(R),
@@ -641,6 +656,7 @@ attn_status run_backward_varlen(const DeviceState& st, const void* q, const void
   // ceil(total_k / 128) + B of them); otherwise the longest sequence's tile
   // count for every sequence.
   p.compact = B <= kCompactMaxB ? 1 : 0;
+  p.tile_major = 0;
   dim3 grid = p.compact ? dim3((vl.total_k + bwd::BN - 1) / bwd::BN + B, Hk, 1)
                         : dim3((vl.max_k + bwd::BN - 1) / bwd::BN, Hk, B);
   bwd::attn_bwd_main_kernel<D, E, true>
@@ -728,12 +744,10 @@ attn_status launch_decode(const DeviceState& st, const void* q, const void* kc, 
   p.timeout_ns = kTimeoutNs;
   // at most 16 query rows per K/V head (one new token, up to 16 query heads
   // each): keys on the tensor-memory lanes; otherwise query rows on the lanes
-  bool transposed = false;
-  if constexpr (D == 128) transposed = group * Sq <= dec::t16::kRows;
-  if (transposed) {
-    if constexpr (D == 128)
-      dec::t16::attn_decode_t16_kernel<E><<<dim3(plan.nsplit, Hk, B), dec::t16::kThreads,
-                                            dec::t16::Cfg::kSmemBytes, stream>>>(mq, mk, mv, p);
+  if (group * Sq <= dec::t16::kRows) {
+    dec::t16::attn_decode_t16_kernel<D, E><<<dim3(plan.nsplit, Hk, B), dec::t16::kThreads,
+                                               dec::t16::Cfg::kSmemBytes, stream>>>(mq, mk, mv,
+                                                                                    p);
   } else {
     dec::attn_decode_kernel<D, E><<<dim3(plan.nsplit, Hk, B), dec::kThreads,
                                     dec::Cfg<D>::kSmemBytes, stream>>>(mq, mk, mv, p);

@@ -119,6 +119,7 @@ struct Params {
   const int* cu_k;
   int total_q, total_k, R;
   int compact;  // packed batches: blockIdx.x numbers the key tiles that have work (compact_tile)
+  int tile_major;  // (B, S, H, D) batches: block order tile-major instead of head-major
   int Hk;  // key/value heads: the CTA's K/V head is shared by H / Hk query heads
   float scale;
   float scale_log2;
@@ -128,65 +129,98 @@ struct Params {
 };
 
 // ---------------------------------------------------------------------------
-// 1. preprocess: one warp per (b, h, row of the padded query axis)
+// 1. preprocess: one warp per kPreRows consecutive rows of (b, h, padded query
+//    axis); the loads of all its rows are issued before any is reduced, so that
+//    enough bytes are in flight to keep HBM busy.
 // ---------------------------------------------------------------------------
+constexpr int kPreRows = 4;  // divides Sq_pad (a multiple of 128) and the packed R
+
+// One lane's share of a row of O or dO: D / 32 16-bit elements in D / 64 words.
+template <int D>
+__device__ __forceinline__ void load_row_words(const uint16_t* __restrict__ src,
+                                               uint32_t (&w)[D / 64]) {
+  const int lane = threadIdx.x % 32;
+  if constexpr (D == 256) {
+    const uint4 v = *reinterpret_cast<const uint4*>(src + lane * 8);
+    w[0] = v.x; w[1] = v.y; w[2] = v.z; w[3] = v.w;
+  } else if constexpr (D == 128) {
+    const uint2 v = *reinterpret_cast<const uint2*>(src + lane * 4);
+    w[0] = v.x; w[1] = v.y;
+  } else {
+    w[0] = *reinterpret_cast<const uint32_t*>(src + lane * 2);
+  }
+}
+
+// Lane sums of O∘dO for kPreRows rows, reduced over the warp; every lane gets
+// all kPreRows dot products.
+template <int D, class E>
+__device__ __forceinline__ void rows_dot(const uint32_t (&ow)[kPreRows][D / 64],
+                                         const uint32_t (&dw)[kPreRows][D / 64],
+                                         float (&dot)[kPreRows]) {
+#pragma unroll
+  for (int r = 0; r < kPreRows; ++r) {
+    dot[r] = 0.f;
+#pragma unroll
+    for (int t = 0; t < D / 64; ++t) {
+      float a0, a1, c0, c1;
+      E::unpack2(ow[r][t], a0, a1);
+      E::unpack2(dw[r][t], c0, c1);
+      dot[r] = fmaf(a0, c0, dot[r]);
+      dot[r] = fmaf(a1, c1, dot[r]);
+    }
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1)
+#pragma unroll
+    for (int r = 0; r < kPreRows; ++r) dot[r] += __shfl_xor_sync(0xffffffffu, dot[r], off);
+}
+
 template <int D, class E>
 __global__ void __launch_bounds__(256) attn_bwd_pre_kernel(
     const uint16_t* __restrict__ o, const uint16_t* __restrict__ dout,
     const float* __restrict__ lse, float* __restrict__ nlse2, float* __restrict__ ndelta,
     float* __restrict__ dq_acc, int B, int H, int Sq, int Sq_pad) {
-  const long long gw = (long long)blockIdx.x * 8 + threadIdx.x / 32;
+  const long long g0 = ((long long)blockIdx.x * 8 + threadIdx.x / 32) * kPreRows;
   const int lane = threadIdx.x % 32;
-  const long long rows = (long long)B * H * Sq_pad;
-  if (gw >= rows) return;
-  const int i = int(gw % Sq_pad);
-  const long long bh = gw / Sq_pad;
+  if (g0 >= (long long)B * H * Sq_pad) return;
+  // the warp's rows share (b, h): Sq_pad is a multiple of kPreRows
+  const int i0 = int(g0 % Sq_pad);
+  const long long bh = g0 / Sq_pad;
   const int h = int(bh % H);
   const int b = int(bh / H);
-  float dot = 0.f;
-  if (i < Sq) {
-    const size_t base = ((size_t(b) * Sq + i) * H + h) * D;
-    constexpr int kPer = D / 32;  // 16-bit elements per lane (2, 4 or 8)
-    uint32_t ow[kPer / 2], dw[kPer / 2];
-    if constexpr (kPer == 8) {
-      const uint4 ov = *reinterpret_cast<const uint4*>(o + base + lane * 8);
-      const uint4 dv = *reinterpret_cast<const uint4*>(dout + base + lane * 8);
-      ow[0] = ov.x; ow[1] = ov.y; ow[2] = ov.z; ow[3] = ov.w;
-      dw[0] = dv.x; dw[1] = dv.y; dw[2] = dv.z; dw[3] = dv.w;
-    } else if constexpr (kPer == 4) {
-      const uint2 ov = *reinterpret_cast<const uint2*>(o + base + lane * 4);
-      const uint2 dv = *reinterpret_cast<const uint2*>(dout + base + lane * 4);
-      ow[0] = ov.x; ow[1] = ov.y;
-      dw[0] = dv.x; dw[1] = dv.y;
-    } else {
-      ow[0] = *reinterpret_cast<const uint32_t*>(o + base + lane * 2);
-      dw[0] = *reinterpret_cast<const uint32_t*>(dout + base + lane * 2);
-    }
+  uint32_t ow[kPreRows][D / 64], dw[kPreRows][D / 64];
 #pragma unroll
-    for (int t = 0; t < kPer / 2; ++t) {
-      float a0, a1, c0, c1;
-      E::unpack2(ow[t], a0, a1);
-      E::unpack2(dw[t], c0, c1);
-      dot = fmaf(a0, c0, dot);
-      dot = fmaf(a1, c1, dot);
+  for (int r = 0; r < kPreRows; ++r) {
+    if (i0 + r < Sq) {
+      const size_t base = ((size_t(b) * Sq + i0 + r) * H + h) * D;
+      load_row_words<D>(o + base, ow[r]);
+      load_row_words<D>(dout + base, dw[r]);
+    } else {
+#pragma unroll
+      for (int t = 0; t < D / 64; ++t) ow[r][t] = dw[r][t] = 0u;
     }
   }
+  float dot[kPreRows];
+  rows_dot<D, E>(ow, dw, dot);
+  if (lane < kPreRows) {
+    // lane r writes row r (dot is warp-uniform after the reduction)
+    float dr = dot[0];
 #pragma unroll
-  for (int off = 16; off > 0; off >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, off);
-  if (lane == 0) {
-    const size_t r = size_t(bh) * Sq_pad + i;
+    for (int r = 1; r < kPreRows; ++r)
+      if (lane == r) dr = dot[r];
+    const int i = i0 + lane;
     float nl2 = -INFINITY;  // padding rows and rows that see no key: P = 0
     if (i < Sq) {
       const float l = lse[size_t(bh) * Sq + i];
       if (l != -INFINITY) nl2 = -l * 1.4426950408889634f;
     }
-    nlse2[r] = nl2;
-    ndelta[r] = -dot;
+    nlse2[g0 + lane] = nl2;
+    ndelta[g0 + lane] = -dr;
   }
   // (no accumulator to clear when dQ is written whole rather than reduced into)
   if (dq_acc == nullptr) return;
-  float4* acc = reinterpret_cast<float4*>(dq_acc + (size_t(bh) * Sq_pad + i) * D);
-  for (int c = lane; c < D / 4; c += 32) acc[c] = make_float4(0.f, 0.f, 0.f, 0.f);
+  float4* acc = reinterpret_cast<float4*>(dq_acc + size_t(g0) * D);
+  for (int c = lane; c < kPreRows * D / 4; c += 32) acc[c] = make_float4(0.f, 0.f, 0.f, 0.f);
 }
 
 // ---------------------------------------------------------------------------
@@ -247,60 +281,57 @@ __device__ __forceinline__ int find_seq(int B, long long x, KeyFn key) {
   return lo;
 }
 
-// One warp per row of the [H][R] row-value layout: Delta and -LSE*log2(e) of
-// query rows, neutral values (P = 0) for the padding rows, dQ accumulator zeroed.
+// One warp per kPreRows rows of the [H][R] row-value layout: Delta and
+// -LSE*log2(e) of query rows, neutral values (P = 0) for the padding rows, dQ
+// accumulator zeroed.  Sequence blocks start at multiples of 4 rows, so the
+// warp's rows lie in one sequence's block and one search finds it.
 template <int D, class E>
 __global__ void __launch_bounds__(256) attn_bwd_pre_varlen_kernel(
     const uint16_t* __restrict__ o, const uint16_t* __restrict__ dout,
     const float* __restrict__ lse, float* __restrict__ nlse2, float* __restrict__ ndelta,
     float* __restrict__ dq_acc, const int* __restrict__ cu_q, const int* __restrict__ cu_k, int B,
     int H, int total_q, int total_k, int max_q, int max_k, int R, uint32_t* err) {
-  const long long gw = (long long)blockIdx.x * 8 + threadIdx.x / 32;
+  static_assert(kPreRows == 4, "sequence blocks are aligned to 4 rows");
+  const long long g0 = ((long long)blockIdx.x * 8 + threadIdx.x / 32) * kPreRows;
   const int lane = threadIdx.x % 32;
-  if (gw >= (long long)H * R) return;
-  const int h = int(gw / R);
-  const long long y = gw % R;
-  const int b = find_seq(B, y, [&](int c) { return rv_start(cu_q, c); });
+  if (g0 >= (long long)H * R) return;
+  const int h = int(g0 / R);
+  const long long y0 = g0 % R;
+  const int b = find_seq(B, y0, [&](int c) { return rv_start(cu_q, c); });
   const SeqSpan sp = seq_span(cu_q, cu_k, b, total_q, total_k, max_q, max_k);
   if (!sp.ok && lane == 0 && h == 0) atomicCAS(err, 0u, kErrSeqlens);
-  const long long i = y - rv_start(cu_q, b);  // query index in the sequence
-  const bool real = sp.ok && i >= 0 && i < sp.Lq;
-  float dot = 0.f;
-  if (real) {
-    const size_t base = ((size_t(sp.q0) + size_t(i)) * H + h) * D;
-    constexpr int kPer = D / 32;
-    uint32_t ow[kPer / 2], dw[kPer / 2];
-    if constexpr (kPer == 4) {
-      const uint2 ov = *reinterpret_cast<const uint2*>(o + base + lane * 4);
-      const uint2 dv = *reinterpret_cast<const uint2*>(dout + base + lane * 4);
-      ow[0] = ov.x; ow[1] = ov.y;
-      dw[0] = dv.x; dw[1] = dv.y;
-    } else {
-      ow[0] = *reinterpret_cast<const uint32_t*>(o + base + lane * 2);
-      dw[0] = *reinterpret_cast<const uint32_t*>(dout + base + lane * 2);
-    }
+  const long long i0 = y0 - rv_start(cu_q, b);  // query index of the first row in the sequence
+  uint32_t ow[kPreRows][D / 64], dw[kPreRows][D / 64];
 #pragma unroll
-    for (int t = 0; t < kPer / 2; ++t) {
-      float a0, a1, c0, c1;
-      E::unpack2(ow[t], a0, a1);
-      E::unpack2(dw[t], c0, c1);
-      dot = fmaf(a0, c0, dot);
-      dot = fmaf(a1, c1, dot);
+  for (int r = 0; r < kPreRows; ++r) {
+    const long long i = i0 + r;
+    if (sp.ok && i >= 0 && i < sp.Lq) {
+      const size_t base = ((size_t(sp.q0) + size_t(i)) * H + h) * D;
+      load_row_words<D>(o + base, ow[r]);
+      load_row_words<D>(dout + base, dw[r]);
+    } else {
+#pragma unroll
+      for (int t = 0; t < D / 64; ++t) ow[r][t] = dw[r][t] = 0u;
     }
   }
+  float dot[kPreRows];
+  rows_dot<D, E>(ow, dw, dot);
+  if (lane < kPreRows) {
+    float dr = dot[0];
 #pragma unroll
-  for (int off = 16; off > 0; off >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, off);
-  if (lane == 0) {
+    for (int r = 1; r < kPreRows; ++r)
+      if (lane == r) dr = dot[r];
+    const long long i = i0 + lane;
     float nl2 = -INFINITY;
-    if (real) {
+    if (sp.ok && i >= 0 && i < sp.Lq) {
       const float l = lse[size_t(h) * total_q + size_t(sp.q0) + size_t(i)];
       if (l != -INFINITY) nl2 = -l * 1.4426950408889634f;
     }
-    nlse2[gw] = nl2;
-    ndelta[gw] = -dot;
+    nlse2[g0 + lane] = nl2;
+    ndelta[g0 + lane] = -dr;
   }
-  float4* acc = reinterpret_cast<float4*>(dq_acc + size_t(gw) * D);
-  for (int c = lane; c < D / 4; c += 32) acc[c] = make_float4(0.f, 0.f, 0.f, 0.f);
+  float4* acc = reinterpret_cast<float4*>(dq_acc + size_t(g0) * D);
+  for (int c = lane; c < kPreRows * D / 4; c += 32) acc[c] = make_float4(0.f, 0.f, 0.f, 0.f);
 }
 
 // dq[x, h, :] = 16-bit(scale * acc[h][rv_start(b) + i]) for packed row x =
@@ -371,12 +402,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     return;
   }
 
-  // Grid: (key tile, K/V head, batch).  The key tiles of one head run side by
-  // side, so they share that head's Q and dO tiles in L2; low key tiles (the
-  // most query tiles when causal) start first.
-  int kt = blockIdx.x;
-  const int hk = blockIdx.y;  // key/value head
-  int b = blockIdx.z;
+  // Grid: (key tile, K/V head, batch).  Head-major order: the key tiles of one
+  // head run side by side, so they share that head's Q and dO tiles in L2; low
+  // key tiles (the most query tiles when causal) start first.  Tile-major order
+  // (problems whose streamed operands fit in L2 all at once): the linear block
+  // index walks key tile 0 of every (head, batch), then tile 1, ..., so the
+  // longest CTAs of all heads start in the first wave.
+  int kt = blockIdx.x, hk = blockIdx.y, b = blockIdx.z;  // hk: key/value head
+  if (p.tile_major) {
+    const int lin = int(blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z));
+    const int nbh = p.Hk * p.B;
+    kt = lin / nbh;
+    const int rem = lin - kt * nbh;
+    hk = rem % p.Hk;
+    b = rem / p.Hk;
+  }
   if constexpr (kVarlen) {
     if (p.compact) {
       // one CTA per key tile that has work, low key tiles (the heaviest when

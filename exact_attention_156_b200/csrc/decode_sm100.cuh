@@ -398,17 +398,19 @@ __global__ void __launch_bounds__(kThreads, 1)
 //   S^T = K Q^T      (M = 128 keys, N = 16 rows; A = K tile, B = Q, both K-major)
 //   O^T += V^T P^T   (M = 128 = head_dim, N = 16 rows; A = V tile read MN-major,
 //                     B = P^T from shared memory, K-major over the keys)
-// so each softmax thread owns one key and 16 scores.  The row maximum is a
+// so each softmax thread owns one key and 16 scores.  At head_dim 64 the same
+// kernel runs with M = 128 for O^T: the K/V slots keep two 64-column boxes, only
+// the first is loaded, and the second is cleared once, so rows 64..127 of O^T
+// stay zero and are never written out.  The row maximum is a
 // reduction over the 128 threads (shuffles within a warp, then shared memory
 // across the four warps); row sums stay per thread until the end.  P^T is
 // written as 16-bit values into a double-buffered 4 KB shared tile.
 namespace t16 {
 constexpr int kRows = 16;       // N of both products
 constexpr int kThreads = 224;   // warps 0-3 softmax, 4 MMA, 5 Q/K loads, 6 V loads
-constexpr int kD = 128;
 struct Cfg {
   static constexpr int kBoxBytes = BN * 128;         // K/V box: 128 rows x 64 columns
-  static constexpr int kTileBytes = BN * kD * 2;      // K or V tile (2 boxes)
+  static constexpr int kTileBytes = 2 * kBoxBytes;    // K or V slot (2 boxes, head_dim <= 128)
   static constexpr int kSmallBox = kRows * 128;       // Q / P^T box: 16 rows x 64 columns
   static constexpr int kSlots = 3;
   static constexpr int kQOff = 0;                                  // 2 small boxes
@@ -454,13 +456,16 @@ __device__ __forceinline__ float warp_reduce16(float (&v)[kRows], Op op) {
   return op(v[0], __shfl_xor_sync(0xffffffffu, v[0], 1));
 }
 
-template <class E>
+// D: head_dim, 64 or 128.
+template <int D, class E>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_decode_t16_kernel(const __grid_constant__ CUtensorMap tmQ,
                            const __grid_constant__ CUtensorMap tmK,
                            const __grid_constant__ CUtensorMap tmV, const Params p) {
+  static_assert(D == 64 || D == 128, "head_dim 64 or 128");
   using C = Cfg;
-  constexpr int D = kD;
+  constexpr int kBoxes = D / 64;                 // 64-column boxes loaded per K/V tile
+  constexpr int kLoadBytes = BN * D * 2;         // bytes landing per K/V tile
   extern __shared__ __align__(1024) uint8_t smem[];
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
@@ -494,6 +499,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   // Q rows past `rows` are never loaded: zero the two small boxes once.
   for (int e = threadIdx.x; e < 2 * C::kSmallBox / 16; e += kThreads)
     reinterpret_cast<uint4*>(smem + C::kQOff)[e] = make_uint4(0u, 0u, 0u, 0u);
+  if constexpr (D == 64) {
+    // second box of every V slot: rows 64..127 of the M = 128 product O^T
+    for (int e = threadIdx.x; e < C::kSlots * C::kBoxBytes / 16; e += kThreads) {
+      const int sl = e / (C::kBoxBytes / 16), off = e % (C::kBoxBytes / 16);
+      reinterpret_cast<uint4*>(smem + C::kVOff + sl * C::kTileBytes + C::kBoxBytes)[off] =
+          make_uint4(0u, 0u, 0u, 0u);
+    }
+  }
   fence_proxy_async_smem();
   if (warp == 0) {
     tmem_alloc(smem_u32(tmem_slot), C::kTmemCols);
@@ -652,7 +665,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (key >= L) {
           const uint32_t vrow = v_addr(t % C::kSlots) + uint32_t(j) * 128;
 #pragma unroll
-          for (int x = 0; x < 2; ++x)
+          for (int x = 0; x < kBoxes; ++x)
 #pragma unroll
             for (int k = 0; k < 8; ++k)
               st_shared_v4(vrow + x * C::kBoxBytes + k * 16, 0u, 0u, 0u, 0u);
@@ -684,10 +697,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int c = 0; c < kRows; ++c) rr[c] = 0u;
       }
-      const int d = j;  // O^T lane = head-dim index
+      const int d = j;  // O^T lane = head-dim index (lanes D..127 hold zeros at D = 64)
 #pragma unroll
       for (int c = 0; c < kRows; ++c) {
-        if (c >= rows) break;
+        if (c >= rows || d >= D) break;
         const float l = rl[c] + rl[kRows + c] + rl[2 * kRows + c] + rl[3 * kRows + c];
         const int i = c / p.group;
         const int h = g * p.group + c % p.group;
@@ -707,7 +720,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_prefetch_desc(&tmQ);
       tma_prefetch_desc(&tmK);
       mbar_arrive_expect_tx(bar(C::kBarQ), rows * D * 2);
-      for (int x = 0; x < 2; ++x)
+      for (int x = 0; x < kBoxes; ++x)
         tma_load_4d(sbase + C::kQOff + x * C::kSmallBox, &tmQ, bar(C::kBarQ), x * 64,
                     g * p.group, 0, b);
       for (int t = 0; t < n_kv; ++t) {
@@ -715,8 +728,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int u = t / C::kSlots;
         if (u > 0 && !bw.wait(bar(C::kBarKEmpty + s), (u - 1) & 1, 65)) break;
         const uint32_t fb = bar(C::kBarKFull + s);
-        mbar_arrive_expect_tx(fb, C::kTileBytes);
-        for (int x = 0; x < 2; ++x)
+        mbar_arrive_expect_tx(fb, kLoadBytes);
+        for (int x = 0; x < kBoxes; ++x)
           tma_load_4d(k_addr(s) + x * C::kBoxBytes, &tmK, fb, x * 64, g, (j0 + t) * BN, b);
       }
     }
@@ -729,15 +742,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int u = t / C::kSlots;
         if (u > 0 && !bw.wait(bar(C::kBarVEmpty + s), (u - 1) & 1, 66)) break;
         const uint32_t fb = bar(C::kBarVFull + s);
-        mbar_arrive_expect_tx(fb, C::kTileBytes);
-        for (int x = 0; x < 2; ++x)
+        mbar_arrive_expect_tx(fb, kLoadBytes);
+        for (int x = 0; x < kBoxes; ++x)
           tma_load_4d(v_addr(s) + x * C::kBoxBytes, &tmV, fb, x * 64, g, (j0 + t) * BN, b);
       }
     }
   } else if (warp == kMmaWarp) {
     if (lane == 0 && n_kv > 0) {
       constexpr uint32_t idesc_s = idesc_f32acc(BN, kRows, false, false, E::kFmt);
-      constexpr uint32_t idesc_o = idesc_f32acc(D, kRows, true, false, E::kFmt);
+      constexpr uint32_t idesc_o = idesc_f32acc(128, kRows, true, false, E::kFmt);  // M = 128 rows of O^T
       const uint64_t q_desc = sdesc_sw128(sbase + C::kQOff, 16);
       bool ok = bw.wait(bar(C::kBarQ), 0, 67);
       // S^T(t) into buffer t % 2 once K(t) has landed (the K slot is handed
@@ -747,8 +760,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int s = t % C::kSlots;
         if (!bw.wait(bar(C::kBarKFull + s), (t / C::kSlots) & 1, 68)) return false;
         tc_fence_after();
-        mma_chain_kk8_b16(tmem + uint32_t((t & 1) * kRows), sdesc_sw128(k_addr(s), 16), q_desc,
-                          idesc_s, 0u);
+        if constexpr (D == 128)
+          mma_chain_kk8_b16(tmem + uint32_t((t & 1) * kRows), sdesc_sw128(k_addr(s), 16), q_desc,
+                            idesc_s, 0u);
+        else
+          mma_chain_kk4(tmem + uint32_t((t & 1) * kRows), sdesc_sw128(k_addr(s), 16), q_desc,
+                        idesc_s, 0u);
         tc_commit(bar(C::kBarS + (t & 1)));
         tc_commit(bar(C::kBarKEmpty + s));
         return true;

@@ -93,6 +93,7 @@ struct Params {
   int causal, win_left, win_right;
   int num_mblocks;   // ceil(Sq / (NQ * BM))
   int compact;       // packed batches: blockIdx.x numbers the tiles that have work (compact_tile)
+  int pair_major;    // (B, S, H, D) batches: block order pair-major instead of head-major
   uint32_t* err;
   uint64_t timeout_ns;
 };
@@ -132,13 +133,24 @@ __global__ void __launch_bounds__(kThreads, 1)
     return;
   }
 
-  // Grid: (query-tile pair, head, batch).  The pairs of one head run side by
-  // side, so they share that head's K/V tiles in L2; causal launches each
-  // head's pairs with the most keys first.
-  int mb = p.causal ? (p.num_mblocks - 1 - int(blockIdx.x)) : int(blockIdx.x);
-  const int h = blockIdx.y;
+  // Grid: (query-tile pair, head, batch).  Head-major order: the pairs of one
+  // head run side by side, so they share that head's K/V tiles in L2; causal
+  // launches each head's pairs with the most keys first.  Pair-major order
+  // (problems whose K/V fit in L2 all at once): the linear block index walks
+  // pair 0 of every (head, batch), then pair 1, ..., so under a causal mask the
+  // longest CTAs of all heads start in the first wave instead of trailing
+  // behind the lighter pairs of the heads before them.
+  int pr = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  if (p.pair_major) {
+    const int lin = int(blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z));
+    const int nbh = p.H * p.B;
+    pr = lin / nbh;
+    const int rem = lin - pr * nbh;
+    h = rem % p.H;
+    b = rem / p.H;
+  }
+  int mb = p.causal ? (p.num_mblocks - 1 - pr) : pr;
   const int hk = h / (p.H / p.Hk);  // the key/value head this query head reads
-  int b = blockIdx.z;
   if constexpr (kVarlen) {
     if (p.compact) {
       // one CTA per query-tile pair that has work, the heaviest pairs first

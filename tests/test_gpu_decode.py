@@ -1,7 +1,7 @@
 """KV-cache decode (attn_decode): the CUDA path against the float64 oracle's
 attention_decode on the same seeded inputs, with the forward parity bars.
-Cases with head_dim 128 and at most 16 query rows per K/V head run the
-keys-on-lanes kernel, the others the rows-on-lanes kernel.
+Cases with at most 16 query rows per K/V head run the keys-on-lanes kernel,
+the others the rows-on-lanes kernel; both at head_dim 64 and 128.
 Cache rows past each sequence's length are filled with NaN and huge values:
 they must not reach the result."""
 import numpy as np
@@ -24,6 +24,9 @@ CASES = [
     (2, 1, 2048, 16, 1, 128, 0, (2048, 1500), "bf16"),     # 16 query heads on one K/V head
     (3, 1, 777, 4, 4, 128, 1, (777, 1, 129), "f16"),       # one row per K/V head, a one-key cache
     (1, 8, 1024, 2, 1, 128, 1, (1000,), "bf16"),           # 8 new positions x 2 heads, causal
+    (2, 2, 1024, 16, 1, 64, 1, (1000, 77), "bf16"),        # 32 rows per K/V head: rows on the lanes
+    (2, 1, 2048, 16, 1, 64, 0, (2048, 1500), "f16"),       # head_dim 64, 16 query heads on one
+    (2, 5, 600, 6, 2, 64, 1, (3, 600), "bf16"),            # 15 rows per K/V head, L < Sq
 ]
 
 
@@ -47,15 +50,17 @@ def test_decode_against_the_oracle(case):
     check_fwd(to_f64(o), lse.cpu().numpy().astype(np.float64), o_ref, lse_ref, str(case))
 
 
-def test_decode_bench_workload_in_full():
-    """The benchmark's decode workload itself (B8, one new row, H32 Hk8, 8192
-    cached rows, D128, inputs N(0,1)*0.5, the seed bench.py uses), every output
-    row against the oracle, through the same call the benchmark times."""
+@pytest.mark.parametrize("name", ["DECODE_WORKLOAD", "DECODE64_WORKLOAD"])
+def test_decode_bench_workload_in_full(name):
+    """The benchmark's decode workloads themselves (B8, one new row, H32 Hk8,
+    8192 cached rows, D128 or D64, inputs N(0,1)*0.5, the seeds bench.py uses),
+    every output row against the oracle, through the same call the benchmark
+    times."""
     import torch
     import bench
     from exact_attention_156_b200 import (attn_decode, attn_decode_workspace_size,
                                           get_last_device_error)
-    w = bench.DECODE_WORKLOAD
+    w = getattr(bench, name)
     B, Sq, H, Hk, S, D = w["B"], w["Sq"], w["H"], w["Hk"], w["Smax"], w["D"]
     bits = make_inputs(B, Sq, S, H, D, w["seed"], w["input_scale"], Hk=Hk)
     q, k, v = (to_device(bits[n]) for n in ("q", "k", "v"))
@@ -68,4 +73,4 @@ def test_decode_bench_workload_in_full():
     o_ref, lse_ref = oracle.attention_decode(f64(bits["q"]), f64(bits["k"]), f64(bits["v"]),
                                              [S] * B, 1.0 / np.sqrt(D), w["causal"])
     check_fwd(to_f64(o), lse.cpu().numpy().astype(np.float64), o_ref, lse_ref,
-              "decode bench workload")
+              f"decode bench workload {w['name']}")
