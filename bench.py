@@ -79,7 +79,8 @@ ORACLE_FULL = [
 ]
 WORKLOADS = {"fwdbwd": WORKLOAD, "gqa": GQA_WORKLOAD, "decode": DECODE_WORKLOAD,
              "decode64": DECODE64_WORKLOAD,
-             "varlen": VARLEN_WORKLOAD, "d256": D256_WORKLOAD, "d256fwd": D256_WORKLOAD,
+             "varlen": VARLEN_WORKLOAD, "padded": VARLEN_WORKLOAD,
+             "d256": D256_WORKLOAD, "d256fwd": D256_WORKLOAD,
              "fwd64": FWD64_WORKLOAD,
              "fwdsweep": None}
 D256_FWD_METRIC = "attention fwd TFLOPS, head_dim 256, bf16 vs B200 dense BF16 peak"
@@ -762,7 +763,17 @@ def varlen_fwd_flops(w, lengths) -> float:
     return f / 2 if w["causal"] else f
 
 
-def varlen_config(w, lengths):
+def varlen_config(w, lengths, padded=False):
+    if padded:
+        B, S = len(lengths), max(lengths)
+        return {"workload": f"padded_b{B}s{S}h{w['H']}d{w['D']}_fwdbwd: fwd+bwd of a padded batch "
+                            f"(B={B}, S={S}, H={w['H']}, D={w['D']}) holding the {w['name']} "
+                            f"sequences ({min(lengths)}..{max(lengths)} tokens, lengths "
+                            f"log-uniform in [{w['len_lo']}, {w['len_hi']}]) with per-sequence "
+                            f"lengths, causal, inputs N(0,1)*{w['input_scale']}, padding rows zero",
+                "B": B, "S": S, "real_tokens": w["total"], "H": w["H"], "D": w["D"],
+                "causal": bool(w["causal"]),
+                "l2": "no flush: inputs (Q,K,V,dO 3.9 GB) exceed the 126 MB L2"}
     return {"workload": f"{w['name']}: fwd+bwd of a packed batch, {len(lengths)} sequences of "
                         f"{min(lengths)}..{max(lengths)} tokens ({w['total']} in all, lengths "
                         f"log-uniform in [{w['len_lo']}, {w['len_hi']}]), H={w['H']} "
@@ -820,7 +831,7 @@ def run_varlen_reference(args):
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": tot_s / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": varlen_config(w, lengths),
+        "config": varlen_config(w, lengths, args.workload == "padded"),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
                          "sample": f"each step: fwd+bwd of one seeded (sequence, head) of "
                                    f"{w['name']}, float64 numpy"},
@@ -830,7 +841,9 @@ def run_varlen_reference(args):
 
 
 def run_varlen(args):
-    """fwd + bwd of a packed variable-length batch (one step = both calls)."""
+    """fwd + bwd of a packed variable-length batch (one step = both calls); with
+    --workload padded, the same sequences in (B, S, H, D) tensors through
+    attn_fwd_padded / attn_bwd_padded."""
     import numpy as np
     import torch
     rank, world, local = dist_env()
@@ -841,39 +854,67 @@ def run_varlen(args):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     device = torch.device("cuda", local if world > 1 else torch.cuda.current_device())
     torch.cuda.set_device(device)
-    from exact_attention_156_b200 import (attn_bwd_varlen, attn_bwd_varlen_workspace_size,
+    from exact_attention_156_b200 import (attn_bwd_padded, attn_bwd_padded_workspace_size,
+                                          attn_bwd_varlen, attn_bwd_varlen_workspace_size,
+                                          attn_fwd_padded, attn_fwd_padded_workspace_size,
                                           attn_fwd_varlen, get_last_device_error)
     from synth import make_inputs
+    padded = args.workload == "padded"
     w = VARLEN_WORKLOAD
     lengths = varlen_lengths(w)
     T, H, D = w["total"], w["H"], w["D"]
+    Bp, Lmax = len(lengths), max(lengths)
     bits = make_inputs(1, T, T, H, D, w["seed"] + rank, w["input_scale"], with_dout=True,
                        Hk=w["Hk"], fmt=args.dtype)
     tdtype = torch.float16 if args.dtype == "f16" else torch.bfloat16
-    host = {n: torch.from_numpy(bits[n][0].view("int16")).view(tdtype).pin_memory()
-            for n in ("q", "k", "v", "do")}
-    cu_host = torch.from_numpy(np.concatenate([[0], np.cumsum(lengths)]).astype(np.int32))
-    host["cu"] = cu_host.pin_memory()
+    if padded:
+        # sequence b's rows first in row block b, zeros after them
+        starts = np.concatenate([[0], np.cumsum(lengths)])
+        host = {}
+        for n in ("q", "k", "v", "do"):
+            a = np.zeros((Bp, Lmax, H, D), dtype=np.int16)
+            for b, L in enumerate(lengths):
+                a[b, :L] = bits[n][0][starts[b]:starts[b] + L].view(np.int16)
+            host[n] = torch.from_numpy(a).view(tdtype).pin_memory()
+        host["cu"] = torch.tensor(lengths, dtype=torch.int32).pin_memory()  # seqlens
+    else:
+        host = {n: torch.from_numpy(bits[n][0].view("int16")).view(tdtype).pin_memory()
+                for n in ("q", "k", "v", "do")}
+        cu_host = torch.from_numpy(np.concatenate([[0], np.cumsum(lengths)]).astype(np.int32))
+        host["cu"] = cu_host.pin_memory()
     dev = {n: t.to(device) for n, t in host.items()}
     q, k, v, do, cu = dev["q"], dev["k"], dev["v"], dev["do"], dev["cu"]
-    Lmax = max(lengths)
     o = torch.empty_like(q)
-    lse = torch.empty((H, T), dtype=torch.float32, device=device)
+    lse = torch.empty((Bp, H, Lmax) if padded else (H, T), dtype=torch.float32, device=device)
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
-    ws = torch.empty(attn_bwd_varlen_workspace_size(len(lengths), T, H, D), dtype=torch.uint8,
-                     device=device)
+    if padded:
+        ws_f = torch.empty(attn_fwd_padded_workspace_size(Bp, Lmax, Lmax, H, H, D),
+                           dtype=torch.uint8, device=device)
+        ws = torch.empty(attn_bwd_padded_workspace_size(Bp, Lmax, Lmax, H, H, D),
+                         dtype=torch.uint8, device=device)
+    else:
+        ws = torch.empty(attn_bwd_varlen_workspace_size(Bp, T, H, D), dtype=torch.uint8,
+                         device=device)
     stream = torch.cuda.current_stream(device)
     causal = bool(w["causal"])
 
     def step(evs=None):
         if evs is not None:
             evs[0].record(stream)
-        attn_fwd_varlen(q, k, v, cu, cu, Lmax, Lmax, causal=causal, out=o, lse=lse,
-                        stream=stream)
+        if padded:
+            attn_fwd_padded(q, k, v, cu, cu, causal=causal, out=o, lse=lse, workspace=ws_f,
+                            stream=stream)
+        else:
+            attn_fwd_varlen(q, k, v, cu, cu, Lmax, Lmax, causal=causal, out=o, lse=lse,
+                            stream=stream)
         if evs is not None:
             evs[1].record(stream)
-        attn_bwd_varlen(q, k, v, o, do, lse, cu, cu, Lmax, Lmax, causal=causal, dq=dq, dk=dk,
-                        dv=dv, workspace=ws, stream=stream)
+        if padded:
+            attn_bwd_padded(q, k, v, o, do, lse, cu, cu, causal=causal, dq=dq, dk=dk, dv=dv,
+                            workspace=ws, stream=stream)
+        else:
+            attn_bwd_varlen(q, k, v, o, do, lse, cu, cu, Lmax, Lmax, causal=causal, dq=dq,
+                            dk=dk, dv=dv, workspace=ws, stream=stream)
         if evs is not None:
             evs[2].record(stream)
 
@@ -935,16 +976,22 @@ def run_varlen(args):
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": args.dtype, "data": "synthetic",
-        "config": varlen_config(w, lengths),
+        "config": varlen_config(w, lengths, padded),
         "roofline": {"bound": "tensor",
-                     "kernel": "attn_bwd_varlen (preprocess + main + dQ finalize launches)",
+                     "kernel": ("attn_bwd_padded (gathers, scans, preprocess + main + dQ "
+                                "finalize, scatters)" if padded else
+                                "attn_bwd_varlen (preprocess + main + dQ finalize launches)"),
                      "achieved": bwd_tf, "peak": peak, "unit": "TFLOP/s", "frac": bwd_tf / peak,
                      "peak_source": f"{peaks.get('source')} bf16_tflops (burst)",
                      "traffic": None},
-        "kernels": {"fwd_varlen": {"ms": fwd_ms, "tflops": fwd_tf, "frac": fwd_tf / peak},
-                    "bwd_varlen": {"ms": bwd_ms, "tflops": bwd_tf, "frac": bwd_tf / peak}},
+        "kernels": {("fwd_padded" if padded else "fwd_varlen"):
+                    {"ms": fwd_ms, "tflops": fwd_tf, "frac": fwd_tf / peak},
+                    ("bwd_padded" if padded else "bwd_varlen"):
+                    {"ms": bwd_ms, "tflops": bwd_tf, "frac": bwd_tf / peak}},
         "e2e": e2e,
-        "gpu_launches": 4 * args.steps,
+        # padded: forward 2 scans + 3 gathers + kernel + 2 scatters; backward 2 scans +
+        # 6 gathers + 3 kernels + 3 scatters
+        "gpu_launches": (22 if padded else 4) * args.steps,
         "clocks": clocks,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -1202,7 +1249,8 @@ def main(argv=None):
                     help="fwdbwd: the headline fwd+bwd workload (default); gqa: the same sizes "
                          "with 8 K/V heads for 32 query heads; decode: KV-cache decode "
                          "(B8 H32 Hk8, 8192 cached rows, one new row); varlen: a packed batch "
-                         "of 32768 tokens in sequences of 128..4096; d256: head_dim 256 forward + "
+                         "of 32768 tokens in sequences of 128..4096; padded: the same sequences "
+                         "in (B, S, H, D) tensors with per-sequence lengths; d256: head_dim 256 forward + "
                          "backward, B1 H16 S8192 causal; d256fwd: its forward alone; fwd64: the "
                          "head_dim 64 forward alone, B2 H32 S8192 causal; decode64: the decode "
                          "step at head_dim 64; fwdsweep: the forward alone on C2-C4")
@@ -1217,7 +1265,7 @@ def main(argv=None):
         ap.error("--warmup must be >= 3")
     if args.workload in ("decode", "decode64"):
         return run_decode_reference(args) if args.impl == "reference" else run_decode(args)
-    if args.workload == "varlen":
+    if args.workload in ("varlen", "padded"):
         return run_varlen_reference(args) if args.impl == "reference" else run_varlen(args)
     if args.workload in ("d256fwd", "fwd64"):
         return run_fwd_only_reference(args) if args.impl == "reference" else run_fwd_only(args)

@@ -553,7 +553,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const bool full = key_ok && n0 + BN - 1 <= Lk - 1 && i0 + BM - 1 <= Lq - 1 &&
                           i0 >= g.qmin(n0 + BN - 1) && i0 + BM - 1 <= g.qmax(n0);
         if (full) {
-          // every entry visible: a quarter of the exponentials on the FMA pipe
+          // every entry visible: no mask
 #pragma unroll
           for (int c = 0; c < BM; c += 4) {
             const float4 l4 = nl[c / 4];
@@ -564,15 +564,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 f2_pack(l4.z, l4.w));
             float a0, a1, a2, a3;
             f2_unpack(x0, a0, a1);
+            f2_unpack(x1, a2, a3);
             pw[c / 2] = E::pack2(ex2_approx(a0), ex2_approx(a1));
-            if ((c & 7) == 4) {
-              f2_unpack(f2_exp2_poly(x1), a2, a3);
-            } else {
-              f2_unpack(x1, a2, a3);
-              a2 = ex2_approx(a2);
-              a3 = ex2_approx(a3);
-            }
-            pw[c / 2 + 1] = E::pack2(a2, a3);
+            pw[c / 2 + 1] = E::pack2(ex2_approx(a2), ex2_approx(a3));
           }
         } else {
           const int c_lo = key_ok ? qmin_k - i0 : (1 << 30);

@@ -308,16 +308,6 @@ __global__ void __launch_bounds__(32, 1)
     for (int e = threadIdx.x; e < 2 * kBox; e += 32) out[e] = smem[e];
 }
 
-__global__ void diag_exp2_kernel(const float* x, float* y, int n) {
-  const int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
-  if (i + 1 < n) {
-    float r0, r1;
-    f2_unpack(f2_exp2_poly(f2_pack(x[i], x[i + 1])), r0, r1);
-    y[i] = r0;
-    y[i + 1] = r1;
-  }
-}
-
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
@@ -400,15 +390,6 @@ __attribute__((visibility("default"))) int attn_diag_tma(const void* A, void* ou
   diag_tma_kernel<<<1, 32, smem, static_cast<cudaStream_t>(stream)>>>(map,
                                                                        static_cast<uint8_t*>(out));
   return cudaGetLastError() == cudaSuccess ? 0 : 5;
-}
-
-// y = the softmax's polynomial 2^x (pairs); n must be even.
-__attribute__((visibility("default"))) int attn_diag_exp2(const float* x, float* y, int n,
-                                                          void* stream) {
-  if (!x || !y || n <= 0 || (n & 1)) return 1;
-  const int pairs = n / 2;
-  diag_exp2_kernel<<<(pairs + 255) / 256, 256, 0, static_cast<cudaStream_t>(stream)>>>(x, y, n);
-  return cudaGetLastError() == cudaSuccess ? 0 : 3;
 }
 
 __attribute__((visibility("default"))) int attn_diag_error(void) {

@@ -324,39 +324,24 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint64_t acc2[4];
 #pragma unroll
       for (int a = 0; a < 4; ++a) acc2[a] = 0ull;  // (+0.0f, +0.0f)
-      // p = 2^(s * scale * log2(e) - m): pairs in f32x2.  On fully visible
-      // tiles one pair in four is exponentiated on the FMA pipe (polynomial),
-      // the rest on MUFU; tiles with masked (-inf) scores use MUFU only, whose
-      // ex2(-inf) is exactly 0.  P goes to tensor memory as 16-bit pairs in two
-      // 64-column halves (columns [0,32) and [32,64) of S_k).
-      auto exp_store = [&](auto use_poly) {
+      // p = 2^(s * scale * log2(e) - m): the scale and subtract as f32x2 pairs,
+      // the exponentials on MUFU (ex2(-inf) is exactly 0 for masked scores).
+      // P goes to tensor memory as 16-bit pairs in two 64-column halves
+      // (columns [0,32) and [32,64) of S_k).
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          uint32_t pk[32];
+      for (int half = 0; half < 2; ++half) {
+        uint32_t pk[32];
 #pragma unroll
-          for (int c = 0; c < 32; ++c) {
-            const int e = half * 64 + 2 * c;
-            const uint64_t x2 = f2_fma(f2_pack(s[e], s[e + 1]), scale2, negm2);
-            uint64_t p2;
-            if (decltype(use_poly)::value && (c & 3) == 3) {
-              p2 = f2_exp2_poly(x2);
-            } else {
-              float x0, x1;
-              f2_unpack(x2, x0, x1);
-              p2 = f2_pack(ex2_approx(x0), ex2_approx(x1));
-            }
-            acc2[c & 3] = f2_add(acc2[c & 3], p2);
-            float p0, p1;
-            f2_unpack(p2, p0, p1);
-            pk[c] = E::pack2(p0, p1);
-          }
-          tmem_st32(tS + half * 32, pk);
+        for (int c = 0; c < 32; ++c) {
+          const int e = half * 64 + 2 * c;
+          const uint64_t x2 = f2_fma(f2_pack(s[e], s[e + 1]), scale2, negm2);
+          float x0, x1;
+          f2_unpack(x2, x0, x1);
+          const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+          acc2[c & 3] = f2_add(acc2[c & 3], f2_pack(p0, p1));
+          pk[c] = E::pack2(p0, p1);
         }
-      };
-      if (full) {
-        exp_store(std::true_type{});
-      } else {
-        exp_store(std::false_type{});
+        tmem_st32(tS + half * 32, pk);
       }
       float row_sum;
       {

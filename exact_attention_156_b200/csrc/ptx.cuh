@@ -651,38 +651,6 @@ __device__ __forceinline__ float max3f(float a, float b, float c) {
   return d;
 }
 
-// 2^x for a pair of floats on the FMA pipe (no MUFU), for x <= 127:
-// x is clamped to >= -126 (so the exponent field cannot underflow), split as x = n + f with n = round(x) (adding and
-// subtracting 1.5 * 2^23 rounds to the nearest integer) and f in [-1/2, 1/2];
-// 2^f comes from a degree-3 polynomial whose coefficients are the
-// relative-error minimax fit on [-1/2, 1/2] computed with the Remez exchange
-// algorithm (max relative error 7.5e-5); 2^n is applied by adding n to the
-// exponent field.  Used for a fixed share of the softmax exponentials so the
-// MUFU unit is not the bottleneck; the result is rounded to bf16 anyway.
-__device__ __forceinline__ uint64_t f2_exp2_poly(uint64_t x) {
-  float x0, x1;
-  f2_unpack(x, x0, x1);
-  const uint64_t xc = f2_pack(fmaxf(x0, -126.0f), fmaxf(x1, -126.0f));
-  const uint64_t magic = f2_pack(12582912.0f, 12582912.0f);
-  const uint64_t neg_magic = f2_pack(-12582912.0f, -12582912.0f);
-  const uint64_t minus_one = f2_pack(-1.0f, -1.0f);
-  const uint64_t j = f2_add(xc, magic);        // round(x) in the low mantissa bits
-  const uint64_t n = f2_add(j, neg_magic);     // round(x) as a float
-  const uint64_t f = f2_fma(n, minus_one, xc); // x - round(x)
-  uint64_t q = f2_fma(f2_pack(0.0551716685295105f, 0.0551716685295105f), f,
-                      f2_pack(0.2426111251115799f, 0.2426111251115799f));
-  q = f2_fma(q, f, f2_pack(0.6932609677314758f, 0.6932609677314758f));
-  q = f2_fma(q, f, f2_pack(0.9999280571937561f, 0.9999280571937561f));
-  float q0, q1, j0, j1;
-  f2_unpack(q, q0, q1);
-  f2_unpack(j, j0, j1);
-  // the integer n sits in the low bits of j; shifted into the exponent field
-  // the constant part of j vanishes (mod 2^32)
-  const float r0 = __int_as_float(__float_as_int(q0) + (__float_as_int(j0) << 23));
-  const float r1 = __int_as_float(__float_as_int(q1) + (__float_as_int(j1) << 23));
-  return f2_pack(r0, r1);
-}
-
 // ----------------------------------------------------------------------------
 // Arithmetic helpers
 // ----------------------------------------------------------------------------

@@ -69,31 +69,6 @@ def test_tcgen05_operand_forms(diag, mode):
     assert err < 1e-5, f"mode {mode}: relative error {err:.3e}"
 
 
-def test_polynomial_exp2_against_float64(diag):
-    """The FMA-pipe 2^x used for part of the softmax: relative error within the
-    minimax bound (7.5e-5, plus float32 rounding) on the range the softmax
-    feeds it, and a tiny non-negative value (not garbage) below -126."""
-    import torch
-    diag.attn_diag_exp2.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p]
-    x = np.concatenate([np.linspace(-126.0, 127.0, 2_000_000),
-                        np.random.default_rng(3).uniform(-30, 8, 1_000_000)]).astype(np.float32)
-    xd = torch.from_numpy(x).cuda()
-    yd = torch.empty_like(xd)
-    assert diag.attn_diag_exp2(xd.data_ptr(), yd.data_ptr(), x.size, None) == 0
-    assert diag.attn_diag_error() == 0
-    y = yd.cpu().numpy().astype(np.float64)
-    ref = np.exp2(x.astype(np.float64))
-    normal = x >= -125.0
-    rel = np.abs(y[normal] - ref[normal]) / ref[normal]
-    assert rel.max() < 8e-5, rel.max()
-    low = np.array([-126.5, -200.0, -1e30, -np.inf], dtype=np.float32)
-    ld = torch.from_numpy(low).cuda()
-    lo = torch.empty_like(ld)
-    assert diag.attn_diag_exp2(ld.data_ptr(), lo.data_ptr(), low.size, None) == 0
-    lo = lo.cpu().numpy()
-    assert np.all(lo >= 0) and np.all(lo < 2.0 ** -124)
-
-
 @pytest.mark.parametrize("mode", [8, 9, 10])
 def test_tcgen05_cta_pair_products(diag, mode):
     """One 256 x 128 x 128 product shared by a pair of CTAs (cta_group::2): each CTA
