@@ -43,12 +43,16 @@ GQA_WORKLOAD = dict(name="gqa_b1h32hk8s8192d128_fwdbwd", B=1, H=32, Hk=8, Sq=819
 # KV-cache decode: one new query row per sequence over a full 8192-row cache
 DECODE_WORKLOAD = dict(name="decode_b8h32hk8l8192d128", B=8, Sq=1, H=32, Hk=8, Smax=8192,
                        D=128, causal=0, input_scale=0.5, seed=1007)
-# the same step at head_dim 64, which runs the rows-on-lanes decode kernel
+# the same step at head_dim 64 (the keys-on-lanes kernel with half-width K/V tiles)
 DECODE64_WORKLOAD = dict(name="decode_b8h32hk8l8192d64", B=8, Sq=1, H=32, Hk=8, Smax=8192,
                          D=64, causal=0, input_scale=0.5, seed=1010)
 # packed variable-length batch: 32768 tokens in sequences of 128..4096 tokens
 VARLEN_WORKLOAD = dict(name="varlen_t32768h32d128_fwdbwd", total=32768, len_lo=128,
                        len_hi=4096, H=32, Hk=32, D=128, causal=1, input_scale=0.5, seed=1008)
+# padded batch: sequences of 128..4096 tokens (8192 in all) in (B, S, H, D) tensors with
+# per-sequence lengths, S = the longest sequence
+PADDED_WORKLOAD = dict(name="padded_t8192h32d128_fwdbwd", total=8192, len_lo=128,
+                       len_hi=4096, H=32, Hk=32, D=128, causal=1, input_scale=0.5, seed=1016)
 # head_dim 64 forward alone: B2 H32 S8192 causal (inputs 192 MiB, larger than L2)
 FWD64_WORKLOAD = dict(name="fwd_b2h32s8192d64_causal", B=2, H=32, Hk=32, Sq=8192, Sk=8192,
                       D=64, causal=1, win_left=-1, win_right=-1, input_scale=0.5, seed=1011)
@@ -79,7 +83,7 @@ ORACLE_FULL = [
 ]
 WORKLOADS = {"fwdbwd": WORKLOAD, "gqa": GQA_WORKLOAD, "decode": DECODE_WORKLOAD,
              "decode64": DECODE64_WORKLOAD,
-             "varlen": VARLEN_WORKLOAD, "padded": VARLEN_WORKLOAD,
+             "varlen": VARLEN_WORKLOAD, "padded": PADDED_WORKLOAD,
              "d256": D256_WORKLOAD, "d256fwd": D256_WORKLOAD,
              "fwd64": FWD64_WORKLOAD,
              "fwdsweep": None}
@@ -582,9 +586,9 @@ DECODE_KERNEL_SOURCES = ["decode_sm100.cuh", "ptx.cuh", "common.cuh"]
 
 
 def decode_kernel_name(w) -> str:
-    """The split kernel attn_decode runs for a workload: keys on the lanes for
-    head_dim 128 with at most 16 query rows per K/V head, else rows on the lanes."""
-    if w["D"] == 128 and (w["H"] // w["Hk"]) * w["Sq"] <= 16:
+    """The split kernel attn_decode runs for a workload: keys on the lanes with
+    at most 16 query rows per K/V head, else rows on the lanes."""
+    if (w["H"] // w["Hk"]) * w["Sq"] <= 16:
         return "attn_decode_t16_kernel"
     return "attn_decode_kernel"
 
@@ -766,14 +770,15 @@ def varlen_fwd_flops(w, lengths) -> float:
 def varlen_config(w, lengths, padded=False):
     if padded:
         B, S = len(lengths), max(lengths)
-        return {"workload": f"padded_b{B}s{S}h{w['H']}d{w['D']}_fwdbwd: fwd+bwd of a padded batch "
-                            f"(B={B}, S={S}, H={w['H']}, D={w['D']}) holding the {w['name']} "
-                            f"sequences ({min(lengths)}..{max(lengths)} tokens, lengths "
-                            f"log-uniform in [{w['len_lo']}, {w['len_hi']}]) with per-sequence "
-                            f"lengths, causal, inputs N(0,1)*{w['input_scale']}, padding rows zero",
+        gb = 4 * B * S * w["H"] * w["D"] * 2 / 1e9
+        return {"workload": f"{w['name']}: fwd+bwd of a padded batch (B={B}, S={S}, "
+                            f"H={w['H']}, D={w['D']}) of {w['total']} real tokens in sequences "
+                            f"of {min(lengths)}..{max(lengths)} (lengths log-uniform in "
+                            f"[{w['len_lo']}, {w['len_hi']}]) with per-sequence lengths, causal, "
+                            f"inputs N(0,1)*{w['input_scale']}, padding rows zero",
                 "B": B, "S": S, "real_tokens": w["total"], "H": w["H"], "D": w["D"],
                 "causal": bool(w["causal"]),
-                "l2": "no flush: inputs (Q,K,V,dO 3.9 GB) exceed the 126 MB L2"}
+                "l2": f"no flush: inputs (Q,K,V,dO {gb:.2f} GB) exceed the 126 MB L2"}
     return {"workload": f"{w['name']}: fwd+bwd of a packed batch, {len(lengths)} sequences of "
                         f"{min(lengths)}..{max(lengths)} tokens ({w['total']} in all, lengths "
                         f"log-uniform in [{w['len_lo']}, {w['len_hi']}]), H={w['H']} "
@@ -815,7 +820,7 @@ def run_varlen_reference(args):
     rank, _, _ = dist_env()
     if rank != 0:
         return 0
-    w = VARLEN_WORKLOAD
+    w = PADDED_WORKLOAD if args.workload == "padded" else VARLEN_WORKLOAD
     lengths = varlen_lengths(w)
     inputs = varlen_oracle_inputs(w)
     for i in range(args.warmup):
@@ -842,8 +847,8 @@ def run_varlen_reference(args):
 
 def run_varlen(args):
     """fwd + bwd of a packed variable-length batch (one step = both calls); with
-    --workload padded, the same sequences in (B, S, H, D) tensors through
-    attn_fwd_padded / attn_bwd_padded."""
+    --workload padded, a smaller batch of such sequences in (B, S, H, D) tensors
+    through attn_fwd_padded / attn_bwd_padded."""
     import numpy as np
     import torch
     rank, world, local = dist_env()
@@ -860,7 +865,7 @@ def run_varlen(args):
                                           attn_fwd_varlen, get_last_device_error)
     from synth import make_inputs
     padded = args.workload == "padded"
-    w = VARLEN_WORKLOAD
+    w = PADDED_WORKLOAD if padded else VARLEN_WORKLOAD
     lengths = varlen_lengths(w)
     T, H, D = w["total"], w["H"], w["D"]
     Bp, Lmax = len(lengths), max(lengths)
@@ -1249,8 +1254,9 @@ def main(argv=None):
                     help="fwdbwd: the headline fwd+bwd workload (default); gqa: the same sizes "
                          "with 8 K/V heads for 32 query heads; decode: KV-cache decode "
                          "(B8 H32 Hk8, 8192 cached rows, one new row); varlen: a packed batch "
-                         "of 32768 tokens in sequences of 128..4096; padded: the same sequences "
-                         "in (B, S, H, D) tensors with per-sequence lengths; d256: head_dim 256 forward + "
+                         "of 32768 tokens in sequences of 128..4096; padded: 8192 tokens in such "
+                         "sequences in (B, S, H, D) tensors with per-sequence lengths; d256: "
+                         "head_dim 256 forward + "
                          "backward, B1 H16 S8192 causal; d256fwd: its forward alone; fwd64: the "
                          "head_dim 64 forward alone, B2 H32 S8192 causal; decode64: the decode "
                          "step at head_dim 64; fwdsweep: the forward alone on C2-C4")
