@@ -23,16 +23,18 @@
 //       dK += dS^T Q  (A = dS^T from shared memory, K-major)
 //       dQ_tile = dS K (A = the same dS^T buffer read MN-major) -> fp32 TMA
 //       bulk reduce-add through a dedicated two-slot staging ring
-//     warps 0-3: P and dS (one thread = one key row); warps 4-7: drain dQ;
-//     warp 8: MMA issue; warp 9: Q loads; warp 10: dO loads.
+//     warps 0-7: P and dS in two groups of four (one thread = one key row and
+//     64 of the tile's 128 query columns; each group keeps its half of P beside
+//     its own scores and writes its half of dS^T); warps 8-11: drain dQ;
+//     warp 12: MMA issue; warp 13: Q loads; warp 14: dO loads.
 //     Q (with its row values) is double buffered, dO single buffered; the MMA
 //     order dV(t), S(t+1), dQ(t), dK(t), dP(t+1) lets the next tile's P run
 //     while the tensor core finishes this tile's gradients.
 //  3. bwd_dq_finalize: dQ = scale * accumulator, rounded to the input format.
 // Q, K, V, dO, P, dS and the gradients are bf16 or f16 (template parameter E);
 // all accumulation is f32.
-// Tensor memory (512 columns): dK [0,D) dV [D,2D) S^T/P^T [2D,2D+128)
-// dP^T / dQ [2D+128, 2D+256).
+// Tensor memory (512 columns): dK [0,D) dV [D,2D) S^T/P^T [2D,2D+128) (P^T as
+// 16-bit pairs in [2D,2D+32) and [2D+64,2D+96)), dP^T / dQ [2D+128, 2D+256).
 #pragma once
 
 #include <cuda.h>
@@ -46,19 +48,21 @@ namespace bwd {
 
 constexpr int BM = 128;  // query rows per tile
 constexpr int BN = 128;  // key rows per CTA
-constexpr int kThreads = 384;  // compute WG, dQ-drain WG, control WG {MMA, Q load, dO load, idle}
-constexpr int kDrainWarp0 = 4;
-constexpr int kMmaWarp = 8;
-constexpr int kLoadQWarp = 9;
-constexpr int kLoadDOWarp = 10;
+// two compute WGs (64 query columns each), dQ-drain WG, control WG {MMA, Q load, dO load, idle}
+constexpr int kThreads = 512;
+constexpr int kDrainWarp0 = 8;
+constexpr int kMmaWarp = 12;
+constexpr int kLoadQWarp = 13;
+constexpr int kLoadDOWarp = 14;
 constexpr int kQStages = 2;
-// Register split after launch (168 per thread at launch: 384 x 168 = 64512):
-// compute 128 x 256 + drain 128 x 152 + control 128 x 96 = 64512.
-constexpr int kLaunchRegs = 168;
-constexpr int kComputeRegs = 256;
-constexpr int kDrainRegs = 152;
-constexpr int kControlRegs = 96;
-static_assert(128 * (kComputeRegs + kDrainRegs + kControlRegs) <= kThreads * kLaunchRegs,
+constexpr int kComputeThreads = 256;
+// Register split after launch (128 per thread at launch: 512 x 128 = 65536):
+// compute 2 x 128 x 136 + drain 128 x 160 + control 128 x 64 = 63488.
+constexpr int kLaunchRegs = 128;
+constexpr int kComputeRegs = 136;
+constexpr int kDrainRegs = 160;
+constexpr int kControlRegs = 64;
+static_assert(128 * (2 * kComputeRegs + kDrainRegs + kControlRegs) <= kThreads * kLaunchRegs,
               "register split exceeds the launch allocation");
 
 template <int D>
@@ -463,7 +467,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::kNumBars; ++i) {
       uint32_t count = 1;
-      if (i == C::kBarP || i == C::kBarDS || i == C::kBarDQEmpty) count = 128;
+      if (i == C::kBarP || i == C::kBarDS) count = kComputeThreads;
+      if (i == C::kBarDQEmpty) count = 128;
       mbar_init(bar(i), count);
     }
     *abort_flag = 0;
@@ -524,38 +529,44 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp < kDrainWarp0) {
     regs_realloc<kLaunchRegs, kComputeRegs>();
     // ------------------------------------------------------------ P and dS
+    // Two groups of four warps: group grp owns query columns [64 grp, 64 grp + 64)
+    // of every key row (one thread = one key row per group).  Each group writes
+    // its half of P as 16-bit pairs into the first 32 of its own 64 score
+    // columns, and its half of dS^T into its own 64-column box.
+    const int grp = warp / 4;
     const int quad = warp % 4;
     const int r = quad * 32 + lane;  // key row within the tile
     const int kk_idx = n0 + r;       // key index
+    const int cb = 64 * grp;         // first query column of this group
     const uint32_t lane_off = uint32_t(quad * 32) << 16;
-    const uint32_t tS = tmem + lane_off + C::kColS;
-    const uint32_t tDP = tmem + lane_off + C::kColDP;
+    const uint32_t tS = tmem + lane_off + C::kColS + uint32_t(cb);
+    const uint32_t tDP = tmem + lane_off + C::kColDP + uint32_t(cb);
     const uint64_t sl2 = f2_pack(p.scale_log2, p.scale_log2);
     const int qmin_k = g.qmin(kk_idx);
     const int qmax_k = min(g.qmax(kk_idx), Lq - 1);
     const bool key_ok = kk_idx < Lk;
     // rows of the dS^T buffer: 128 bytes per 64 columns, 16-byte chunks swizzled by row % 8
-    const uint32_t ds_row = ds_addr + uint32_t(r) * 128;
+    const uint32_t ds_row = ds_addr + uint32_t(grp) * C::kBoxBytes + uint32_t(r) * 128;
     const uint32_t sw = uint32_t(r & 7);
     bool ok = true;
     for (int t = 0; t < nq; ++t) {
       const int s = t % kQStages;
       const int i0 = item_row0(t);
-      const float4* nl = reinterpret_cast<const float4*>(smem + C::kLseOff + s * BM * 4);
-      const float4* nd = reinterpret_cast<const float4*>(smem + C::kDeltaOff + s * BM * 4);
+      const float4* nl = reinterpret_cast<const float4*>(smem + C::kLseOff + s * BM * 4 + cb * 4);
+      const float4* nd = reinterpret_cast<const float4*>(smem + C::kDeltaOff + s * BM * 4 + cb * 4);
       // P = 2^(scale*log2e*S - LSE*log2e), kept as 16-bit pairs (what dV uses) for dS too
       if (!bw.wait_warp(bar(C::kBarS), t & 1, 27)) { ok = false; break; }
       tc_fence_after();
-      uint32_t pw[BM / 2];
+      uint32_t pw[32];
       {
-        uint32_t rr[BM];
-        tmem_ld128(tS, rr);
+        uint32_t rr[64];
+        tmem_ld64(tS, rr);
         const bool full = key_ok && n0 + BN - 1 <= Lk - 1 && i0 + BM - 1 <= Lq - 1 &&
                           i0 >= g.qmin(n0 + BN - 1) && i0 + BM - 1 <= g.qmax(n0);
         if (full) {
           // every entry visible: no mask
 #pragma unroll
-          for (int c = 0; c < BM; c += 4) {
+          for (int c = 0; c < 64; c += 4) {
             const float4 l4 = nl[c / 4];
             const uint64_t x0 = f2_fma(f2_pack(__uint_as_float(rr[c]), __uint_as_float(rr[c + 1])),
                                        sl2, f2_pack(l4.x, l4.y));
@@ -569,10 +580,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             pw[c / 2 + 1] = E::pack2(ex2_approx(a2), ex2_approx(a3));
           }
         } else {
-          const int c_lo = key_ok ? qmin_k - i0 : (1 << 30);
-          const int c_hi = qmax_k - i0;
+          const int c_lo = key_ok ? qmin_k - i0 - cb : (1 << 30);
+          const int c_hi = qmax_k - i0 - cb;
 #pragma unroll
-          for (int c = 0; c < BM; c += 4) {
+          for (int c = 0; c < 64; c += 4) {
             const float4 l4 = nl[c / 4];
             const uint64_t x0 = f2_fma(f2_pack(__uint_as_float(rr[c]), __uint_as_float(rr[c + 1])),
                                        sl2, f2_pack(l4.x, l4.y));
@@ -592,18 +603,18 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
-      tmem_st64(tS, pw);
+      tmem_st32(tS, pw);
       tc_fence_before();
       mbar_arrive(bar(C::kBarP));
 
       // dS = P * (dP - Delta) -> 16-bit, written swizzled for the dK and dQ products
       if (!bw.wait_warp(bar(C::kBarDP), t & 1, 28)) { ok = false; break; }
       tc_fence_after();
-      uint32_t rr[BM];
-      tmem_ld128(tDP, rr);
+      uint32_t rr[64];
+      tmem_ld64(tDP, rr);
       if (t > 0 && !bw.wait_warp(bar(C::kBarDSEmpty), (t - 1) & 1, 29)) { ok = false; break; }
 #pragma unroll
-      for (int c = 0; c < BM; c += 8) {
+      for (int c = 0; c < 64; c += 8) {
         const float4 d0 = nd[c / 4];
         const float4 d1 = nd[c / 4 + 1];
         const float dl[8] = {d0.x, d0.y, d0.z, d0.w, d1.x, d1.y, d1.z, d1.w};
@@ -620,44 +631,41 @@ __global__ void __launch_bounds__(kThreads, 1)
           f2_unpack(f2_mul(p2, gd), a0, a1);
           w[e] = E::pack2(a0, a1);
         }
-        const uint32_t box = uint32_t(c / 64);
-        const uint32_t chunk = uint32_t((c % 64) / 8);
-        st_shared_v4(ds_row + box * C::kBoxBytes + ((chunk ^ sw) << 4), w[0], w[1], w[2], w[3]);
+        const uint32_t chunk = uint32_t(c / 8);
+        st_shared_v4(ds_row + ((chunk ^ sw) << 4), w[0], w[1], w[2], w[3]);
       }
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(bar(C::kBarDS));
     }
-    // epilogue: dK = scale * acc, dV = acc (16-bit), once the last dK product is done
+    // epilogue: group 0 writes dK = scale * acc, group 1 dV = acc (16-bit), once the
+    // last dK product is done
     if (ok && nq > 0) ok = bw.wait_warp(bar(C::kBarDSEmpty), (nq - 1) & 1, 30);
     if (ok) {
       tc_fence_after();
       const size_t orow =
           ((kVarlen ? size_t(k_row0) + kk_idx : size_t(b) * p.Sk + size_t(kk_idx)) * p.Hk + hk) * D;
+      const uint32_t col = grp == 0 ? C::kColDK : C::kColDV;
+      const float mul = grp == 0 ? p.scale : 1.0f;
+      uint16_t* outp = grp == 0 ? p.dk : p.dv;
 #pragma unroll 1
-      for (int which = 0; which < 2; ++which) {
-        const uint32_t col = which == 0 ? C::kColDK : C::kColDV;
-        const float mul = which == 0 ? p.scale : 1.0f;
-        uint16_t* outp = which == 0 ? p.dk : p.dv;
-#pragma unroll 1
-        for (int c0 = 0; c0 < D; c0 += 32) {
-          uint32_t rr[32];
-          if (nq > 0) {
-            tmem_ld32(tmem + lane_off + col + c0, rr);
-          } else {
+      for (int c0 = 0; c0 < D; c0 += 32) {
+        uint32_t rr[32];
+        if (nq > 0) {
+          tmem_ld32(tmem + lane_off + col + c0, rr);
+        } else {
 #pragma unroll
-            for (int c = 0; c < 32; ++c) rr[c] = 0u;
-          }
-          uint32_t w[16];
+          for (int c = 0; c < 32; ++c) rr[c] = 0u;
+        }
+        uint32_t w[16];
 #pragma unroll
-          for (int c = 0; c < 16; ++c)
-            w[c] = E::pack2(__uint_as_float(rr[2 * c]) * mul, __uint_as_float(rr[2 * c + 1]) * mul);
-          if (key_ok) {
-            uint8_t* dst = reinterpret_cast<uint8_t*>(outp + orow + c0);
+        for (int c = 0; c < 16; ++c)
+          w[c] = E::pack2(__uint_as_float(rr[2 * c]) * mul, __uint_as_float(rr[2 * c + 1]) * mul);
+        if (key_ok) {
+          uint8_t* dst = reinterpret_cast<uint8_t*>(outp + orow + c0);
 #pragma unroll
-            for (int v = 0; v < 4; ++v)
-              st_global_v4(dst + 16 * v, w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
-          }
+          for (int v = 0; v < 4; ++v)
+            st_global_v4(dst + 16 * v, w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
         }
       }
     }
@@ -683,7 +691,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       uint32_t rr[D];
       if constexpr (D == 128) {
-        tmem_ld128(tDQ, rr);
+        uint32_t (&lo)[64] = *reinterpret_cast<uint32_t(*)[64]>(&rr[0]);
+        uint32_t (&hi)[64] = *reinterpret_cast<uint32_t(*)[64]>(&rr[64]);
+        tmem_ld64(tDQ, lo);
+        tmem_ld64(tDQ + 64, hi);
       } else {
         tmem_ld64(tDQ, rr);
       }
@@ -788,8 +799,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         // dV += P^T dO   (A = P^T in tensor memory, K = query index)
         if (!bw.wait(bar(C::kBarP), t & 1, 23)) { ok = false; break; }
         tc_fence_after();
-        mma_chain_ts_mn8(tmem + C::kColDV, tmem + C::kColS,
-                         sdesc_sw128(do_addr, C::kBoxBytes), id_dv, t > 0 ? 1u : 0u);
+        mma_chain_ts_mn8_split64(tmem + C::kColDV, tmem + C::kColS,
+                                 sdesc_sw128(do_addr, C::kBoxBytes), id_dv, t > 0 ? 1u : 0u);
         tc_commit(bar(C::kBarDOEmpty));
         // next S^T: overwrites P^T only after dV has read it (same issue order)
         if (more) {

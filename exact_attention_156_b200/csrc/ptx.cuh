@@ -424,6 +424,45 @@ __device__ __forceinline__ void mma_chain_ts_mn8(uint32_t d_tmem, uint32_t a_tme
       : "memory");
 }
 
+// As mma_chain_ts_mn8, with A's 16-bit pairs in two blocks of 32 columns 64
+// apart (K-steps 0-3 from columns [0,32), K-steps 4-7 from [64,96)): the layout
+// two thread groups leave when each writes its half of P beside its own scores.
+__device__ __forceinline__ void mma_chain_ts_mn8_split64(uint32_t d_tmem, uint32_t a_tmem,
+                                                         uint64_t b_desc, uint32_t idesc,
+                                                         uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .b32 blo, bhi, bl, at;\n\t.reg .b64 bd;\n\t.reg .pred pa, pt;\n\t"
+      "mov.b64 {blo, bhi}, %2;\n\t"
+      "setp.ne.b32 pa, %4, 0;\n\tsetp.eq.b32 pt, 0, 0;\n\t"
+      "add.u32 at, %1, 0;\n\tadd.u32 bl, blo, 0;\n\t"
+      "mov.b64 bd, {bl, bhi};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [at], bd, %3, pa;\n\t"
+      "add.u32 at, %1, 8;\n\tadd.u32 bl, blo, 128;\n\t"
+      "mov.b64 bd, {bl, bhi};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [at], bd, %3, pt;\n\t"
+      "add.u32 at, %1, 16;\n\tadd.u32 bl, blo, 256;\n\t"
+      "mov.b64 bd, {bl, bhi};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [at], bd, %3, pt;\n\t"
+      "add.u32 at, %1, 24;\n\tadd.u32 bl, blo, 384;\n\t"
+      "mov.b64 bd, {bl, bhi};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [at], bd, %3, pt;\n\t"
+      "add.u32 at, %1, 64;\n\tadd.u32 bl, blo, 512;\n\t"
+      "mov.b64 bd, {bl, bhi};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [at], bd, %3, pt;\n\t"
+      "add.u32 at, %1, 72;\n\tadd.u32 bl, blo, 640;\n\t"
+      "mov.b64 bd, {bl, bhi};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [at], bd, %3, pt;\n\t"
+      "add.u32 at, %1, 80;\n\tadd.u32 bl, blo, 768;\n\t"
+      "mov.b64 bd, {bl, bhi};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [at], bd, %3, pt;\n\t"
+      "add.u32 at, %1, 88;\n\tadd.u32 bl, blo, 896;\n\t"
+      "mov.b64 bd, {bl, bhi};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [at], bd, %3, pt;\n\t"
+      "}"
+      :: "r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // Instruction descriptor for kind::f16 with 16-bit A/B of format `fmt`
 // (0 = f16, 1 = bf16; A and B always the same) and f32 accumulate.
 __host__ __device__ constexpr uint32_t idesc_f32acc(int M, int N, bool a_mn_major,
