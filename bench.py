@@ -43,7 +43,8 @@ GQA_WORKLOAD = dict(name="gqa_b1h32hk8s8192d128_fwdbwd", B=1, H=32, Hk=8, Sq=819
 # KV-cache decode: one new query row per sequence over a full 8192-row cache
 DECODE_WORKLOAD = dict(name="decode_b8h32hk8l8192d128", B=8, Sq=1, H=32, Hk=8, Smax=8192,
                        D=128, causal=0, input_scale=0.5, seed=1007)
-# the same step at head_dim 64 (the keys-on-lanes kernel with half-width K/V tiles)
+# the same step at head_dim 64 (the keys-on-lanes kernel with half-width K/V tiles,
+# two CTAs per SM)
 DECODE64_WORKLOAD = dict(name="decode_b8h32hk8l8192d64", B=8, Sq=1, H=32, Hk=8, Smax=8192,
                          D=64, causal=0, input_scale=0.5, seed=1010)
 # packed variable-length batch: 32768 tokens in sequences of 128..4096 tokens

@@ -98,8 +98,8 @@ attn_status device_state(DeviceState** out) {
         ok = ok &&
              set_smem(dec::attn_decode_kernel<D, E>, dec::Cfg<D>::kSmemBytes) == cudaSuccess &&
              set_smem(fwd256::attn_fwd_d256_kernel<E>, fwd256::Cfg::kSmemBytes) == cudaSuccess;
-        ok = ok && set_smem(dec::t16::attn_decode_t16_kernel<D, E>, dec::t16::Cfg::kSmemBytes) ==
-                       cudaSuccess;
+        ok = ok && set_smem(dec::t16::attn_decode_t16_kernel<D, E>,
+                            dec::t16::Cfg<D>::kSmemBytes) == cudaSuccess;
       };
       ok = ok &&
            set_smem(bwd256::attn_bwd_d256_kernel<ElemBF16>, bwd256::Cfg::kSmemBytes) ==
@@ -723,7 +723,12 @@ attn_status launch_decode(const DeviceState& st, const void* q, const void* kc, 
   if (make_map(&mk, kc, B, Smax, Hk, D, dt) != ATTN_OK ||
       make_map(&mv, vc, B, Smax, Hk, D, dt) != ATTN_OK)
     return ATTN_ERR_LAUNCH;
-  const DecodePlan plan = decode_plan(B, Smax, Hk, st.num_sms > 0 ? st.num_sms : 148);
+  // keys on the tensor-memory lanes (at most 16 query rows per K/V head): at
+  // head_dim 64 two CTAs share an SM, so a wave holds twice the SM count
+  const bool keys_on_lanes = group * Sq <= dec::t16::kRows;
+  const int sms = st.num_sms > 0 ? st.num_sms : 148;
+  const DecodePlan plan =
+      decode_plan(B, Smax, Hk, keys_on_lanes ? sms * dec::t16::Cfg<D>::kCtasPerSm : sms);
   // partial results are laid out for the largest split count (the workspace size)
   const size_t rows = size_t(B) * H * Sq * decode_max_splits(Smax);
   dec::Params p;
@@ -744,10 +749,10 @@ attn_status launch_decode(const DeviceState& st, const void* q, const void* kc, 
   p.timeout_ns = kTimeoutNs;
   // at most 16 query rows per K/V head (one new token, up to 16 query heads
   // each): keys on the tensor-memory lanes; otherwise query rows on the lanes
-  if (group * Sq <= dec::t16::kRows) {
+  if (keys_on_lanes) {
     dec::t16::attn_decode_t16_kernel<D, E><<<dim3(plan.nsplit, Hk, B), dec::t16::kThreads,
-                                               dec::t16::Cfg::kSmemBytes, stream>>>(mq, mk, mv,
-                                                                                    p);
+                                               dec::t16::Cfg<D>::kSmemBytes, stream>>>(mq, mk, mv,
+                                                                                       p);
   } else {
     dec::attn_decode_kernel<D, E><<<dim3(plan.nsplit, Hk, B), dec::kThreads,
                                     dec::Cfg<D>::kSmemBytes, stream>>>(mq, mk, mv, p);

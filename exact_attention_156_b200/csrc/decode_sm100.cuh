@@ -399,25 +399,31 @@ __global__ void __launch_bounds__(kThreads, 1)
 //   O^T += V^T P^T   (M = 128 = head_dim, N = 16 rows; A = V tile read MN-major,
 //                     B = P^T from shared memory, K-major over the keys)
 // so each softmax thread owns one key and 16 scores.  At head_dim 64 the same
-// kernel runs with M = 128 for O^T: the K/V slots keep two 64-column boxes, only
-// the first is loaded, and the second is cleared once, so rows 64..127 of O^T
-// stay zero and are never written out.  The row maximum is a
+// kernel runs with M = 128 for O^T: the second 64-row block of its A operand
+// (V^T) is a box cleared once per CTA, so rows 64..127 of O^T stay zero and are
+// never written out; the smaller slots let two CTAs share an SM.  The row maximum is a
 // reduction over the 128 threads (shuffles within a warp, then shared memory
 // across the four warps); row sums stay per thread until the end.  P^T is
 // written as 16-bit values into a double-buffered 4 KB shared tile.
 namespace t16 {
 constexpr int kRows = 16;       // N of both products
 constexpr int kThreads = 224;   // warps 0-3 softmax, 4 MMA, 5 Q/K loads, 6 V loads
+// D: head_dim.  At D = 64 the K and V slots hold one 64-column box, the
+// rings have two slots, and one cleared box after the V ring stands in for
+// rows 64..127 of the M = 128 product O^T (its descriptor's M stride points
+// there): about 93 KB of shared memory, so two CTAs share an SM.
+template <int D>
 struct Cfg {
   static constexpr int kBoxBytes = BN * 128;         // K/V box: 128 rows x 64 columns
-  static constexpr int kTileBytes = 2 * kBoxBytes;    // K or V slot (2 boxes, head_dim <= 128)
+  static constexpr int kTileBytes = (D / 64) * kBoxBytes;  // K or V slot
   static constexpr int kSmallBox = kRows * 128;       // Q / P^T box: 16 rows x 64 columns
-  static constexpr int kSlots = 3;
+  static constexpr int kSlots = D == 128 ? 3 : 2;
   static constexpr int kQOff = 0;                                  // 2 small boxes
   static constexpr int kPOff = 2 * kSmallBox;                      // 2 buffers x 2 small boxes
   static constexpr int kKOff = kPOff + 4 * kSmallBox;              // K ring (1024-aligned)
   static constexpr int kVOff = kKOff + kSlots * kTileBytes;        // V ring
-  static constexpr int kRedOff = kVOff + kSlots * kTileBytes;      // [2][4 warps][16] floats
+  static constexpr int kZeroOff = kVOff + kSlots * kTileBytes;     // D = 64: one cleared box
+  static constexpr int kRedOff = kZeroOff + (D == 64 ? kBoxBytes : 0);  // [2][4 warps][16] floats
   static constexpr int kBarOff = kRedOff + 2 * 4 * kRows * 4;
   static constexpr int kBarQ = 0;
   static constexpr int kBarKFull = 1;
@@ -433,10 +439,14 @@ struct Cfg {
   static constexpr int kNumBars = kBarDone + 1;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kSmemBytes = kMiscOff + 16;
+  static constexpr int kCtasPerSm = D == 128 ? 1 : 2;
   static constexpr uint32_t kColO = 2 * kRows;        // S^T buffers at 0 and 16, O^T at 32
   static constexpr int kTmemCols = 64;
-  static_assert(kKOff % 1024 == 0 && kVOff % 1024 == 0, "swizzled tiles need 1024-byte alignment");
+  static_assert(kKOff % 1024 == 0 && kVOff % 1024 == 0 && kZeroOff % 1024 == 0,
+                "swizzled tiles need 1024-byte alignment");
   static_assert(kSmemBytes <= 232448, "shared memory exceeds the 227 KB per block of sm_100");
+  static_assert(kCtasPerSm == 1 || kSmemBytes + 1024 <= 233472 / 2,
+                "two CTAs per SM must fit the SM's shared memory");
 };
 
 // Butterfly reduction of 16 per-lane values over the 32 lanes of a warp: 16
@@ -458,12 +468,12 @@ __device__ __forceinline__ float warp_reduce16(float (&v)[kRows], Op op) {
 
 // D: head_dim, 64 or 128.
 template <int D, class E>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, Cfg<D>::kCtasPerSm)
     attn_decode_t16_kernel(const __grid_constant__ CUtensorMap tmQ,
                            const __grid_constant__ CUtensorMap tmK,
                            const __grid_constant__ CUtensorMap tmV, const Params p) {
   static_assert(D == 64 || D == 128, "head_dim 64 or 128");
-  using C = Cfg;
+  using C = Cfg<D>;
   constexpr int kBoxes = D / 64;                 // 64-column boxes loaded per K/V tile
   constexpr int kLoadBytes = BN * D * 2;         // bytes landing per K/V tile
   extern __shared__ __align__(1024) uint8_t smem[];
@@ -500,12 +510,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   for (int e = threadIdx.x; e < 2 * C::kSmallBox / 16; e += kThreads)
     reinterpret_cast<uint4*>(smem + C::kQOff)[e] = make_uint4(0u, 0u, 0u, 0u);
   if constexpr (D == 64) {
-    // second box of every V slot: rows 64..127 of the M = 128 product O^T
-    for (int e = threadIdx.x; e < C::kSlots * C::kBoxBytes / 16; e += kThreads) {
-      const int sl = e / (C::kBoxBytes / 16), off = e % (C::kBoxBytes / 16);
-      reinterpret_cast<uint4*>(smem + C::kVOff + sl * C::kTileBytes + C::kBoxBytes)[off] =
-          make_uint4(0u, 0u, 0u, 0u);
-    }
+    // the cleared box: rows 64..127 of the M = 128 product O^T
+    for (int e = threadIdx.x; e < C::kBoxBytes / 16; e += kThreads)
+      reinterpret_cast<uint4*>(smem + C::kZeroOff)[e] = make_uint4(0u, 0u, 0u, 0u);
   }
   fence_proxy_async_smem();
   if (warp == 0) {
@@ -777,7 +784,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!bw.wait(bar(C::kBarP), t & 1, 69)) break;
         if (!bw.wait(bar(C::kBarVFull + s), (t / C::kSlots) & 1, 70)) break;
         tc_fence_after();
-        mma_chain_mnk8_b16(tmem + C::kColO, sdesc_sw128(v_addr(s), C::kBoxBytes),
+        // A = V^T: at D = 64 its second 64-row block is the cleared box
+        const uint32_t m_stride = D == 128 ? uint32_t(C::kBoxBytes)
+                                           : sbase + C::kZeroOff - v_addr(s);
+        mma_chain_mnk8_b16(tmem + C::kColO, sdesc_sw128(v_addr(s), m_stride),
                            sdesc_sw128(p_addr(t & 1), 16), idesc_o, t > 0 ? 1u : 0u);
         tc_commit(bar(C::kBarO));
         tc_commit(bar(C::kBarVEmpty + s));

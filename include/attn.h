@@ -353,8 +353,10 @@ ATTN_API attn_status attn_bwd_varlen(const void* q, const void* k, const void* v
  * only, no device call): the cache's 128-key tiles are cut into *nsplit splits
  * of *tiles_per_split tiles, one CTA per (split, K/V head, sequence), chosen to
  * minimise ceil(CTAs / num_sms) x (tiles_per_split + 3) with at least two tiles
- * per split when the cache has more than one tile.  attn_decode passes the
- * current device's SM count.  Errors: ATTN_ERR_NULLPTR, ATTN_ERR_SHAPE (an
+ * per split when the cache has more than one tile.  num_sms is the number of
+ * CTAs one wave holds: attn_decode passes the current device's SM count, twice
+ * that at head_dim 64 with at most 16 query rows per K/V head (two CTAs of
+ * that kernel share an SM).  Errors: ATTN_ERR_NULLPTR, ATTN_ERR_SHAPE (an
  * argument < 1).
  */
 ATTN_API attn_status attn_decode_split_plan(int B, int Smax, int Hk, int num_sms, int* nsplit,

@@ -63,6 +63,7 @@ def _one_call(case, seed):
 PAIRS = [
     ((1, 1000, 1000, 4, 128, 1, -1, -1), (1, 900, 1000, 3, 128, 1, -1, -1)),
     ((2, 300, 457, 3, 64, 0, 50, 20), (1, 260, 300, 2, 64, 0, -1, 7)),
+    ((1, 300, 300, 2, 256, 1, -1, -1), (1, 257, 300, 1, 256, 1, 60, 0)),
 ]
 
 
