@@ -309,8 +309,11 @@ def cpu_baseline(w, budget_s: float = 15.0):
         tot_s += dt
         tot_f += fl
         n += 1
-    return {"value": tot_f / tot_s / 1e12, "unit": UNIT, "cores": blas_threads(),
+    value = tot_f / tot_s / 1e12
+    return {"value": value, "unit": UNIT, "cores": blas_threads(),
             "kind": "oracle",
+            # the whole workload at the sampled rate (extrapolated per visible pair)
+            "extrapolated_full_step_s": step_flops(w) / (value * 1e12),
             "sample": f"{n} samples x {ORACLE_ROWS_PER_SAMPLE} seeded query rows of one head of "
                       f"{w['name']} (fwd O/LSE, bwd dQ rows and their dK/dV share), float64 numpy, "
                       f"{tot_s:.1f} s total; flops counted as 14*D per visible pair"}
@@ -325,12 +328,28 @@ def oracle_full_forward():
     for w in ORACLE_FULL:
         bits = make_inputs(w["B"], w["Sq"], w["Sk"], w["H"], w["D"], w["seed"], w["input_scale"])
         x = {n: bits_to_f32(bits[n]) for n in ("q", "k", "v")}
-        t0 = time.perf_counter()
-        oracle.attention_forward(x["q"], x["k"], x["v"], 1.0 / math.sqrt(w["D"]), w["causal"])
-        dt = time.perf_counter() - t0
+
+        def timed():
+            t0 = time.perf_counter()
+            oracle.attention_forward(x["q"], x["k"], x["v"], 1.0 / math.sqrt(w["D"]),
+                                     w["causal"])
+            return time.perf_counter() - t0
+
+        dt = timed()
         out.append({"workload": w["name"], "seconds": dt,
                     "tflops": fwd_flops(w) / dt / 1e12, "cores": blas_threads(),
                     "sample": "whole configuration, forward, float64 numpy"})
+        if w["Sq"] * w["Sk"] * w["B"] * w["H"] <= 1 << 20:
+            # the smallest configuration also on one host core
+            try:
+                from threadpoolctl import threadpool_limits
+                with threadpool_limits(limits=1):
+                    dt1 = timed()
+                out.append({"workload": w["name"], "seconds": dt1,
+                            "tflops": fwd_flops(w) / dt1 / 1e12, "cores": 1,
+                            "sample": "whole configuration, forward, float64 numpy, one thread"})
+            except ImportError:
+                pass
     return out
 
 
