@@ -47,6 +47,10 @@ DECODE_WORKLOAD = dict(name="decode_b8h32hk8l8192d128", B=8, Sq=1, H=32, Hk=8, S
 # two CTAs per SM)
 DECODE64_WORKLOAD = dict(name="decode_b8h32hk8l8192d64", B=8, Sq=1, H=32, Hk=8, Smax=8192,
                          D=64, causal=0, input_scale=0.5, seed=1010)
+# four new rows per sequence (speculative steps) on one shared K/V head: 128 query rows per
+# K/V head, so the rows-on-lanes decode kernel runs; a 32768-row cache (134 MB) exceeds L2
+DECODE_ROWS_WORKLOAD = dict(name="decode_b8q4h32hk1l32768d128", B=8, Sq=4, H=32, Hk=1,
+                            Smax=32768, D=128, causal=1, input_scale=0.5, seed=1017)
 # packed variable-length batch: 32768 tokens in sequences of 128..4096 tokens
 VARLEN_WORKLOAD = dict(name="varlen_t32768h32d128_fwdbwd", total=32768, len_lo=128,
                        len_hi=4096, H=32, Hk=32, D=128, causal=1, input_scale=0.5, seed=1008)
@@ -83,7 +87,7 @@ ORACLE_FULL = [
          win_left=-1, win_right=-1, input_scale=1.0, seed=1002),
 ]
 WORKLOADS = {"fwdbwd": WORKLOAD, "gqa": GQA_WORKLOAD, "decode": DECODE_WORKLOAD,
-             "decode64": DECODE64_WORKLOAD,
+             "decode64": DECODE64_WORKLOAD, "decoderows": DECODE_ROWS_WORKLOAD,
              "varlen": VARLEN_WORKLOAD, "padded": PADDED_WORKLOAD,
              "d256": D256_WORKLOAD, "d256fwd": D256_WORKLOAD,
              "fwd64": FWD64_WORKLOAD,
@@ -1279,7 +1283,9 @@ def main(argv=None):
                          "head_dim 256 forward + "
                          "backward, B1 H16 S8192 causal; d256fwd: its forward alone; fwd64: the "
                          "head_dim 64 forward alone, B2 H32 S8192 causal; decode64: the decode "
-                         "step at head_dim 64; fwdsweep: the forward alone on C2-C4")
+                         "step at head_dim 64; decoderows: four new rows per sequence on one "
+                         "K/V head (rows-on-lanes decode kernel); fwdsweep: the forward alone "
+                         "on C2-C4")
     ap.add_argument("--no-cpu-baseline", action="store_true",
                     help="skip the timed oracle sample (it adds ~15 s of CPU time)")
     ap.add_argument("--no-c3", action="store_true",
@@ -1289,7 +1295,7 @@ def main(argv=None):
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
-    if args.workload in ("decode", "decode64"):
+    if args.workload in ("decode", "decode64", "decoderows"):
         return run_decode_reference(args) if args.impl == "reference" else run_decode(args)
     if args.workload in ("varlen", "padded"):
         return run_varlen_reference(args) if args.impl == "reference" else run_varlen(args)

@@ -50,12 +50,13 @@ def test_decode_against_the_oracle(case):
     check_fwd(to_f64(o), lse.cpu().numpy().astype(np.float64), o_ref, lse_ref, str(case))
 
 
-@pytest.mark.parametrize("name", ["DECODE_WORKLOAD", "DECODE64_WORKLOAD"])
+@pytest.mark.parametrize("name", ["DECODE_WORKLOAD", "DECODE64_WORKLOAD", "DECODE_ROWS_WORKLOAD"])
 def test_decode_bench_workload_in_full(name):
     """The benchmark's decode workloads themselves (B8, one new row, H32 Hk8,
-    8192 cached rows, D128 or D64, inputs N(0,1)*0.5, the seeds bench.py uses),
-    every output row against the oracle, through the same call the benchmark
-    times."""
+    8192 cached rows, D128 or D64; and four causal new rows of 32 query heads on
+    one K/V head over 32768 cached rows; inputs N(0,1)*0.5, the seeds bench.py
+    uses), every output row against the oracle, through the same call the
+    benchmark times."""
     import torch
     import bench
     from exact_attention_156_b200 import (attn_decode, attn_decode_workspace_size,
