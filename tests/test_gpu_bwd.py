@@ -34,6 +34,7 @@ BWD_CASES = [
     (1, 300, 300, 3, 64, 0, 40, 25),      # two-sided window, D = 64
     (1, 128, 128, 1, 128, 0, 0, 0),       # diagonal only
     (1, 1, 1, 1, 64, 0, -1, -1),
+    (48, 70, 90, 2, 128, 1, -1, -1),      # many short problems (tile-major block order)
 ]
 
 

@@ -66,9 +66,10 @@ EDGE = [
     (1, 260, 260, 2, 128, 0, 0, 0),       # diagonal window: O = V
     (1, 1000, 1000, 4, 64, 1, -1, -1),    # D = 64, several tiles
     (1, 640, 640, 2, 128, 1, 130, 0),     # window crossing tile edges
-    (2, 1100, 1100, 20, 128, 1, -1, -1),  # 200 work tiles > 148 SMs (persistent loop)
+    (2, 1100, 1100, 20, 128, 1, -1, -1),  # more CTAs than SMs
     (2, 700, 900, 40, 64, 0, 200, 100),   # 240 work tiles, window, Sq != Sk
     (3, 96, 96, 5, 128, 1, -1, -1),       # Sq smaller than one tile
+    (300, 40, 40, 1, 64, 0, -1, -1),      # many tiny problems (pair-major block order)
 ]
 
 

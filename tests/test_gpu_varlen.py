@@ -19,6 +19,8 @@ CASES = [
     ((200, 0, 513, 64), (300, 100, 513, 1), 8, 2, 64, 1, None, "bf16"),
     ((129, 77, 640), (129, 0, 700), 2, 2, 128, 0, (32, 16), "f16"),
     ("many", None, 4, 1, 128, 1, None, "bf16"),
+    # more sequences than a compact grid takes: the grid of the longest sequence's tiles
+    ("many300", None, 2, 2, 64, 1, None, "bf16"),
 ]
 
 
@@ -27,6 +29,9 @@ def _lengths(case):
     if lq == "many":  # 40 short sequences, a packed fine-tuning batch
         rng = np.random.default_rng(77)
         lq = tuple(int(x) for x in rng.integers(1, 300, size=40))
+    elif lq == "many300":  # 300 sequences: above the 256 that get compact grids
+        rng = np.random.default_rng(78)
+        lq = tuple(int(x) for x in rng.integers(0, 200, size=300))
     return lq, (lq if lk is None else lk)
 
 
