@@ -175,6 +175,59 @@ def aggregate_value(per_rank_flops: float, n_ranks: int, max_ms: float) -> float
     return per_rank_flops * n_ranks / (max_ms * 1e-3) / 1e12
 
 
+def pipelined_e2e(device, stream, host_in, dev_sets, out_names, run, n_steps):
+    """End-to-end milliseconds per step through the public API, fed the way a
+    training or serving loop feeds a GPU: step i's inputs are copied from pinned
+    host memory on one copy stream while step i-1 computes on `stream` and step
+    i-2's results are copied back to pinned host memory on a second copy stream.
+    Device inputs and outputs are double-buffered (`dev_sets`, two dicts of
+    tensors); every step's host->device and device->host copies lie inside the
+    timed region, which ends when the last results are in host memory.
+    run(d) launches one step on `stream` reading and writing the tensors of d."""
+    import torch
+    s_in, s_out = torch.cuda.Stream(device), torch.cuda.Stream(device)
+    out_host = [{n: torch.empty(d[n].shape, dtype=d[n].dtype).pin_memory() for n in out_names}
+                for d in dev_sets]
+    ev = lambda: torch.cuda.Event()
+    ev_in, ev_comp, ev_out = [ev(), ev()], [ev(), ev()], [ev(), ev()]
+
+    def one(i):
+        slot = i & 1
+        d = dev_sets[slot]
+        s_in.wait_stream(stream) if i == 0 else None
+        if i >= 2:
+            s_in.wait_event(ev_comp[slot])  # step i-2 has finished reading these inputs
+        with torch.cuda.stream(s_in):
+            for n, t in host_in.items():
+                d[n].copy_(t, non_blocking=True)
+        ev_in[slot].record(s_in)
+        stream.wait_event(ev_in[slot])
+        if i >= 2:
+            stream.wait_event(ev_out[slot])  # step i-2's results have left these outputs
+        run(d)
+        ev_comp[slot].record(stream)
+        s_out.wait_event(ev_comp[slot])
+        with torch.cuda.stream(s_out):
+            for n in out_names:
+                out_host[slot][n].copy_(d[n], non_blocking=True)
+        ev_out[slot].record(s_out)
+
+    for i in range(2):  # warm-up of the copy streams and both buffer sets
+        one(i)
+    torch.cuda.synchronize(device)
+    barrier(device)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    s_in.wait_event(e0)
+    for i in range(n_steps):
+        one(i)
+    stream.wait_stream(s_out)
+    e1.record(stream)
+    torch.cuda.synchronize(device)
+    barrier(device)
+    return reduce_max(e0.elapsed_time(e1), device) / n_steps
+
+
 # ---------------------------------------------------------------------------
 # peaks, clocks, committed ncu traffic
 # ---------------------------------------------------------------------------
@@ -473,14 +526,16 @@ def run_gpu(args):
     stream = torch.cuda.current_stream(device)
 
     names = ["fwd", "bwd_preprocess", "bwd_main", "bwd_dq_finalize"]
+    set0 = {"q": q, "k": k, "v": v, "do": do, "o": o, "lse": lse, "dq": dq, "dk": dk, "dv": dv}
 
-    def step(evs=None):
+    def step(evs=None, d=set0):
         if evs is not None:
             evs[0].record(stream)
-        attn_fwd(q, k, v, causal=causal, window_size=win, out=o, lse=lse, stream=stream)
+        attn_fwd(d["q"], d["k"], d["v"], causal=causal, window_size=win, out=d["o"],
+                 lse=d["lse"], stream=stream)
         rec = (lambda i: evs[i + 1].record(stream)) if evs is not None else None
-        attn_bwd_stages(q, k, v, o, do, lse, dq, dk, dv, ws, causal=causal, window_size=win,
-                        stream=stream, between=rec)
+        attn_bwd_stages(d["q"], d["k"], d["v"], d["o"], d["do"], d["lse"], d["dq"], d["dk"],
+                        d["dv"], ws, causal=causal, window_size=win, stream=stream, between=rec)
 
     for _ in range(args.warmup):
         step()
@@ -512,37 +567,27 @@ def run_gpu(args):
     ms_per_step = max_ms / args.steps
     value = aggregate_value(step_flops(w), world, ms_per_step)
 
-    # end to end through the public API with host buffers: H2D of the step's
-    # inputs from pinned memory, the step, D2H of its results (O, LSE, dQ, dK, dV)
-    out_host = {n: torch.empty(t.shape, dtype=t.dtype).pin_memory()
-                for n, t in (("o", o), ("lse", lse), ("dq", dq), ("dk", dk), ("dv", dv))}
+    # end to end through the public API with host buffers: every step copies its
+    # inputs (Q, K, V, dO) from pinned memory and its results (O, LSE, dQ, dK, dV)
+    # back, pipelined across steps on two copy streams (pipelined_e2e)
+    out_names = ("o", "lse", "dq", "dk", "dv")
     e2e_steps = max(3, min(args.steps, 10))
     h2d = sum(t.numel() * t.element_size() for t in host.values())
-    d2h = sum(t.numel() * t.element_size() for t in out_host.values())
-
-    def e2e_step():
-        for n in ("q", "k", "v", "do"):
-            dev[n].copy_(host[n], non_blocking=True)
-        step()
-        for n, t in (("o", o), ("lse", lse), ("dq", dq), ("dk", dk), ("dv", dv)):
-            out_host[n].copy_(t, non_blocking=True)
+    d2h = sum(set0[n].numel() * set0[n].element_size() for n in out_names)
 
     e2e = None
     if not args.no_e2e:
-        e2e_step()
-        torch.cuda.synchronize(device)
-        barrier(device)
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(e2e_steps):
-            e2e_step()
-        e1.record(stream)
-        torch.cuda.synchronize(device)
-        barrier(device)
-        e2e_ms = reduce_max(e0.elapsed_time(e1), device) / e2e_steps
+        set1 = {n: torch.empty_like(t) for n, t in set0.items()}
+        e2e_ms = pipelined_e2e(device, stream, host, [set0, set1], out_names,
+                               lambda d: step(None, d), e2e_steps)
+        if get_last_device_error() != 0:
+            raise RuntimeError("device-side timeout during the end-to-end leg")
         e2e = {"value": aggregate_value(step_flops(w), world, e2e_ms), "unit": UNIT,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
-               "steps": e2e_steps}
+               "steps": e2e_steps,
+               "pipelining": "inputs of step i copied in while step i-1 computes and step "
+                             "i-2's results are copied out (two copy streams, double-buffered "
+                             "device tensors); every step's copies inside the timed region"}
 
     c3 = None
     if args.workload == "fwdbwd" and args.dtype == "bf16" and not args.no_c3:
@@ -926,24 +971,28 @@ def run_varlen(args):
                          device=device)
     stream = torch.cuda.current_stream(device)
     causal = bool(w["causal"])
+    set0 = {"q": q, "k": k, "v": v, "do": do, "cu": cu, "o": o, "lse": lse, "dq": dq,
+            "dk": dk, "dv": dv}
 
-    def step(evs=None):
+    def step(evs=None, d=set0):
         if evs is not None:
             evs[0].record(stream)
         if padded:
-            attn_fwd_padded(q, k, v, cu, cu, causal=causal, out=o, lse=lse, workspace=ws_f,
-                            stream=stream)
+            attn_fwd_padded(d["q"], d["k"], d["v"], d["cu"], d["cu"], causal=causal, out=d["o"],
+                            lse=d["lse"], workspace=ws_f, stream=stream)
         else:
-            attn_fwd_varlen(q, k, v, cu, cu, Lmax, Lmax, causal=causal, out=o, lse=lse,
-                            stream=stream)
+            attn_fwd_varlen(d["q"], d["k"], d["v"], d["cu"], d["cu"], Lmax, Lmax, causal=causal,
+                            out=d["o"], lse=d["lse"], stream=stream)
         if evs is not None:
             evs[1].record(stream)
         if padded:
-            attn_bwd_padded(q, k, v, o, do, lse, cu, cu, causal=causal, dq=dq, dk=dk, dv=dv,
-                            workspace=ws, stream=stream)
+            attn_bwd_padded(d["q"], d["k"], d["v"], d["o"], d["do"], d["lse"], d["cu"], d["cu"],
+                            causal=causal, dq=d["dq"], dk=d["dk"], dv=d["dv"], workspace=ws,
+                            stream=stream)
         else:
-            attn_bwd_varlen(q, k, v, o, do, lse, cu, cu, Lmax, Lmax, causal=causal, dq=dq,
-                            dk=dk, dv=dv, workspace=ws, stream=stream)
+            attn_bwd_varlen(d["q"], d["k"], d["v"], d["o"], d["do"], d["lse"], d["cu"], d["cu"],
+                            Lmax, Lmax, causal=causal, dq=d["dq"], dk=d["dk"], dv=d["dv"],
+                            workspace=ws, stream=stream)
         if evs is not None:
             evs[2].record(stream)
 
@@ -970,33 +1019,23 @@ def run_varlen(args):
     ms = reduce_max(start.elapsed_time(end), device) / args.steps
     ff = varlen_fwd_flops(w, lengths)
     value = world * 3.5 * ff / (ms * 1e-3) / 1e12
-    out_host = {n: torch.empty(t.shape, dtype=t.dtype).pin_memory()
-                for n, t in (("o", o), ("lse", lse), ("dq", dq), ("dk", dk), ("dv", dv))}
+    out_names = ("o", "lse", "dq", "dk", "dv")
     e2e = None
     if not args.no_e2e:
-        def e2e_step():
-            for n in ("q", "k", "v", "do", "cu"):
-                dev[n].copy_(host[n], non_blocking=True)
-            step()
-            for n, t in (("o", o), ("lse", lse), ("dq", dq), ("dk", dk), ("dv", dv)):
-                out_host[n].copy_(t, non_blocking=True)
-        e2e_step()
-        torch.cuda.synchronize(device)
-        barrier(device)
         n_e2e = max(3, min(args.steps, 10))
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(n_e2e):
-            e2e_step()
-        e1.record(stream)
-        torch.cuda.synchronize(device)
-        barrier(device)
-        e2e_ms = reduce_max(e0.elapsed_time(e1), device) / n_e2e
+        set1 = {n: torch.empty_like(t) for n, t in set0.items()}
+        e2e_ms = pipelined_e2e(device, stream, host, [set0, set1], out_names,
+                               lambda d: step(None, d), n_e2e)
+        if get_last_device_error() != 0:
+            raise RuntimeError("device-side error during the end-to-end leg")
         e2e = {"value": world * 3.5 * ff / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
                "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in host.values()),
-               "d2h_bytes_per_step": sum(t.numel() * t.element_size()
-                                         for t in out_host.values()),
-               "ms_per_step": e2e_ms, "steps": n_e2e}
+               "d2h_bytes_per_step": sum(set0[n].numel() * set0[n].element_size()
+                                         for n in out_names),
+               "ms_per_step": e2e_ms, "steps": n_e2e,
+               "pipelining": "inputs of step i copied in while step i-1 computes and step "
+                             "i-2's results are copied out (two copy streams, double-buffered "
+                             "device tensors); every step's copies inside the timed region"}
     peaks = load_peaks()
     peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
     bwd_tf = 2.5 * ff / (bwd_ms * 1e-3) / 1e12
@@ -1093,27 +1132,21 @@ def run_fwd_only(args):
     tf = ff / (ms * 1e-3) / 1e12
     e2e = None
     if not args.no_e2e:
-        o_host = torch.empty(o.shape, dtype=o.dtype).pin_memory()
-        l_host = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
         n_e2e = max(3, min(args.steps, 10))
-        torch.cuda.synchronize(device)
-        barrier(device)
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(n_e2e):
-            for n in ("q", "k", "v"):
-                dev[n].copy_(host[n], non_blocking=True)
-            step()
-            o_host.copy_(o, non_blocking=True)
-            l_host.copy_(lse, non_blocking=True)
-        e1.record(stream)
-        torch.cuda.synchronize(device)
-        barrier(device)
-        e2e_ms = reduce_max(e0.elapsed_time(e1), device) / n_e2e
+        set0 = {"q": q, "k": k, "v": v, "o": o, "lse": lse}
+        set1 = {n: torch.empty_like(t) for n, t in set0.items()}
+        run = lambda d: attn_fwd(d["q"], d["k"], d["v"], causal=causal, out=d["o"],
+                                 lse=d["lse"], stream=stream)
+        e2e_ms = pipelined_e2e(device, stream, host, [set0, set1], ("o", "lse"), run, n_e2e)
+        if get_last_device_error() != 0:
+            raise RuntimeError("device-side timeout during the end-to-end leg")
         e2e = {"value": world * ff / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
                "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in host.values()),
-               "d2h_bytes_per_step": o_host.numel() * o_host.element_size()
-               + l_host.numel() * l_host.element_size(), "ms_per_step": e2e_ms, "steps": n_e2e}
+               "d2h_bytes_per_step": o.numel() * o.element_size() + lse.numel() * lse.element_size(),
+               "ms_per_step": e2e_ms, "steps": n_e2e,
+               "pipelining": "inputs of step i copied in while step i-1 computes and step "
+                             "i-2's results are copied out (two copy streams, double-buffered "
+                             "device tensors); every step's copies inside the timed region"}
     peaks = load_peaks()
     peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
     line = {
