@@ -28,9 +28,14 @@ namespace {
 __device__ uint32_t g_attn_err = 0;
 
 constexpr uint64_t kTimeoutNs = 1000000000ull;  // 1 s per device-side wait
-// Forward block order: pair-major while the K and V of all heads take at most
-// this many bytes (well inside the 126 MB L2, next to Q and O traffic).
-constexpr double kPairMajorMaxKV = 48.0 * 1024 * 1024;
+// Block order: the operands that the CTAs of a chunk of heads stream (K/V in
+// the forward; Q, dO and the dQ accumulator in the backward) may take this many
+// bytes, about half the 126 MB L2.
+constexpr double kOrderChunkBytes = 64.0 * 1024 * 1024;
+int order_chunk(double bytes_per_unit, int units) {
+  const double c = bytes_per_unit > 0 ? kOrderChunkBytes / bytes_per_unit : units;
+  return c >= units ? units : (c < 1.0 ? 1 : int(c));
+}
 constexpr int kMaxDevices = 64;
 
 struct DeviceState {
@@ -283,12 +288,9 @@ attn_status launch_fwd(const DeviceState& st, const void* q, const void* k, cons
   p.total_k = 0;
   p.num_mblocks = (Sq + fwd::NQ * fwd::BM - 1) / (fwd::NQ * fwd::BM);
   p.compact = 0;
-  // Block order: while every head's K and V fit in L2 together, nothing is lost
-  // by running the pairs of many heads at once, and pair-major order starts the
-  // longest causal CTAs of all heads first; larger problems keep the pairs of
-  // one head side by side so that they share its K/V tiles in L2.
-  const double kv_bytes = 2.0 * B * double(Sk) * Hk * D * 2.0;
-  p.pair_major = kv_bytes <= kPairMajorMaxKV ? 1 : 0;
+  // Block order: pair-major within chunks of heads whose K and V fit in L2
+  // together (K/V bytes per query head: a K/V head's, shared by H / Hk heads)
+  p.order_chunk = order_chunk(2.0 * double(Sk) * D * 2.0 * Hk / H, H * B);
   p.err = st.err;
   p.timeout_ns = kTimeoutNs;
   dim3 grid(p.num_mblocks, H, B);
@@ -387,10 +389,10 @@ attn_status launch_bwd_main(const DeviceState& st, const void* q, const void* k,
   p.total_k = 0;
   p.R = 0;
   p.compact = 0;
-  // Block order (as in the forward): tile-major while the operands every CTA
-  // streams (Q, dO, the fp32 dQ accumulator) of all heads fit in L2 together.
-  const double stream_bytes = double(B) * H * double(Sq) * D * (2.0 + 2.0 + 4.0);
-  p.tile_major = stream_bytes <= kPairMajorMaxKV ? 1 : 0;
+  // Block order (as in the forward): tile-major within chunks of K/V heads
+  // whose streamed operands (Q, dO and the fp32 dQ accumulator of the H / Hk
+  // query heads each serves) fit in L2 together.
+  p.order_chunk = order_chunk(double(H / Hk) * double(Sq) * D * (2.0 + 2.0 + 4.0), Hk * B);
   p.Hk = Hk;
   p.scale = scale;
   p.scale_log2 = scale * 1.4426950408889634f;
@@ -591,7 +593,7 @@ attn_status launch_fwd_varlen(const DeviceState& st, const void* q, const void* 
   // (at most ceil(total_q / 256) + B of them); otherwise the longest sequence's
   // pair count for every sequence.
   p.compact = B <= kCompactMaxB ? 1 : 0;
-  p.pair_major = 0;
+  p.order_chunk = 1;
   const int rows = fwd::NQ * fwd::BM;
   dim3 grid = p.compact ? dim3((vl.total_q + rows - 1) / rows + B, H, 1)
                         : dim3(p.num_mblocks, H, B);
@@ -656,7 +658,7 @@ attn_status run_backward_varlen(const DeviceState& st, const void* q, const void
   // ceil(total_k / 128) + B of them); otherwise the longest sequence's tile
   // count for every sequence.
   p.compact = B <= kCompactMaxB ? 1 : 0;
-  p.tile_major = 0;
+  p.order_chunk = 1;
   dim3 grid = p.compact ? dim3((vl.total_k + bwd::BN - 1) / bwd::BN + B, Hk, 1)
                         : dim3((vl.max_k + bwd::BN - 1) / bwd::BN, Hk, B);
   bwd::attn_bwd_main_kernel<D, E, true>

@@ -123,7 +123,7 @@ struct Params {
   const int* cu_k;
   int total_q, total_k, R;
   int compact;  // packed batches: blockIdx.x numbers the key tiles that have work (compact_tile)
-  int tile_major;  // (B, S, H, D) batches: block order tile-major instead of head-major
+  int order_chunk;  // (B, S, H, D) batches: K/V-head-batch combinations per block-order chunk
   int Hk;  // key/value heads: the CTA's K/V head is shared by H / Hk query heads
   float scale;
   float scale_log2;
@@ -406,20 +406,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     return;
   }
 
-  // Grid: (key tile, K/V head, batch).  Head-major order: the key tiles of one
-  // head run side by side, so they share that head's Q and dO tiles in L2; low
-  // key tiles (the most query tiles when causal) start first.  Tile-major order
-  // (problems whose streamed operands fit in L2 all at once): the linear block
-  // index walks key tile 0 of every (head, batch), then tile 1, ..., so the
-  // longest CTAs of all heads start in the first wave.
+  // Grid: (key tile, K/V head, batch), visited in chunked order
+  // (chunked_order): key tile 0 (the most query tiles when causal) of every K/V
+  // head of a chunk whose Q, dO and dQ accumulator fit in L2 together, then
+  // key tile 1, ...
   int kt = blockIdx.x, hk = blockIdx.y, b = blockIdx.z;  // hk: key/value head
-  if (p.tile_major) {
+  if (p.order_chunk > 1) {
     const int lin = int(blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z));
-    const int nbh = p.Hk * p.B;
-    kt = lin / nbh;
-    const int rem = lin - kt * nbh;
-    hk = rem % p.Hk;
-    b = rem / p.Hk;
+    const ChunkedOrder o = chunked_order(lin, int(gridDim.x), p.Hk * p.B, p.order_chunk);
+    kt = o.tile;
+    hk = o.hb % p.Hk;
+    b = o.hb / p.Hk;
   }
   if constexpr (kVarlen) {
     if (p.compact) {

@@ -47,6 +47,36 @@ struct MaskGeom {
   __host__ __device__ int qmax(int j) const { return j - delta + left; }
 };
 
+// Block order of a (tile, head-batch) grid.  The linear block index walks the
+// head-batch combinations in chunks of `chunk`; inside a chunk it takes tile 0
+// of every combination, then tile 1, and so on (tile 0 is the heaviest under a
+// causal mask).  chunk = 1 is head-major order (one head's tiles side by side,
+// sharing its operands in L2); chunk = n_hb is tile-major over the whole grid.
+// A chunk whose operands fit in L2 together keeps that sharing while the
+// heaviest tiles of every head start early, instead of the heaviest tiles of
+// the last heads trailing after everything else.
+struct ChunkedOrder {
+  int tile, hb;
+};
+__device__ __forceinline__ ChunkedOrder chunked_order(int lin, int n_tiles, int n_hb, int chunk) {
+  const int per = n_tiles * chunk;  // blocks of one full chunk
+  const int full = n_hb / chunk;
+  int c, rem, csz;
+  if (lin < full * per) {
+    c = lin / per;
+    rem = lin - c * per;
+    csz = chunk;
+  } else {
+    c = full;
+    rem = lin - full * per;
+    csz = n_hb - full * chunk;
+  }
+  ChunkedOrder o;
+  o.tile = rem / csz;
+  o.hb = c * chunk + rem % csz;
+  return o;
+}
+
 // Device error word code for malformed packed-sequence boundaries.
 constexpr uint32_t kErrSeqlens = 13u;
 

@@ -93,7 +93,7 @@ struct Params {
   int causal, win_left, win_right;
   int num_mblocks;   // ceil(Sq / (NQ * BM))
   int compact;       // packed batches: blockIdx.x numbers the tiles that have work (compact_tile)
-  int pair_major;    // (B, S, H, D) batches: block order pair-major instead of head-major
+  int order_chunk;   // (B, S, H, D) batches: head-batch combinations per block-order chunk
   uint32_t* err;
   uint64_t timeout_ns;
 };
@@ -133,21 +133,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     return;
   }
 
-  // Grid: (query-tile pair, head, batch).  Head-major order: the pairs of one
-  // head run side by side, so they share that head's K/V tiles in L2; causal
-  // launches each head's pairs with the most keys first.  Pair-major order
-  // (problems whose K/V fit in L2 all at once): the linear block index walks
-  // pair 0 of every (head, batch), then pair 1, ..., so under a causal mask the
-  // longest CTAs of all heads start in the first wave instead of trailing
-  // behind the lighter pairs of the heads before them.
+  // Grid: (query-tile pair, head, batch), visited in chunked order
+  // (chunked_order): pair 0 (the heaviest when causal) of every head of a chunk
+  // of heads whose K/V fit in L2 together, then pair 1, ...
   int pr = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-  if (p.pair_major) {
+  if (p.order_chunk > 1) {
     const int lin = int(blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z));
-    const int nbh = p.H * p.B;
-    pr = lin / nbh;
-    const int rem = lin - pr * nbh;
-    h = rem % p.H;
-    b = rem / p.H;
+    const ChunkedOrder o = chunked_order(lin, p.num_mblocks, p.H * p.B, p.order_chunk);
+    pr = o.tile;
+    h = o.hb % p.H;
+    b = o.hb / p.H;
   }
   int mb = p.causal ? (p.num_mblocks - 1 - pr) : pr;
   const int hk = h / (p.H / p.Hk);  // the key/value head this query head reads
