@@ -323,6 +323,7 @@ attn_status launch_fwd_d256(const DeviceState& st, const void* q, const void* k,
   p.win_left = win_left;
   p.win_right = win_right;
   p.num_mblocks = (Sq + fwd256::BM - 1) / fwd256::BM;
+  p.order_chunk = order_chunk(2.0 * double(Sk) * 256 * 2.0 * Hk / H, H * B);
   p.err = st.err;
   p.timeout_ns = kTimeoutNs;
   fwd256::attn_fwd_d256_kernel<E><<<dim3(p.num_mblocks, H, B), fwd256::kThreads,
@@ -439,6 +440,8 @@ attn_status launch_bwd_main_d256(const DeviceState& st, const void* q, const voi
   p.Sq_pad = w.Sq_pad;
   p.n_ktiles = (Sk + bwd256::BR - 1) / bwd256::BR;
   p.n_qtiles = (Sq + bwd256::BR - 1) / bwd256::BR;
+  // chunked block order over the heads (Q, dO and the float32 dQ rows of a head)
+  p.order_chunk = order_chunk(double(Sq) * 256 * (2.0 + 2.0 + 4.0), H * B);
   p.scale = scale;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.causal = causal ? 1 : 0;
@@ -593,7 +596,9 @@ attn_status launch_fwd_varlen(const DeviceState& st, const void* q, const void* 
   // (at most ceil(total_q / 256) + B of them); otherwise the longest sequence's
   // pair count for every sequence.
   p.compact = B <= kCompactMaxB ? 1 : 0;
-  p.order_chunk = 1;
+  // chunked block order over the heads (a head's K/V: every sequence's rows)
+  p.order_chunk = order_chunk(2.0 * double(vl.total_k) * D * 2.0 * Hk / H,
+                              p.compact ? H : H * B);
   const int rows = fwd::NQ * fwd::BM;
   dim3 grid = p.compact ? dim3((vl.total_q + rows - 1) / rows + B, H, 1)
                         : dim3(p.num_mblocks, H, B);
@@ -658,7 +663,10 @@ attn_status run_backward_varlen(const DeviceState& st, const void* q, const void
   // ceil(total_k / 128) + B of them); otherwise the longest sequence's tile
   // count for every sequence.
   p.compact = B <= kCompactMaxB ? 1 : 0;
-  p.order_chunk = 1;
+  // chunked block order over the K/V heads (Q, dO and the dQ accumulator of the
+  // query heads each serves, every sequence's rows)
+  p.order_chunk = order_chunk(double(H / Hk) * double(vl.total_q) * D * (2.0 + 2.0 + 4.0),
+                              p.compact ? Hk : Hk * B);
   dim3 grid = p.compact ? dim3((vl.total_k + bwd::BN - 1) / bwd::BN + B, Hk, 1)
                         : dim3((vl.max_k + bwd::BN - 1) / bwd::BN, Hk, B);
   bwd::attn_bwd_main_kernel<D, E, true>

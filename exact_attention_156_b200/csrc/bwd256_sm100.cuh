@@ -105,6 +105,7 @@ struct Params {
   const float* ndelta;  // [B*H][Sq_pad] -Delta
   int B, H, Hk, Sq, Sk, Sq_pad;
   int n_ktiles, n_qtiles;  // ceil(Sk / 128), ceil(Sq / 128)
+  int order_chunk;         // head-batch combinations per block-order chunk (chunked_order)
   float scale;
   float scale_log2;
   int causal, win_left, win_right;
@@ -139,24 +140,38 @@ __global__ void __launch_bounds__(kThreads, 1)
     return;
   }
 
-  // blockIdx.x: [0, 2 n_ktiles) key tiles (dK, dV interleaved, low keys first:
-  // with a causal mask they see the most queries), then the query tiles for dQ
-  // (with a causal mask the most keys first).  blockIdx.y: the query head (dQ)
-  // or key/value head (dK, dV; CTAs with y >= Hk have nothing to do).
-  const int bx = blockIdx.x;
+  // Block index x (per head): in threes, the dK and dV tiles of key tile l and
+  // the dQ tile of the l-th heaviest query tile (with a causal mask low key
+  // tiles see the most queries and high query tiles the most keys), then the
+  // remaining tiles of the longer axis.  y: the query head (dQ) or key/value
+  // head (dK, dV; CTAs with y >= Hk have nothing to do).  The (x, head) pairs
+  // are visited in chunked order over the heads (chunked_order).
+  int bx = blockIdx.x, hy = blockIdx.y, b = blockIdx.z;  // hy: dQ query head, dK/dV K/V head
+  if (p.order_chunk > 1) {
+    const int lin = int(blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z));
+    const ChunkedOrder o =
+        chunked_order(lin, int(gridDim.x), int(gridDim.y * gridDim.z), p.order_chunk);
+    bx = o.tile;
+    hy = o.hb % int(gridDim.y);
+    b = o.hb / int(gridDim.y);
+  }
+  const int nmin = min(p.n_ktiles, p.n_qtiles);
   int mode, tile;
-  if (bx < 2 * p.n_ktiles) {
-    mode = bx & 1 ? kModeDV : kModeDK;
-    tile = bx >> 1;
+  if (bx < 3 * nmin) {
+    const int l = bx / 3, m = bx % 3;
+    mode = m == 0 ? kModeDK : (m == 1 ? kModeDV : kModeDQ);
+    tile = (m == 2 && p.causal) ? p.n_qtiles - 1 - l : l;
+  } else if (p.n_ktiles > nmin) {
+    const int r = bx - 3 * nmin;
+    mode = r & 1 ? kModeDV : kModeDK;
+    tile = nmin + (r >> 1);
   } else {
     mode = kModeDQ;
-    tile = bx - 2 * p.n_ktiles;
-    if (p.causal) tile = p.n_qtiles - 1 - tile;
+    const int q = nmin + (bx - 3 * nmin);
+    tile = p.causal ? p.n_qtiles - 1 - q : q;
   }
-  const int b = blockIdx.z;
   const int group = p.H / p.Hk;
-  if (mode != kModeDQ && int(blockIdx.y) >= p.Hk) return;
-  const int hy = blockIdx.y;  // dQ: query head; dK / dV: key/value head
+  if (mode != kModeDQ && hy >= p.Hk) return;
   const MaskGeom g = MaskGeom::make(p.Sq, p.Sk, p.causal, p.win_left, p.win_right);
   const int r0 = tile * BR;   // first accumulator row (key, or query in dQ mode)
   const int r1 = mode == kModeDQ ? min(r0 + BR - 1, p.Sq - 1) : min(r0 + BR - 1, p.Sk - 1);

@@ -413,17 +413,19 @@ __global__ void __launch_bounds__(kThreads, 1)
   int kt = blockIdx.x, hk = blockIdx.y, b = blockIdx.z;  // hk: key/value head
   if (p.order_chunk > 1) {
     const int lin = int(blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z));
-    const ChunkedOrder o = chunked_order(lin, int(gridDim.x), p.Hk * p.B, p.order_chunk);
+    const ChunkedOrder o =
+        chunked_order(lin, int(gridDim.x), int(gridDim.y * gridDim.z), p.order_chunk);
     kt = o.tile;
-    hk = o.hb % p.Hk;
-    b = o.hb / p.Hk;
+    hk = o.hb % int(gridDim.y);
+    b = o.hb / int(gridDim.y);
   }
+  const int cidx = kt;  // compact grids: the tile's index in the compact numbering
   if constexpr (kVarlen) {
     if (p.compact) {
       // one CTA per key tile that has work, low key tiles (the heaviest when
       // causal) first
       b = compact_tile(p.cu_q, p.cu_k, p.B, p.total_q, p.total_k, p.Sq, p.Sk, true, BN,
-                       int(blockIdx.x), kt);
+                       cidx, kt);
       if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x < 32)
         compact_check(p.cu_q, p.cu_k, p.B, p.total_q, p.total_k, p.Sq, p.Sk, true, BN,
                       (long long)gridDim.x, p.err);

@@ -91,6 +91,7 @@ struct Params {
   float scale_log2;
   int causal, win_left, win_right;
   int num_mblocks;  // ceil(Sq / 128)
+  int order_chunk;  // head-batch combinations per block-order chunk (chunked_order)
   uint32_t* err;
   uint64_t timeout_ns;
 };
@@ -114,11 +115,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     return;
   }
 
-  // causal launches the query tiles with the most keys first
-  const int mb = p.causal ? (p.num_mblocks - 1 - int(blockIdx.x)) : int(blockIdx.x);
-  const int h = blockIdx.y;
+  // causal launches the query tiles with the most keys first, in chunked
+  // order over the heads (chunked_order)
+  int x = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  if (p.order_chunk > 1) {
+    const int lin = int(blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z));
+    const ChunkedOrder o =
+        chunked_order(lin, int(gridDim.x), int(gridDim.y * gridDim.z), p.order_chunk);
+    x = o.tile;
+    h = o.hb % int(gridDim.y);
+    b = o.hb / int(gridDim.y);
+  }
+  const int mb = p.causal ? (p.num_mblocks - 1 - x) : x;
   const int hk = h / (p.H / p.Hk);
-  const int b = blockIdx.z;
   const MaskGeom g = MaskGeom::make(p.Sq, p.Sk, p.causal, p.win_left, p.win_right);
   const int r0 = mb * BM;
   const int r1 = min(r0 + BM - 1, p.Sq - 1);

@@ -139,10 +139,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   int pr = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   if (p.order_chunk > 1) {
     const int lin = int(blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z));
-    const ChunkedOrder o = chunked_order(lin, p.num_mblocks, p.H * p.B, p.order_chunk);
+    const ChunkedOrder o =
+        chunked_order(lin, int(gridDim.x), int(gridDim.y * gridDim.z), p.order_chunk);
     pr = o.tile;
-    h = o.hb % p.H;
-    b = o.hb / p.H;
+    h = o.hb % int(gridDim.y);
+    b = o.hb / int(gridDim.y);
   }
   int mb = p.causal ? (p.num_mblocks - 1 - pr) : pr;
   const int hk = h / (p.H / p.Hk);  // the key/value head this query head reads
@@ -151,7 +152,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // one CTA per query-tile pair that has work, the heaviest pairs first
       int tile = 0;
       b = compact_tile(p.cu_q, p.cu_k, p.B, p.total_q, p.total_k, p.Sq, p.Sk, false, NQ * BM,
-                       int(blockIdx.x), tile);
+                       pr, tile);
       if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x < 32)
         compact_check(p.cu_q, p.cu_k, p.B, p.total_q, p.total_k, p.Sq, p.Sk, false, NQ * BM,
                       (long long)gridDim.x, p.err);
