@@ -66,6 +66,34 @@ constexpr int kLoad2Warp = 10;
 constexpr int kComputeThreads = 256;  // two groups: columns [0,32) and [32,64) of a step
 constexpr int kModeDK = 0, kModeDV = 1, kModeDQ = 2;
 
+// The gradient (mode) and tile of block index x of one head, for n_k key tiles
+// and n_q query tiles: in threes, the dK and dV tiles of key tile l and the dQ
+// tile of the l-th heaviest query tile (with a causal mask low key tiles see
+// the most queries and high query tiles the most keys), then the remaining
+// tiles of the longer axis, dK and dV alternating.  The 2 n_k + n_q indices
+// name every (mode, tile) once.
+struct D256Work {
+  int mode, tile;
+};
+__host__ __device__ __forceinline__ D256Work d256_work(int bx, int n_k, int n_q, int causal) {
+  const int nmin = n_k < n_q ? n_k : n_q;
+  D256Work w;
+  if (bx < 3 * nmin) {
+    const int l = bx / 3, m = bx % 3;
+    w.mode = m == 0 ? kModeDK : (m == 1 ? kModeDV : kModeDQ);
+    w.tile = (m == 2 && causal) ? n_q - 1 - l : l;
+  } else if (n_k > nmin) {
+    const int r = bx - 3 * nmin;
+    w.mode = r & 1 ? kModeDV : kModeDK;
+    w.tile = nmin + (r >> 1);
+  } else {
+    w.mode = kModeDQ;
+    const int q = nmin + (bx - 3 * nmin);
+    w.tile = causal ? n_q - 1 - q : q;
+  }
+  return w;
+}
+
 struct Cfg {
   static constexpr int kRBox = BR * 128;        // 128 rows x 64 columns (16 KB)
   static constexpr int kRBytes = 4 * kRBox;     // a resident 128 x 256 tile (64 KB)
@@ -140,12 +168,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     return;
   }
 
-  // Block index x (per head): in threes, the dK and dV tiles of key tile l and
-  // the dQ tile of the l-th heaviest query tile (with a causal mask low key
-  // tiles see the most queries and high query tiles the most keys), then the
-  // remaining tiles of the longer axis.  y: the query head (dQ) or key/value
-  // head (dK, dV; CTAs with y >= Hk have nothing to do).  The (x, head) pairs
-  // are visited in chunked order over the heads (chunked_order).
+  // Block index x (per head): the gradient and tile of d256_work.  y: the
+  // query head (dQ) or key/value head (dK, dV; CTAs with y >= Hk have nothing
+  // to do).  The (x, head) pairs are visited in chunked order over the heads
+  // (chunked_order).
   int bx = blockIdx.x, hy = blockIdx.y, b = blockIdx.z;  // hy: dQ query head, dK/dV K/V head
   if (p.order_chunk > 1) {
     const int lin = int(blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z));
@@ -155,21 +181,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     hy = o.hb % int(gridDim.y);
     b = o.hb / int(gridDim.y);
   }
-  const int nmin = min(p.n_ktiles, p.n_qtiles);
-  int mode, tile;
-  if (bx < 3 * nmin) {
-    const int l = bx / 3, m = bx % 3;
-    mode = m == 0 ? kModeDK : (m == 1 ? kModeDV : kModeDQ);
-    tile = (m == 2 && p.causal) ? p.n_qtiles - 1 - l : l;
-  } else if (p.n_ktiles > nmin) {
-    const int r = bx - 3 * nmin;
-    mode = r & 1 ? kModeDV : kModeDK;
-    tile = nmin + (r >> 1);
-  } else {
-    mode = kModeDQ;
-    const int q = nmin + (bx - 3 * nmin);
-    tile = p.causal ? p.n_qtiles - 1 - q : q;
-  }
+  const D256Work work = d256_work(bx, p.n_ktiles, p.n_qtiles, p.causal);
+  const int mode = work.mode, tile = work.tile;
   const int group = p.H / p.Hk;
   if (mode != kModeDQ && hy >= p.Hk) return;
   const MaskGeom g = MaskGeom::make(p.Sq, p.Sk, p.causal, p.win_left, p.win_right);

@@ -372,7 +372,7 @@ __global__ void __launch_bounds__(256) attn_bwd_dq_varlen_kernel(
 // 2. main backward kernel
 // ---------------------------------------------------------------------------
 // Query-tile range [qlo, qhi) that can see keys [n0, n1]; empty if qhi <= qlo.
-__device__ __forceinline__ void qtile_range(const MaskGeom& g, int n0, int n1, int& qlo, int& qhi) {
+__host__ __device__ __forceinline__ void qtile_range(const MaskGeom& g, int n0, int n1, int& qlo, int& qhi) {
   const int a = max(0, g.qmin(n0));
   const int z = min(g.Sq - 1, g.qmax(n1));
   if (n0 >= g.Sk || z < a) {

@@ -58,7 +58,7 @@ struct MaskGeom {
 struct ChunkedOrder {
   int tile, hb;
 };
-__device__ __forceinline__ ChunkedOrder chunked_order(int lin, int n_tiles, int n_hb, int chunk) {
+__host__ __device__ __forceinline__ ChunkedOrder chunked_order(int lin, int n_tiles, int n_hb, int chunk) {
   const int per = n_tiles * chunk;  // blocks of one full chunk
   const int full = n_hb / chunk;
   int c, rem, csz;

@@ -19,11 +19,21 @@
 //   attn_diag_tma: a TMA load of a (1, 128, 1, 128) bf16 tensor with the
 //     same 4-D map and 128-byte swizzle as the kernels; the raw shared-memory
 //     bytes are copied out so the test can check the placement.
+//   attn_diag_mask_bounds, attn_diag_fwd_tile_ranges, attn_diag_bwd_qtile_ranges,
+//   attn_diag_chunked_order, attn_diag_d256_work: host-only views of the index
+//     arithmetic the kernels pick their work with (mask bounds per row and per
+//     key, the key-tile range of a query tile and the query-tile range of a key
+//     tile, the block order, the head_dim 256 backward's gradient per block);
+//     they launch nothing, so the CPU tests check them exhaustively.
 // Not part of the product library.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "bwd256_sm100.cuh"
+#include "bwd_sm100.cuh"
+#include "common.cuh"
+#include "fwd_sm100.cuh"
 #include "ptx.cuh"
 #include "ptx_pair.cuh"
 
@@ -399,6 +409,88 @@ __attribute__((visibility("default"))) int attn_diag_error(void) {
   const uint32_t z = 0;
   cudaMemcpyToSymbol(g_diag_err, &z, sizeof(z));
   return int(w);
+}
+
+// Mask bounds of every query row (lo, hi: keys lo..hi visible, none if hi < lo)
+// and of every key (qmin, qmax: the rows that see it, before clipping to
+// [0, Sq)), as the kernels compute them.
+__attribute__((visibility("default"))) int attn_diag_mask_bounds(int Sq, int Sk, int causal,
+                                                                 int win_left, int win_right,
+                                                                 int* lo, int* hi, int* qmin,
+                                                                 int* qmax) {
+  if (Sq < 0 || Sk < 0 || !lo || !hi || !qmin || !qmax) return 1;
+  const MaskGeom g = MaskGeom::make(Sq, Sk, causal, win_left, win_right);
+  for (int i = 0; i < Sq; ++i) {
+    lo[i] = g.lo(i);
+    hi[i] = g.hi(i);
+  }
+  for (int j = 0; j < Sk; ++j) {
+    qmin[j] = g.qmin(j);
+    qmax[j] = g.qmax(j);
+  }
+  return 0;
+}
+
+// Key-tile range [jlo, jhi) the forward visits for query tiles 0..n_tiles-1
+// (rows r0 = t * BM .. min(r0 + BM - 1, Sq - 1)); *bm, *bn: its tile sizes.
+__attribute__((visibility("default"))) int attn_diag_fwd_tile_ranges(int Sq, int Sk, int causal,
+                                                                     int win_left, int win_right,
+                                                                     int n_tiles, int* jlo,
+                                                                     int* jhi, int* bm, int* bn) {
+  if (Sq < 0 || Sk < 0 || n_tiles < 0 || !jlo || !jhi || !bm || !bn) return 1;
+  const MaskGeom g = MaskGeom::make(Sq, Sk, causal, win_left, win_right);
+  for (int t = 0; t < n_tiles; ++t) {
+    const int r0 = t * fwd::BM;
+    const int r1 = r0 + fwd::BM - 1 < Sq - 1 ? r0 + fwd::BM - 1 : Sq - 1;
+    fwd::tile_range(g, r0, r1, jlo[t], jhi[t]);
+  }
+  *bm = fwd::BM;
+  *bn = fwd::BN;
+  return 0;
+}
+
+// Query-tile range [qlo, qhi) the backward visits for key tiles 0..n_tiles-1
+// (keys n0 = t * BN .. min(n0 + BN - 1, Sk - 1)); *bm, *bn: its tile sizes.
+__attribute__((visibility("default"))) int attn_diag_bwd_qtile_ranges(int Sq, int Sk, int causal,
+                                                                      int win_left, int win_right,
+                                                                      int n_tiles, int* qlo,
+                                                                      int* qhi, int* bm, int* bn) {
+  if (Sq < 0 || Sk < 0 || n_tiles < 0 || !qlo || !qhi || !bm || !bn) return 1;
+  const MaskGeom g = MaskGeom::make(Sq, Sk, causal, win_left, win_right);
+  for (int t = 0; t < n_tiles; ++t) {
+    const int n0 = t * bwd::BN;
+    const int n1 = n0 + bwd::BN - 1 < Sk - 1 ? n0 + bwd::BN - 1 : Sk - 1;
+    bwd::qtile_range(g, n0, n1, qlo[t], qhi[t]);
+  }
+  *bm = bwd::BM;
+  *bn = bwd::BN;
+  return 0;
+}
+
+// (tile, head-batch) of every linear block index of an n_tiles x n_hb grid
+// visited in chunked order.
+__attribute__((visibility("default"))) int attn_diag_chunked_order(int n_tiles, int n_hb,
+                                                                   int chunk, int* tile, int* hb) {
+  if (n_tiles < 0 || n_hb < 0 || chunk < 1 || !tile || !hb) return 1;
+  for (int lin = 0; lin < n_tiles * n_hb; ++lin) {
+    const ChunkedOrder o = chunked_order(lin, n_tiles, n_hb, chunk);
+    tile[lin] = o.tile;
+    hb[lin] = o.hb;
+  }
+  return 0;
+}
+
+// (mode, tile) of every block index x of the head_dim 256 backward's grid
+// (2 n_k + n_q per head); mode 0 dK, 1 dV, 2 dQ.
+__attribute__((visibility("default"))) int attn_diag_d256_work(int n_k, int n_q, int causal,
+                                                               int* mode, int* tile) {
+  if (n_k < 0 || n_q < 0 || !mode || !tile) return 1;
+  for (int x = 0; x < 2 * n_k + n_q; ++x) {
+    const bwd256::D256Work w = bwd256::d256_work(x, n_k, n_q, causal);
+    mode[x] = w.mode;
+    tile[x] = w.tile;
+  }
+  return 0;
 }
 
 }  // extern "C"

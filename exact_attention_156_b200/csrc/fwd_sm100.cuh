@@ -99,7 +99,7 @@ struct Params {
 };
 
 // Key-tile range [jlo, jhi) for query rows [r0, r1]; empty if jhi <= jlo.
-__device__ __forceinline__ void tile_range(const MaskGeom& g, int r0, int r1, int& jlo, int& jhi) {
+__host__ __device__ __forceinline__ void tile_range(const MaskGeom& g, int r0, int r1, int& jlo, int& jhi) {
   const int klo = g.lo(r0);
   const int khi = g.hi(r1);
   if (r0 >= g.Sq || khi < klo || khi < 0) {
