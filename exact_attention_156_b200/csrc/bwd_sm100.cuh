@@ -2,8 +2,8 @@
 //
 // Method: the backward rebuilds the attention probabilities from Q, K and the
 // forward's per-row log-sum-exp instead of storing them (flash-attn install
-// guide, yfxerp.com, section 1: "the backward recomputes the attention
-// scores"; FlashAttention-2 overview, lshu.cn, section 2.1, second anti-pattern:
+// guide, yfxerp.com, section 1, on the backward recomputing the attention
+// scores; FlashAttention-2 overview, lshu.cn, section 2.1, second anti-pattern:
 // the standard backward re-reads Q, K, V several times).  The gradient is the
 // analytic one of O = softmax(scale Q K^T) V:
 //   P = exp(scale S - LSE), dV = P^T dO, dP = dO V^T, Delta_i = rowsum(dO*O),

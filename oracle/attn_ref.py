@@ -6,8 +6,8 @@ module.  It shares no code with the CUDA path.
 
 What it computes.  The pages call the method exact (FlashAttention-2
 overview, lshu.cn, section 1; flash-attn install guide, yfxerp.com,
-section 1: "IO-aware exact attention"), so the oracle is the plain
-definition, the "standard attention" of the FlashAttention-2 overview,
+section 1, which describes it as exact and IO-aware), so the oracle is
+the plain definition, the standard attention of the FlashAttention-2 overview,
 section 2.1 (first anti-pattern): scores S = Q K^T, a row-wise softmax with
 the row maximum subtracted first (section 2.1, third anti-pattern, on
 stability), then the weighted sum of V.  Everything runs in float64 on the
@@ -17,7 +17,7 @@ Readings of points the pages leave open:
   * scale multiplies the scores: S = scale * Q K^T.  ``softmax_scale=None``
     in the pages' ``flash_attn_func`` call (section 3.3 snippet) means
     1/sqrt(head_dim); callers here always pass it explicitly.
-  * causal ("upper-triangular mask", section 4.2 problem 4) is aligned to the
+  * causal (an upper-triangular mask, section 4.2 problem 4) is aligned to the
     bottom-right corner: key j is visible to query i iff j <= i + (Sk - Sq).
   * window (``window_size`` is only named on the yfxerp.com page, section 1):
     with delta = Sk - Sq, key j is visible to query i iff
