@@ -7,7 +7,7 @@ tensors of that layout: "flash-attn install guide for CUDA 12.8 + PyTorch
 2.7" (yfxerp.com), section 3.3; "RTX 5060 flash-attention" (pptc.cn),
 section 4.4).  Some workloads scale the draws by 0.5.
 
-Recipe (fixed here, the pages only say "random"):
+Recipe (fixed here; the pages only say the inputs are random):
   * generator: numpy ``Generator(PCG64(seed))``;
   * draw order: Q, K, V, dO, each ``standard_normal`` in float32 of shape
     (B, S, H, D) (K and V with Hk heads when the key/value heads are
